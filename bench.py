@@ -1,0 +1,344 @@
+#!/usr/bin/env python
+"""Throughput of exact minimax FP16 group-scale selection (W4, group 128).
+
+One step = one call of the C ABI over the whole 0.8B-scale sweep workload
+(30,336 x 16,384 fp16 weights = 3,883,008 groups, E=4 per-column diagonals),
+inputs already resident in HBM.  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cq|reference]
+
+N > 1 runs under torch.distributed (one process per GPU, NCCL used only for
+the barrier and the max-over-ranks time): every rank solves its own matrix of
+the same workload, so per-GPU work is fixed (weak scaling).
+The reference arm (--impl reference) times the exhaustive CPU oracle on the
+host cores over bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "groups/sec (and % of binding roofline) for W4/G128 minimax scale selection"
+WORKLOAD = 3
+SMS, FP32_LANES, FP64_LANES = 148, 128, 64
+
+
+def flop_run(E: int) -> int:
+    """Counted FP32 flops per constant-code run: transition update 4E, vertices
+    E, pairwise roots 12 E(E-1)/2, and a closed-form max over E environments
+    (2 FMA + 1 max each) at the two run ends, E vertices, E(E-1) roots and two
+    grid neighbours."""
+    return 4 * E + E + 12 * E * (E - 1) // 2 + (E * E + 4) * (5 * E - 1)
+
+
+def counted_flops(Wg: np.ndarray, E: int):
+    """(fp32 flops, fp64 flops) of the method's candidate work for these groups:
+    per non-trivial group (T_g + 1) runs with T_g = 7 #(w>0) + 8 #(w<0), plus
+    fp64 rescoring of two finalists (2 * 128 * E * 5)."""
+    nz = (Wg & 0x7FFF) != 0
+    neg = nz & ((Wg & 0x8000) != 0)
+    T = 7 * nz.sum(axis=1, dtype=np.int64) + neg.sum(axis=1, dtype=np.int64)
+    live = nz.any(axis=1)
+    f32 = int(((T + 1) * live).sum()) * flop_run(E)
+    f64 = int(live.sum()) * 2 * 128 * E * 5
+    return f32, f64
+
+
+def peaks():
+    """(fp32 TFLOP/s, fp64 TFLOP/s, clock MHz, source) from unit counts and the max SM clock."""
+    mhz, src = 1965.0, "recipe clocks.max.sm 1965 MHz"
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            mp = json.load(f)
+        if mp.get("sm_max_mhz"):
+            mhz, src = float(mp["sm_max_mhz"]), "MEASURED_PEAKS.json sm_max_mhz"
+    except OSError:
+        pass
+    p32 = SMS * FP32_LANES * 2 * mhz * 1e6 / 1e12
+    p64 = SMS * FP64_LANES * 2 * mhz * 1e6 / 1e12
+    return p32, p64, mhz, f"148 SMs x {FP32_LANES} FP32 / {FP64_LANES} FP64 lanes x 2 x {mhz:.0f} MHz ({src})"
+
+
+def kernel_source_hash() -> str:
+    p = os.path.join(ROOT, "minimax_scale_search_b200", "csrc", "cq_select.cu")
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+def recorded_traffic(groups: int):
+    """DRAM bytes per launch of the main kernel from the committed ncu summary,
+    scaled to `groups`; None when the kernel changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "select_kernel_traffic.txt")
+    try:
+        kv = dict(tok.split("=", 1) for tok in open(path).read().split() if "=" in tok)
+    except OSError:
+        return None
+    if kv.get("kernel_sha") != kernel_source_hash():
+        return None
+    return float(kv["dram_bytes"]) / float(kv["groups"]) * groups
+
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of SM clock and throttle reasons."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str):
+        self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
+                                          "-i", gpu_index, "-lms", "200"], stdout=self.tmp,
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self, t0: float, t1: float):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.tmp.flush()
+        rows = []
+        for ln in open(self.tmp.name).read().splitlines():
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                ts += float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                rows.append((ts, float(parts[1].split()[0]), float(parts[2].split()[0]), parts[4:]))
+            except (ValueError, IndexError):
+                continue
+        os.unlink(self.tmp.name)
+        inside = [r for r in rows if t0 - 0.25 <= r[0] <= t1 + 0.25] or rows
+        if not inside:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in inside for n, v in zip(names, r[3][1:]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": reasons, "samples": len(inside)}
+
+
+def gpu_index_for(local_rank: int) -> str:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+def oracle_rate(Wg, D, K, groups_target_s: float, seed: int = 5):
+    """Time the oracle, as it stands, on a bounded sample; returns (groups/s, n, seconds, threads)."""
+    import oracle
+    threads = os.cpu_count() or 1
+    rng = np.random.default_rng(seed)
+    probe = rng.choice(Wg.shape[0], size=min(Wg.shape[0], 2 * threads), replace=False)
+    t0 = time.perf_counter()
+    oracle.solve(Wg, D, K=K, sel=np.sort(probe), threads=threads)
+    per = (time.perf_counter() - t0) / len(probe)
+    n = int(max(len(probe), min(Wg.shape[0], groups_target_s / max(per, 1e-6))))
+    sel = np.sort(rng.choice(Wg.shape[0], size=n, replace=False))
+    t0 = time.perf_counter()
+    oracle.solve(Wg, D, K=K, sel=sel, threads=threads)
+    dt = time.perf_counter() - t0
+    return n / dt, n, dt, threads
+
+
+def run_reference(args, wl):
+    """The oracle arm: each step solves a bounded sample on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from minimax_scale_search_b200 import synth
+    import oracle
+    W = synth.make_weights(WORKLOAD, 0, 512)  # 65,536 groups drawn like the full workload
+    D = synth.make_diagonals(WORKLOAD)
+    Wg = W.reshape(-1, 128)
+    threads = os.cpu_count() or 1
+    per_step_s = max(1.0, 150.0 / (args.steps + args.warmup))
+    _, n_probe, dt_probe, _ = oracle_rate(Wg, D, wl.cols, 2.0)
+    n = max(threads, int(n_probe / dt_probe * per_step_s))
+    n = min(n, Wg.shape[0])
+    rng = np.random.default_rng(17)
+    times = []
+    for s in range(args.warmup + args.steps):
+        sel = np.sort(rng.choice(Wg.shape[0], size=n, replace=False))
+        t0 = time.perf_counter()
+        oracle.solve(Wg, D, K=wl.cols, sel=sel, threads=threads)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            times.append(dt)
+    tot = sum(times)
+    value = n * len(times) / tot
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "groups/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "groups_per_step": n, "E": wl.E, "K": wl.cols},
+            "cpu_baseline": {"value": value, "unit": "groups/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{n} groups per step drawn from rows 0-511 (65,536 groups) of the "
+                                       f"{wl.name} workload, exhaustive fp64 over 31,743 scales"},
+            "e2e": {"value": value, "unit": "groups/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="cq", choices=["cq", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    from minimax_scale_search_b200 import synth
+    wl = synth.workload(WORKLOAD)
+    if args.impl == "reference":
+        run_reference(args, wl)
+        return
+
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    from minimax_scale_search_b200 import cq
+    W = synth.make_weights(WORKLOAD, matrix=rank)
+    D = synth.make_diagonals(WORKLOAD, matrix=rank)
+    Wg = W.reshape(-1, 128)
+    G = Wg.shape[0]
+    f32, f64 = counted_flops(Wg, wl.E)
+    Wd = torch.from_numpy(W.view(np.int16)).to(dev)
+    Dd = torch.from_numpy(D).to(dev)
+    out_s = torch.empty(G, dtype=torch.int16, device=dev)
+    out_c = torch.empty((G, 16), dtype=torch.int32, device=dev)
+    ws = torch.empty(cq.workspace_bytes(G, wl.E), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        return cq.select_scales(Wd, Dd, wl.cols, out_scales=out_s, out_codes=out_c, workspace=ws,
+                                main_events=evs)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    counters = cq.read_counters(ws)
+
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(gpu_index_for(local))
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    w0 = time.time()
+    t_start.record(stream)
+    for k in range(args.steps):
+        step(kev[k])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    w1 = time.time()
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop(w0, w1)
+    ms_total = t_start.elapsed_time(t_end)
+    kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+    if dist:
+        t = torch.tensor([ms_total, kernel_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total, kernel_ms = float(t[0]), float(t[1])
+    ms_step = ms_total / args.steps
+    value = world * G / (ms_step / 1e3)
+
+    # ---- end to end through the host-buffer entry point (pinned host memory)
+    e2e = None
+    if not args.no_e2e:
+        Wp = torch.from_numpy(W.view(np.int16)).pin_memory()
+        Dp = torch.from_numpy(D).pin_memory()
+        sp = torch.empty(G, dtype=torch.int16).pin_memory()
+        cp = torch.empty((G, 16), dtype=torch.int32).pin_memory()
+        Wn, Dn, sn, cn = Wp.numpy(), Dp.numpy(), sp.numpy().view(np.uint16), cp.numpy().view(np.uint32)
+        for _ in range(2):
+            cq.select_scales_host(Wn, Dn, out_scales=sn, out_codes=cn)
+        n_e2e = max(3, min(args.steps, 10))
+        if dist:
+            dist.barrier()
+        t0 = time.perf_counter()
+        for _ in range(n_e2e):
+            cq.select_scales_host(Wn, Dn, out_scales=sn, out_codes=cn)
+        e2e_s = (time.perf_counter() - t0) / n_e2e
+        if dist:
+            t = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_s = float(t[0])
+        dev_s = out_s.cpu().numpy().view(np.uint16)
+        assert np.array_equal(dev_s, sn), "host entry point disagrees with the device entry point"
+        e2e = {"value": world * G / e2e_s, "unit": "groups/s", "h2d_bytes_per_step": int(W.nbytes + D.nbytes),
+               "d2h_bytes_per_step": int(sn.nbytes + cn.nbytes), "ms_per_step": 1e3 * e2e_s, "steps": n_e2e}
+
+    p32, p64, mhz, psrc = peaks()
+    t_roof = f32 / (p32 * 1e12) + f64 / (p64 * 1e12)
+    achieved = (f32 + f64 * p32 / p64) / (kernel_ms / 1e3) / 1e12
+    traffic = recorded_traffic(G)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, n, dt, threads = oracle_rate(Wg, D, wl.cols, 12.0)
+        cpu = {"value": rate, "unit": "groups/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n} groups sampled from the {wl.name} workload (rank 0's matrix), exhaustive "
+                         f"fp64 over 31,743 scales, {dt:.1f} s"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "groups/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": wl.name, "groups_per_gpu": G, "weights_per_gpu": G * 128, "E": wl.E,
+                           "K": wl.cols, "diagonals": "per-column [4, 16384] fp32",
+                           "l2": "inputs (994 MB of W per GPU) larger than the 126 MB L2; no flush"},
+                "weights_per_s": value * 128,
+                "roofline": {"bound": "alu", "achieved": achieved, "peak": p32, "unit": "TFLOP/s",
+                             "frac": achieved / p32, "traffic": traffic,
+                             "kernel": f"select_kernel<{wl.E}>", "kernel_ms": kernel_ms,
+                             "roofline_ms": 1e3 * t_roof, "fp32_flops": f32, "fp64_flops": f64,
+                             "peak_note": f"fp32-equivalent (fp64 flops weighted x{p32 / p64:.0f}); {psrc}"},
+                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps,
+                "clocks": clocks, "counters": counters}
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

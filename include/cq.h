@@ -1,0 +1,144 @@
+/*
+ * cq.h — C ABI of libcq.so: exact minimax FP16 group-scale selection for
+ * symmetric W4 quantisation with group size 128, on NVIDIA B200 (sm_100a).
+ *
+ * The operation (CliffQuant project page, "What CliffQuant changes"): for each
+ * group of 128 weights w_i and E environment diagonals d_{e,i} >= 0, choose the
+ * positive finite IEEE binary16 scale s minimising
+ *
+ *     f(s) = max_e  sum_i d_{e,i} * (w_i - s * q_i(s))^2,
+ *     q_i(s) = clip(round-half-even(w_i / s), -8, 7),
+ *
+ * over all 31,743 such scales, an exact objective tie going to the lower FP16
+ * bit pattern, and emit the 4-bit codes.  The codes are packed as (q + 8)
+ * nibbles, 8 per uint32, low nibble first: word j of a group holds codes
+ * 8j .. 8j+7.  The quantiser is QuantizerSpec(qmin=-8, qmax=7) of the page's
+ * "Use the solver" example.  The candidate scales the page's solver outline
+ * names (code transitions, quadratic vertices, environment intersections) are
+ * realised here as a search over the runs of constant codes between code
+ * transitions; the exhaustive enumeration of all 31,743 values is the
+ * fallback when a group's screen cannot certify its answer.
+ *
+ * Conventions for every entry point:
+ *  - All pointers named W, D, out_* and workspace are DEVICE pointers on the
+ *    current CUDA device, except where a name ends in _host.  The caller owns
+ *    every buffer; the library keeps no pointer after a call returns.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Device work is enqueued on it asynchronously; nothing here
+ *    synchronises the host unless its comment says so.
+ *  - Argument errors are returned synchronously, before anything is enqueued.
+ *    CQ_ERR_CUDA means a CUDA runtime call failed (the CUDA error is left
+ *    for cudaGetLastError()).
+ *  - Results are deterministic: the same inputs give the same output bytes.
+ *  - Non-finite or negative inputs never trap: the affected group gets scale
+ *    0x0001 and all codes 0 (nibble 8), and the NONFINITE counter and flag are
+ *    set; cq_read_counters() reports it as CQ_ERR_NONFINITE.
+ */
+#ifndef CQ_H
+#define CQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define CQ_GROUP 128          /* weights per group */
+#define CQ_WORDS 16           /* packed uint32 words per group */
+#define CQ_MAX_E 8            /* environments supported */
+#define CQ_NUM_COUNTERS 8
+
+typedef enum {
+    CQ_OK = 0,
+    CQ_ERR_INVALID_ARG = 1,      /* null pointer, bad size, layout or alignment */
+    CQ_ERR_UNSUPPORTED = 2,      /* E > CQ_MAX_E, or G >= 2^32 */
+    CQ_ERR_CUDA = 3,             /* a CUDA runtime call failed */
+    CQ_ERR_NONFINITE = 4,        /* (cq_read_counters) some group had non-finite/negative input */
+    CQ_ERR_WORKSPACE = 5         /* workspace missing, too small or misaligned */
+} cq_status;
+
+/* Indices into the device counters kept in the workspace. */
+enum {
+    CQ_CNT_FALLBACK = 0,     /* groups decided by the exhaustive 31,743-scale pass */
+    CQ_CNT_NEAR_TIE = 1,     /* groups whose best two candidates are within flag_rel_gap */
+    CQ_CNT_NONFINITE = 2,    /* groups with non-finite weights or non-finite/negative d */
+    CQ_CNT_TRIVIAL = 3,      /* all-zero groups (scale 0x0001, codes 0) */
+    CQ_CNT_FINALISTS = 4,    /* total fp64-rescored candidate scales */
+    CQ_CNT_UNCERTAIN = 5,    /* runs whose screen could not be certified */
+    CQ_CNT_QUEUE = 6,        /* internal: fallback queue length */
+    CQ_CNT_RESERVED = 7
+};
+
+/* Per-group flag bits written to out_flags. */
+#define CQ_FLAG_TRIVIAL   0x01
+#define CQ_FLAG_FALLBACK  0x02
+#define CQ_FLAG_NEAR_TIE  0x04
+#define CQ_FLAG_NONFINITE 0x08
+
+typedef struct {
+    int32_t finalist_cap;     /* max fp64-rescored scales per group before the exhaustive
+                                 fallback; 1..64, 0 = default (32) */
+    int32_t force_exhaustive; /* nonzero: decide every non-trivial group by the exhaustive pass */
+    double flag_rel_gap;      /* CQ_FLAG_NEAR_TIE when the best two finalists are within this
+                                 relative gap; 0 = default (1e-12) */
+    void *ev_main_begin;      /* nullable cudaEvent_t recorded on `stream` just before the main
+                                 selection kernel (profiling hook) */
+    void *ev_main_end;        /* nullable cudaEvent_t recorded just after it, before the fallback */
+} cq_opts;
+
+/* Bytes of device workspace cq_select_scales_ex needs for G groups.  The
+ * workspace holds the counters and the fallback queue (4 bytes per group). */
+size_t cq_workspace_bytes(int64_t G, int E);
+
+/* Select scales and codes for G groups.
+ *  W          [G][128] binary16 bit patterns, 16-byte aligned.
+ *  D          fp32 diagonals, 16-byte aligned, in one of two layouts:
+ *               K > 0:  per column [E][K]; K % 128 == 0 and G % (K/128) == 0;
+ *                       group g uses columns (g % (K/128))*128 .. +127, i.e. W
+ *                       is a row-major [G/(K/128)][K] matrix grouped along rows.
+ *               K == 0: per group [E][G][128].
+ *  E          number of environments, 1..CQ_MAX_E.
+ *  out_scales [G] binary16 bit patterns of the chosen scales (0x0001..0x7BFF).
+ *  out_codes  [G][16] packed codes, 4-byte aligned.
+ * Allocates its workspace with cudaMallocAsync/cudaFreeAsync on `stream`. */
+cq_status cq_select_scales(const uint16_t *W, int64_t G, const float *D, int E, int64_t K,
+                           uint16_t *out_scales, uint32_t *out_codes, void *stream);
+
+/* As cq_select_scales, with caller-provided workspace (device, 256-byte
+ * aligned, at least cq_workspace_bytes(G, E)), options (nullable = defaults)
+ * and optional outputs:
+ *  out_objective  nullable, fp64 [G]: the objective at the chosen scale.
+ *  out_flags      nullable, uint8 [G]: CQ_FLAG_* bits.
+ * The workspace counters are reset at the start of every call.  Calls that
+ * share a workspace must be ordered on one stream. */
+cq_status cq_select_scales_ex(const uint16_t *W, int64_t G, const float *D, int E, int64_t K,
+                              uint16_t *out_scales, uint32_t *out_codes, void *stream,
+                              const cq_opts *opts, void *workspace, size_t workspace_bytes,
+                              double *out_objective, uint8_t *out_flags);
+
+/* Host-buffer variant: W_host, D_host, out_scales_host and out_codes_host are
+ * HOST pointers (page-locked memory gives overlapped copies).  The call
+ * allocates device buffers, streams the groups through them in chunks with
+ * host<->device copies overlapped with compute on `stream`, and returns
+ * after the results are in the host buffers (it synchronises `stream`). */
+cq_status cq_select_scales_host(const uint16_t *W_host, int64_t G, const float *D_host, int E,
+                                int64_t K, uint16_t *out_scales_host, uint32_t *out_codes_host,
+                                void *stream);
+
+/* Copy the workspace counters to host_counters[CQ_NUM_COUNTERS] (host
+ * memory).  Synchronises `stream`.  Returns CQ_ERR_NONFINITE when the last
+ * call saw non-finite input, else CQ_OK (or CQ_ERR_CUDA / CQ_ERR_INVALID_ARG). */
+cq_status cq_read_counters(const void *workspace, uint32_t *host_counters, void *stream);
+
+/* Static, human-readable name of a status code. */
+const char *cq_status_string(cq_status status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int cq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CQ_H */

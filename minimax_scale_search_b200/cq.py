@@ -1,0 +1,230 @@
+"""ctypes binding of libcq.so (argument marshalling only).
+
+Every step of the selection runs in the library's CUDA kernels; PyTorch is used
+for device memory, pinned host memory and streams.  Importing this module loads
+``libcq.so`` from this package's directory and raises if it is missing: there
+is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcq.so")
+
+CQ_OK, CQ_ERR_INVALID_ARG, CQ_ERR_UNSUPPORTED, CQ_ERR_CUDA, CQ_ERR_NONFINITE, CQ_ERR_WORKSPACE = range(6)
+CQ_NUM_COUNTERS = 8
+COUNTER_NAMES = ("fallback", "near_tie", "nonfinite", "trivial", "finalists", "uncertain", "queue", "reserved")
+FLAG_TRIVIAL, FLAG_FALLBACK, FLAG_NEAR_TIE, FLAG_NONFINITE = 0x01, 0x02, 0x04, 0x08
+GROUP = 128
+WORDS = 16
+MAX_E = 8
+
+# Symbols the C header declares, in declaration order.
+EXPORTS = ("cq_workspace_bytes", "cq_select_scales", "cq_select_scales_ex", "cq_select_scales_host",
+           "cq_read_counters", "cq_status_string", "cq_version")
+
+
+class CQError(RuntimeError):
+    def __init__(self, status: int, where: str = ""):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}" if where else status_string(status))
+
+
+class Opts(ctypes.Structure):
+    _fields_ = [("finalist_cap", ctypes.c_int32), ("force_exhaustive", ctypes.c_int32),
+                ("flag_rel_gap", ctypes.c_double), ("ev_main_begin", ctypes.c_void_p),
+                ("ev_main_end", ctypes.c_void_p)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m minimax_scale_search_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    L.cq_workspace_bytes.restype = ctypes.c_size_t
+    L.cq_workspace_bytes.argtypes = [i64, i32]
+    L.cq_select_scales.restype = i32
+    L.cq_select_scales.argtypes = [vp, i64, vp, i32, i64, vp, vp, vp]
+    L.cq_select_scales_ex.restype = i32
+    L.cq_select_scales_ex.argtypes = [vp, i64, vp, i32, i64, vp, vp, vp, ctypes.POINTER(Opts), vp,
+                                      ctypes.c_size_t, vp, vp]
+    L.cq_select_scales_host.restype = i32
+    L.cq_select_scales_host.argtypes = [vp, i64, vp, i32, i64, vp, vp, vp]
+    L.cq_read_counters.restype = i32
+    L.cq_read_counters.argtypes = [vp, vp, vp]
+    L.cq_status_string.restype = ctypes.c_char_p
+    L.cq_status_string.argtypes = [i32]
+    L.cq_version.restype = i32
+    L.cq_version.argtypes = []
+    return L
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.cq_status_string(int(status)).decode()
+
+
+def version() -> int:
+    return int(lib.cq_version())
+
+
+def workspace_bytes(G: int, E: int) -> int:
+    return int(lib.cq_workspace_bytes(int(G), int(E)))
+
+
+def _check(status: int, where: str):
+    if status != CQ_OK:
+        raise CQError(status, where)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    if t is None:
+        return ctypes.c_void_p(None)
+    if isinstance(t, np.ndarray):
+        return ctypes.c_void_p(t.ctypes.data)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+@dataclass
+class Result:
+    scales: "object"          # torch.int16 [G]: binary16 bit patterns
+    codes: "object"           # torch.int32 [G, 16]: packed nibble words (uint32 bits)
+    objective: "object" = None  # torch.float64 [G]
+    flags: "object" = None      # torch.uint8 [G]
+    workspace: "object" = None  # torch.uint8: counters + fallback queue
+
+    def counters(self, stream=None) -> dict:
+        return read_counters(self.workspace, stream)
+
+
+def _shapes(W, D, K):
+    if W.dim() != 2 or W.shape[-1] % GROUP:
+        raise ValueError("W must be 2-D with a multiple of 128 columns")
+    G = W.numel() // GROUP
+    if D.dim() == 2:
+        E, Kd = D.shape
+        if K is not None and K != Kd:
+            raise ValueError("K does not match D")
+        K = Kd
+    elif D.dim() == 3:
+        E = D.shape[0]
+        if D.shape[1:] != (G, GROUP):
+            raise ValueError("per-group D must be [E, G, 128]")
+        K = 0
+    else:
+        raise ValueError("D must be [E, K] or [E, G, 128]")
+    return G, E, K
+
+
+def select_scales(W, D, K: int | None = None, *, stream=None, finalist_cap: int = 0,
+                  force_exhaustive: bool = False, flag_rel_gap: float = 0.0,
+                  out_scales=None, out_codes=None, want_objective: bool = False,
+                  want_flags: bool = False, workspace=None, main_events=None) -> Result:
+    """Exact minimax FP16 scales and packed W4 codes for every 128-weight group.
+
+    W: CUDA tensor of binary16 bit patterns (int16/uint16/float16), [R, K] grouped
+       along rows or [G, 128].  D: CUDA float32, per column [E, K] or per group
+       [E, G, 128].  Runs asynchronously on ``stream`` (default: current).
+       main_events: optional pair of torch.cuda.Event (enable_timing=True)
+       recorded just before and after the main selection kernel."""
+    import torch
+    if not (W.is_cuda and D.is_cuda):
+        raise ValueError("W and D must be CUDA tensors")
+    if W.element_size() != 2:
+        raise ValueError("W must hold 16-bit binary16 patterns")
+    if D.dtype != torch.float32:
+        raise ValueError("D must be float32")
+    if not (W.is_contiguous() and D.is_contiguous()):
+        raise ValueError("W and D must be contiguous")
+    G, E, K = _shapes(W, D, K)
+    dev = W.device
+    if out_scales is None:
+        out_scales = torch.empty(G, dtype=torch.int16, device=dev)
+    if out_codes is None:
+        out_codes = torch.empty((G, WORDS), dtype=torch.int32, device=dev)
+    obj = torch.empty(G, dtype=torch.float64, device=dev) if want_objective else None
+    flags = torch.empty(G, dtype=torch.uint8, device=dev) if want_flags else None
+    wsb = workspace_bytes(G, E)
+    if workspace is None or workspace.numel() < wsb:
+        workspace = torch.empty(wsb, dtype=torch.uint8, device=dev)
+    ev0 = ev1 = None
+    if main_events is not None:  # (torch.cuda.Event, torch.cuda.Event) around the main kernel
+        for e in main_events:  # torch creates the event lazily, at its first record
+            if not e.cuda_event:
+                e.record(stream)
+        ev0, ev1 = (ctypes.c_void_p(e.cuda_event) for e in main_events)
+    opts = Opts(int(finalist_cap), int(bool(force_exhaustive)), float(flag_rel_gap), ev0, ev1)
+    st = lib.cq_select_scales_ex(_ptr(W), G, _ptr(D), E, K, _ptr(out_scales), _ptr(out_codes),
+                                 _stream_handle(stream), ctypes.byref(opts), _ptr(workspace), wsb,
+                                 _ptr(obj), _ptr(flags))
+    _check(st, "cq_select_scales_ex")
+    return Result(out_scales, out_codes, obj, flags, workspace)
+
+
+def select_scales_plain(W, D, K: int | None = None, *, stream=None, out_scales=None, out_codes=None):
+    """The plain entry point (library-allocated workspace); returns (scales, codes)."""
+    import torch
+    G, E, K = _shapes(W, D, K)
+    if out_scales is None:
+        out_scales = torch.empty(G, dtype=torch.int16, device=W.device)
+    if out_codes is None:
+        out_codes = torch.empty((G, WORDS), dtype=torch.int32, device=W.device)
+    st = lib.cq_select_scales(_ptr(W), G, _ptr(D), E, K, _ptr(out_scales), _ptr(out_codes),
+                              _stream_handle(stream))
+    _check(st, "cq_select_scales")
+    return out_scales, out_codes
+
+
+def select_scales_host(W, D, K: int | None = None, *, stream=None, out_scales=None, out_codes=None):
+    """Host-buffer entry point: W, D and the outputs live in host memory (numpy
+    arrays or CPU tensors; page-locked memory overlaps the copies).  Blocks
+    until the results are on the host.  Returns (scales uint16 [G], codes uint32 [G, 16])."""
+    W = W.numpy() if hasattr(W, "numpy") and not isinstance(W, np.ndarray) else W
+    D = D.numpy() if hasattr(D, "numpy") and not isinstance(D, np.ndarray) else D
+    if W.dtype.itemsize != 2 or W.ndim != 2 or W.shape[-1] % GROUP or not W.flags.c_contiguous:
+        raise ValueError("W must be a contiguous 2-D array of 16-bit patterns")
+    if D.dtype != np.float32 or not D.flags.c_contiguous:
+        raise ValueError("D must be contiguous float32")
+    G = W.size // GROUP
+    if D.ndim == 2:
+        E, K = D.shape
+    else:
+        E, K = D.shape[0], 0
+    if out_scales is None:
+        out_scales = np.empty(G, dtype=np.uint16)
+    if out_codes is None:
+        out_codes = np.empty((G, WORDS), dtype=np.uint32)
+    st = lib.cq_select_scales_host(_ptr(W), G, _ptr(D), E, K, _ptr(out_scales), _ptr(out_codes),
+                                   _stream_handle(stream))
+    _check(st, "cq_select_scales_host")
+    return out_scales, out_codes
+
+
+def read_counters(workspace, stream=None) -> dict:
+    """Synchronises ``stream`` and returns the counters of the last call."""
+    host = np.zeros(CQ_NUM_COUNTERS, dtype=np.uint32)
+    st = lib.cq_read_counters(_ptr(workspace), _ptr(host), _stream_handle(stream))
+    if st not in (CQ_OK, CQ_ERR_NONFINITE):
+        raise CQError(st, "cq_read_counters")
+    return {n: int(v) for n, v in zip(COUNTER_NAMES, host)}
+
+
+def to_numpy_bits(res: Result):
+    """(scales uint16 [G], codes uint32 [G, 16]) on the host."""
+    s = res.scales.cpu().numpy().view(np.uint16)
+    c = res.codes.cpu().numpy().view(np.uint32)
+    return s, c

@@ -1,0 +1,1095 @@
+// Exact minimax FP16 group-scale selection (W4, group 128) for sm_100a.
+//
+// Operation (CliffQuant project page, "What CliffQuant changes"): for every
+// group of 128 weights w_i and E environment diagonals d_{e,i}, pick the
+// positive finite binary16 scale s minimising
+//     f(s) = max_e sum_i d_{e,i} (w_i - s q_i(s))^2,
+//     q_i(s) = clip(round-half-even(w_i / s), -8, 7),
+// with an exact tie going to the lower bit pattern, and emit the codes packed
+// as (q+8) nibbles, 8 per uint32, low nibble first.
+//
+// Design (one warp per group, persistent grid, no tensor cores: the work is
+// comparisons and short fp64 dot products, not a dense contraction):
+//
+//  1. Load: 8-byte weight loads and 16-byte diagonal loads per lane; the
+//     group's w and d are staged in shared memory for indexed access.
+//  2. Code transitions ("candidates induced by code transitions"): weight i
+//     changes |q_i| from k+1 to k at the smallest grid index t_{i,k} where
+//     |w_i| < s (k + 1/2) (or equality with k even).  t is found from an fp32
+//     estimate and fixed by exact fp32 threshold tests (s * (k + 1/2) has at
+//     most 16 significant bits, so the product is exact).
+//  3. Ordering: the <= 1024 keys (t, i, k) are bitonic-sorted in registers.
+//  4. Coefficient scan: on a run of constant codes F_e(s) = A_e - 2 B_e s +
+//     C_e s^2 with B_e = sum d|w||q|, C_e = sum d q^2 ("quadratic"); B and C
+//     are exact-term fp64 suffix sums over the sorted transitions.
+//  5. Per run: max_e F_e is convex in s, so the leftmost grid minimiser is
+//     found by a binary search on the sign of f(s_{j+1}) - f(s_j).  Every
+//     comparison is certified against a rigorous bound on the fp64 evaluation
+//     error (2^-44 of sum_e-max of A + 2Bs + Cs^2); a run with an uncertified
+//     comparison falls back to a lower bound from its quadratic vertices
+//     ("quadratic vertices"), and the group goes to the exhaustive pass if
+//     that run could still hold the minimum.
+//  6. Finalists: the runs whose certified lower bound is within 2^-40 of the
+//     best certified upper bound; each is rescored with the direct fp64
+//     objective (exact codes, exact residuals) and the (objective, pattern)
+//     minimum wins.
+//  7. Exhaustive fallback (the page's conservative exhaustive-grid check):
+//     queued groups are solved over all 31,743 scales in the definition's
+//     own fp64 evaluation order by a second kernel, one CTA per group.
+//  8. Pack: each lane packs 4 codes; pairs of lanes form one uint32.
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cfloat>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "cq.h"
+
+namespace cq {
+
+constexpr int kGroup = 128;
+constexpr uint32_t kLast = 0x7BFFu;    // largest finite binary16 pattern (65504)
+constexpr uint32_t kBeyond = 0x7C00u;  // one past the grid
+constexpr int kWarps = 8;              // warps (groups in flight) per CTA of the main kernel
+constexpr int kKeys = 1024;            // 128 weights x up to 8 transitions
+constexpr uint32_t kInvalidKey = 0xFFFFFFFFu;
+constexpr int kMaxFinalists = 64;
+constexpr int kDefaultFinalists = 32;
+constexpr uint32_t kUncertainBit = 0x8000u;
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
+struct Params {
+    const uint16_t *W;
+    const float *D;
+    int64_t G;
+    int64_t K;    // 0: per-group diagonals
+    int64_t gpr;  // groups per row when K > 0
+    uint16_t *out_scales;
+    uint32_t *out_codes;
+    double *out_obj;
+    uint8_t *out_flags;
+    uint32_t *counters;
+    uint32_t *queue;
+    int finalist_cap;
+    int force_exhaustive;
+    double flag_rel_gap;
+    cudaEvent_t ev_begin;
+    cudaEvent_t ev_end;
+};
+
+__device__ __forceinline__ float half_value(uint32_t bits)
+{
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(bits)));
+}
+
+__device__ __forceinline__ const float *diag_ptr(const Params &p, int64_t g, int e)
+{
+    if (p.K > 0)
+        return p.D + static_cast<int64_t>(e) * p.K + (g % p.gpr) * kGroup;
+    return p.D + (static_cast<int64_t>(e) * p.G + g) * kGroup;
+}
+
+// |q| >= m for |w| = aw at scale s, before clipping: round-half-even(aw/s) >= m.
+// s * (m - 1/2) is exact in fp32 (11-bit s times a 5-bit odd/2 factor).
+__device__ __forceinline__ bool code_at_least(float aw, float s, int m)
+{
+    const float t = s * (static_cast<float>(m) - 0.5f);
+    return aw > t || (aw == t && (m & 1) == 0);
+}
+
+// min(round-half-even(aw / s), K), exact: an fp32 estimate corrected by the
+// exact threshold tests above (the estimate is within one of the answer).
+__device__ __forceinline__ int abs_code(float aw, float s, int K)
+{
+    const float x = fminf(__fdividef(aw, s), 15.0f);
+    int n = __float2int_rn(x);
+    if (n > 0 && !code_at_least(aw, s, n))
+        n -= 1;
+    else if (code_at_least(aw, s, n + 1))
+        n += 1;
+    return min(n, K);
+}
+
+// Smallest grid index j in [1, kBeyond] with |q(s_j)| <= k, kBeyond meaning
+// "still above k at 65504".  The fp32 estimate |w|/(k+1/2) rounded up to
+// binary16 is at most one pattern away from the answer.
+template <int k>
+__device__ __forceinline__ uint32_t transition_index(float aw)
+{
+    constexpr float inv = 2.0f / static_cast<float>(2 * k + 1);
+    const float x = aw * inv;
+    uint32_t j0 = __half_as_ushort(__float2half_ru(x));
+    if (j0 > kBeyond)
+        j0 = kBeyond;
+    if (j0 < 1u)
+        j0 = 1u;
+    if (j0 > 1u && !code_at_least(aw, half_value(j0 - 1), k + 1))
+        return j0 - 1;
+    if (j0 == kBeyond || !code_at_least(aw, half_value(j0), k + 1))
+        return j0;
+    return j0 + 1;
+}
+
+// Bank-conflict-free placement of position p = 32*lane + x in a per-warp array.
+__device__ __forceinline__ int swz(int p)
+{
+    return (p & ~31) | ((p ^ (p >> 5)) & 31);
+}
+
+template <typename T>
+__device__ __forceinline__ T warp_sum(T v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v += __shfl_xor_sync(kFull, v, o);
+    return v;
+}
+
+// Ascending bitonic sort of 1024 keys, blocked layout: lane L holds positions
+// 32L .. 32L+31 in key[0..31].
+__device__ __forceinline__ void bitonic_sort_1024(uint32_t (&key)[32], int lane)
+{
+#pragma unroll
+    for (int k = 2; k <= kKeys; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            if (j >= 32) {
+                const int lm = j >> 5;
+                const bool upper = (lane & lm) != 0;
+                const bool asc = ((32 * lane) & k) == 0;
+                const bool keep_min = (asc != upper);
+#pragma unroll
+                for (int x = 0; x < 32; x++) {
+                    const uint32_t other = __shfl_xor_sync(kFull, key[x], lm);
+                    key[x] = keep_min ? min(key[x], other) : max(key[x], other);
+                }
+            } else {
+#pragma unroll
+                for (int x = 0; x < 32; x++) {
+                    const int y = x ^ j;
+                    if (y > x) {
+                        const bool asc = (k >= 32) ? (((32 * lane) & k) == 0) : ((x & k) == 0);
+                        const uint32_t a = key[x], b = key[y];
+                        const uint32_t lo = min(a, b), hi = max(a, b);
+                        key[x] = asc ? lo : hi;
+                        key[y] = asc ? hi : lo;
+                    }
+                }
+            }
+        }
+    }
+}
+
+template <int E>
+struct WarpSmem {
+    float d[E][kGroup];
+    float w[kGroup];
+    uint32_t keys[kKeys];
+    float lb[kKeys + 1];          // certified lower bound of each run's minimum
+    uint16_t jf[kKeys + 2];       // each run's minimiser | kUncertainBit
+    int fin[kMaxFinalists];
+};
+
+struct RunResult {
+    float lb;
+    double ub;
+    uint32_t j;
+    bool uncertain;
+};
+
+template <int E>
+__device__ __forceinline__ double screen(const double (&A)[E], const double (&nb2)[E], const double (&C)[E],
+                                         double s)
+{
+    double f = fma(fma(C[0], s, nb2[0]), s, A[0]);
+#pragma unroll
+    for (int e = 1; e < E; e++)
+        f = fmax(f, fma(fma(C[e], s, nb2[e]), s, A[e]));
+    return f;
+}
+
+// Leftmost grid minimiser of max_e (A_e - 2 B_e s + C_e s^2) over grid
+// indices [ja, jb], with a certified bracket (see the file comment, step 5).
+template <int E>
+__device__ RunResult solve_run(const double (&A)[E], const double (&B)[E], const double (&C)[E],
+                               uint32_t ja, uint32_t jb)
+{
+    RunResult r;
+    double cmax = C[0], amax = A[0];
+#pragma unroll
+    for (int e = 1; e < E; e++) {
+        cmax = fmax(cmax, C[e]);
+        amax = fmax(amax, A[e]);
+    }
+    if (cmax == 0.0) {
+        // every code with d > 0 is zero: f is the constant max_e A_e (exact terms)
+        const double delta = amax * 0x1p-44;
+        r.j = ja;
+        r.ub = amax + delta;
+        r.lb = __double2float_rd(amax - delta);
+        r.uncertain = false;
+        return r;
+    }
+    const double sa = half_value(ja), sb = half_value(jb);
+    double P = 0.0, nb2[E];
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        nb2[e] = -2.0 * B[e];
+        P = fmax(P, fma(fma(C[e], sb, 2.0 * B[e]), sb, A[e]));
+    }
+    const double delta = P * 0x1p-44;  // >= |screen - exact| anywhere on the run
+    uint32_t lo = ja, hi = jb;
+    bool unc = false;
+    while (lo < hi) {
+        const uint32_t mid = (lo + hi) >> 1;
+        const double S0 = screen<E>(A, nb2, C, half_value(mid));
+        const double S1 = screen<E>(A, nb2, C, half_value(mid + 1));
+        const double Dd = S1 - S0;
+        if (fabs(Dd) <= 2.0 * delta + 0x1p-40 * fmax(fabs(S0), fabs(S1)))
+            unc = true;
+        if (Dd >= 0.0)
+            hi = mid;
+        else
+            lo = mid + 1;
+    }
+    const double Sf = screen<E>(A, nb2, C, half_value(lo));
+    r.j = lo;
+    r.ub = Sf + delta;
+    r.uncertain = unc;
+    if (!unc) {
+        r.lb = __double2float_rd(Sf - delta);
+    } else {
+        // max_e of each environment's own minimum over [sa, sb]: a lower bound
+        double L = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < E; e++) {
+            double v = sb;
+            if (C[e] > 0.0)
+                v = fmin(fmax(B[e] / C[e], sa), sb);
+            L = fmax(L, fma(fma(C[e], v, nb2[e]), v, A[e]));
+        }
+        r.lb = __double2float_rd(L - delta);
+    }
+    return r;
+}
+
+// Best two objectives within rel of each other (an exact tie always counts).
+__device__ __forceinline__ bool near_tie(double best, double second, double rel)
+{
+    if (second == best)
+        return true;
+    if (!isfinite(second))
+        return false;
+    const double m = fmax(fabs(best), fabs(second));
+    return m > 0.0 && fabs(second - best) <= rel * m;
+}
+
+__device__ __forceinline__ uint32_t pack_lane_codes(const int (&q)[4], int lane)
+{
+    uint32_t h = 0;
+#pragma unroll
+    for (int m = 0; m < 4; m++)
+        h |= static_cast<uint32_t>((q[m] + 8) & 0xF) << (4 * m);
+    const uint32_t up = __shfl_down_sync(kFull, h, 1);
+    return h | (up << 16);  // valid on even lanes: codes 8*(lane/2) .. +7
+}
+
+__device__ __forceinline__ void write_constant_group(const Params &p, int64_t g, int lane, uint8_t flag,
+                                                     int counter)
+{
+    if (lane < 16)
+        p.out_codes[g * 16 + lane] = 0x88888888u;
+    if (lane == 0) {
+        p.out_scales[g] = 0x0001;
+        if (p.out_obj)
+            p.out_obj[g] = 0.0;
+        if (p.out_flags)
+            p.out_flags[g] = flag;
+        atomicAdd(&p.counters[counter], 1u);
+    }
+}
+
+__device__ __forceinline__ void enqueue(const Params &p, int64_t g, int lane)
+{
+    if (lane == 0) {
+        const uint32_t at = atomicAdd(&p.counters[CQ_CNT_QUEUE], 1u);
+        p.queue[at] = static_cast<uint32_t>(g);
+        atomicAdd(&p.counters[CQ_CNT_FALLBACK], 1u);
+    }
+}
+
+template <int E>
+__device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int lane)
+{
+    // ---- 1. load -------------------------------------------------------
+    const uint2 wv = *reinterpret_cast<const uint2 *>(p.W + g * kGroup + 4 * lane);
+    const uint32_t wb[4] = {wv.x & 0xFFFFu, wv.x >> 16, wv.y & 0xFFFFu, wv.y >> 16};
+    float wf[4];
+    float dr[E][4];
+    bool bad = false, nonzero = false;
+#pragma unroll
+    for (int m = 0; m < 4; m++) {
+        wf[m] = half_value(wb[m]);
+        bad |= (wb[m] & 0x7C00u) == 0x7C00u;
+        nonzero |= (wb[m] & 0x7FFFu) != 0u;
+        sm.w[4 * lane + m] = wf[m];
+    }
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        const float4 dv = *reinterpret_cast<const float4 *>(diag_ptr(p, g, e) + 4 * lane);
+        dr[e][0] = dv.x;
+        dr[e][1] = dv.y;
+        dr[e][2] = dv.z;
+        dr[e][3] = dv.w;
+#pragma unroll
+        for (int m = 0; m < 4; m++) {
+            bad |= !(dr[e][m] >= 0.0f && dr[e][m] <= FLT_MAX);
+            sm.d[e][4 * lane + m] = dr[e][m];
+        }
+    }
+    bad = __any_sync(kFull, bad);
+    nonzero = __any_sync(kFull, nonzero);
+    if (bad) {
+        write_constant_group(p, g, lane, CQ_FLAG_NONFINITE, CQ_CNT_NONFINITE);
+        return;
+    }
+    if (!nonzero) {
+        write_constant_group(p, g, lane, CQ_FLAG_TRIVIAL, CQ_CNT_TRIVIAL);
+        return;
+    }
+    if (p.force_exhaustive) {
+        enqueue(p, g, lane);
+        return;
+    }
+
+    // ---- 2. A_e = sum d w^2 (exact terms) -------------------------------
+    double A[E];
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        double a = 0.0;
+#pragma unroll
+        for (int m = 0; m < 4; m++)
+            a += static_cast<double>(dr[e][m]) * (static_cast<double>(wf[m]) * static_cast<double>(wf[m]));
+        A[e] = warp_sum(a);
+    }
+
+    // ---- 3. transitions -------------------------------------------------
+    uint32_t key[32];
+#pragma unroll
+    for (int m = 0; m < 4; m++) {
+        const float aw = fabsf(wf[m]);
+        const int Kc = ((wb[m] & 0x7FFFu) == 0u) ? 0 : ((wb[m] & 0x8000u) ? 8 : 7);
+        const uint32_t ib = static_cast<uint32_t>(4 * lane + m) << 3;
+#define CQ_T(kk)                                                                                     \
+    key[8 * m + kk] = (kk < Kc) ? ((transition_index<kk>(aw) << 10) | ib | static_cast<uint32_t>(kk)) \
+                                : kInvalidKey;
+        CQ_T(0) CQ_T(1) CQ_T(2) CQ_T(3) CQ_T(4) CQ_T(5) CQ_T(6) CQ_T(7)
+#undef CQ_T
+    }
+
+    // ---- 4. order -------------------------------------------------------
+    bitonic_sort_1024(key, lane);
+
+    // ---- 5. coefficient scan: lane totals, then suffix across lanes ----
+    double TB[E], TC[E];
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        TB[e] = 0.0;
+        TC[e] = 0.0;
+    }
+#pragma unroll
+    for (int x = 0; x < 32; x++) {
+        sm.keys[swz(32 * lane + x)] = key[x];
+    }
+    __syncwarp();
+#pragma unroll 4
+    for (int x = 0; x < 32; x++) {
+        const uint32_t kk = sm.keys[swz(32 * lane + x)];
+        if (kk != kInvalidKey) {
+            const int i = (kk >> 3) & 127;
+            const double aw = fabs(static_cast<double>(sm.w[i]));
+            const double c = static_cast<double>(2 * (kk & 7) + 1);
+#pragma unroll
+            for (int e = 0; e < E; e++) {
+                const double dd = sm.d[e][i];
+                TB[e] += dd * aw;
+                TC[e] += dd * c;
+            }
+        }
+    }
+    double RB[E], RC[E];
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        double vb = TB[e], vc = TC[e];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double ub = __shfl_down_sync(kFull, vb, o);
+            const double uc = __shfl_down_sync(kFull, vc, o);
+            if (lane + o < 32) {
+                vb += ub;
+                vc += uc;
+            }
+        }
+        const double xb = __shfl_down_sync(kFull, vb, 1);
+        const double xc = __shfl_down_sync(kFull, vc, 1);
+        RB[e] = (lane == 31) ? 0.0 : xb;
+        RC[e] = (lane == 31) ? 0.0 : xc;
+    }
+
+    // ---- 6. runs ----------------------------------------------------------
+    uint32_t next_t = kBeyond;
+    {
+        const uint32_t kn = (lane < 31) ? sm.keys[swz(32 * lane + 32)] : kInvalidKey;
+        if (kn != kInvalidKey)
+            next_t = kn >> 10;
+    }
+    double ub_min = INFINITY;
+    for (int x = 31; x >= 0; --x) {
+        const int pos = 32 * lane + x;
+        const uint32_t kk = sm.keys[swz(pos)];
+        float lbv = INFINITY;
+        uint32_t jv = 0;
+        if (kk != kInvalidKey) {
+            const uint32_t t = kk >> 10;
+            if (t <= kLast && t != next_t) {
+                const RunResult rr = solve_run<E>(A, RB, RC, t, min(next_t, kBeyond) - 1u);
+                lbv = rr.lb;
+                jv = rr.j | (rr.uncertain ? kUncertainBit : 0u);
+                ub_min = fmin(ub_min, rr.ub);
+            }
+            const int i = (kk >> 3) & 127;
+            const double aw = fabs(static_cast<double>(sm.w[i]));
+            const double c = static_cast<double>(2 * (kk & 7) + 1);
+#pragma unroll
+            for (int e = 0; e < E; e++) {
+                const double dd = sm.d[e][i];
+                RB[e] += dd * aw;
+                RC[e] += dd * c;
+            }
+            next_t = t;
+        }
+        sm.lb[swz(pos)] = lbv;
+        sm.jf[swz(pos)] = static_cast<uint16_t>(jv);
+    }
+    if (lane == 0) {
+        // the run below every transition: [1, t_0 - 1], all transitions active
+        float lbv = INFINITY;
+        uint32_t jv = 0;
+        if (next_t > 1u) {
+            const RunResult rr = solve_run<E>(A, RB, RC, 1u, min(next_t, kBeyond) - 1u);
+            lbv = rr.lb;
+            jv = rr.j | (rr.uncertain ? kUncertainBit : 0u);
+            ub_min = fmin(ub_min, rr.ub);
+        }
+        sm.lb[kKeys] = lbv;
+        sm.jf[kKeys] = static_cast<uint16_t>(jv);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        ub_min = fmin(ub_min, __shfl_xor_sync(kFull, ub_min, o));
+    const float T = __double2float_ru(ub_min * (1.0 + 0x1p-40));
+    __syncwarp();
+
+    // ---- 7. finalists -----------------------------------------------------
+    int cnt = 0;
+    bool unc_comp = false, unc_any = false;
+    for (int x = 0; x < 33; x++) {
+        if (x == 32 && lane != 0)
+            break;
+        const int at = (x == 32) ? kKeys : swz(32 * lane + x);
+        const uint32_t jv = sm.jf[at];
+        unc_any |= (jv & kUncertainBit) != 0u && sm.lb[at] < INFINITY;
+        if (sm.lb[at] <= T) {
+            if (jv & kUncertainBit)
+                unc_comp = true;
+            else
+                cnt++;
+        }
+    }
+    if (__any_sync(kFull, unc_any) && lane == 0)
+        atomicAdd(&p.counters[CQ_CNT_UNCERTAIN], 1u);
+    unc_comp = __any_sync(kFull, unc_comp);
+    int excl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(kFull, excl, o);
+        if (lane >= o)
+            excl += u;
+    }
+    const int total = __shfl_sync(kFull, excl, 31);
+    excl -= cnt;
+    if (unc_comp || total > p.finalist_cap || total == 0) {
+        enqueue(p, g, lane);
+        return;
+    }
+    {
+        int o = excl;
+        for (int x = 0; x < 33; x++) {
+            if (x == 32 && lane != 0)
+                break;
+            const int at = (x == 32) ? kKeys : swz(32 * lane + x);
+            if (sm.lb[at] <= T && !(sm.jf[at] & kUncertainBit))
+                sm.fin[o++] = sm.jf[at];
+        }
+    }
+    __syncwarp();
+
+    // ---- 8. fp64 rescoring of the finalists -------------------------------
+    int Kc[4];
+#pragma unroll
+    for (int m = 0; m < 4; m++)
+        Kc[m] = (wb[m] & 0x8000u) ? 8 : 7;
+    double best = INFINITY, second = INFINITY;
+    uint32_t bj = 0;
+    for (int f = 0; f < total; f++) {
+        const uint32_t j = static_cast<uint32_t>(sm.fin[f]);
+        const float s = half_value(j);
+        const double sd = s;
+        double acc[E];
+#pragma unroll
+        for (int e = 0; e < E; e++)
+            acc[e] = 0.0;
+#pragma unroll
+        for (int m = 0; m < 4; m++) {
+            const int aq = abs_code(fabsf(wf[m]), s, Kc[m]);
+            const double q = (wb[m] & 0x8000u) ? -static_cast<double>(aq) : static_cast<double>(aq);
+            const double r = static_cast<double>(wf[m]) - sd * q;  // exact
+            const double rr = __dmul_rn(r, r);
+#pragma unroll
+            for (int e = 0; e < E; e++)
+                acc[e] = __dadd_rn(acc[e], __dmul_rn(static_cast<double>(dr[e][m]), rr));
+        }
+        double v = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < E; e++)
+            v = fmax(v, warp_sum(acc[e]));
+        if (v < best || (v == best && j < bj)) {
+            second = best;
+            best = v;
+            bj = j;
+        } else if (v < second) {
+            second = v;
+        }
+    }
+
+    // ---- 9. pack and store ------------------------------------------------
+    const float s = half_value(bj);
+    int q[4];
+#pragma unroll
+    for (int m = 0; m < 4; m++) {
+        const int aq = abs_code(fabsf(wf[m]), s, Kc[m]);
+        q[m] = (wb[m] & 0x8000u) ? -aq : aq;
+    }
+    const uint32_t word = pack_lane_codes(q, lane);
+    if ((lane & 1) == 0)
+        p.out_codes[g * 16 + (lane >> 1)] = word;
+    if (lane == 0) {
+        p.out_scales[g] = static_cast<uint16_t>(bj);
+        if (p.out_obj)
+            p.out_obj[g] = best;
+        const bool near = near_tie(best, second, p.flag_rel_gap);
+        if (p.out_flags)
+            p.out_flags[g] = near ? CQ_FLAG_NEAR_TIE : 0;
+        if (near)
+            atomicAdd(&p.counters[CQ_CNT_NEAR_TIE], 1u);
+        atomicAdd(&p.counters[CQ_CNT_FINALISTS], static_cast<uint32_t>(total));
+    }
+}
+
+template <int E>
+__global__ void __launch_bounds__(kWarps * 32) select_kernel(Params p)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int lane = threadIdx.x & 31;
+    const int wib = threadIdx.x >> 5;
+    WarpSmem<E> &sm = reinterpret_cast<WarpSmem<E> *>(smem_raw)[wib];
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * kWarps;
+    for (int64_t g = static_cast<int64_t>(blockIdx.x) * kWarps + wib; g < p.G; g += stride) {
+        process_group<E>(p, sm, g, lane);
+        __syncwarp();
+    }
+}
+
+// ---- exhaustive fallback: one CTA per queued group, all 31,743 scales ------
+
+constexpr int kExThreads = 256;
+
+struct Best3 {
+    double best, second;
+    uint32_t j;
+};
+
+__device__ __forceinline__ Best3 combine(Best3 a, Best3 b)
+{
+    if (a.best < b.best || (a.best == b.best && a.j < b.j)) {
+        a.second = fmin(a.second, b.best);
+        return a;
+    }
+    b.second = fmin(b.second, a.best);
+    return b;
+}
+
+template <int E>
+__global__ void __launch_bounds__(kExThreads) exhaustive_kernel(Params p)
+{
+    __shared__ float ws[kGroup];
+    __shared__ float ds[E][kGroup];
+    __shared__ Best3 red[kExThreads / 32];
+    __shared__ uint32_t nib[kGroup];
+    const int tid = threadIdx.x;
+    const uint32_t count = p.counters[CQ_CNT_QUEUE];
+    for (uint32_t qi = blockIdx.x; qi < count; qi += gridDim.x) {
+        const int64_t g = p.queue[qi];
+        if (tid < kGroup) {
+            ws[tid] = half_value(p.W[g * kGroup + tid]);
+#pragma unroll
+            for (int e = 0; e < E; e++)
+                ds[e][tid] = diag_ptr(p, g, e)[tid];
+        }
+        __syncthreads();
+        Best3 b{INFINITY, INFINITY, 0u};
+        for (uint32_t j = 1u + tid; j <= kLast; j += kExThreads) {
+            const float s = half_value(j);
+            const double sd = s;
+            double acc[E];
+#pragma unroll
+            for (int e = 0; e < E; e++)
+                acc[e] = 0.0;
+            // the definition's own order: i ascending, one sum per environment
+            for (int i = 0; i < kGroup; i++) {
+                const float w = ws[i];
+                const int aq = abs_code(fabsf(w), s, w < 0.0f ? 8 : 7);
+                const double q = (w < 0.0f) ? -static_cast<double>(aq) : static_cast<double>(aq);
+                const double r = static_cast<double>(w) - sd * q;
+                const double rr = __dmul_rn(r, r);
+#pragma unroll
+                for (int e = 0; e < E; e++)
+                    acc[e] = __dadd_rn(acc[e], __dmul_rn(static_cast<double>(ds[e][i]), rr));
+            }
+            double v = acc[0];
+#pragma unroll
+            for (int e = 1; e < E; e++)
+                v = fmax(v, acc[e]);
+            if (v < b.best) {  // j ascends within a thread: strict < keeps the lowest
+                b.second = b.best;
+                b.best = v;
+                b.j = j;
+            } else if (v < b.second) {
+                b.second = v;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            Best3 other;
+            other.best = __shfl_xor_sync(kFull, b.best, o);
+            other.second = __shfl_xor_sync(kFull, b.second, o);
+            other.j = __shfl_xor_sync(kFull, b.j, o);
+            b = combine(b, other);
+        }
+        if ((tid & 31) == 0)
+            red[tid >> 5] = b;
+        __syncthreads();
+        if (tid == 0) {
+            Best3 r = red[0];
+            for (int w = 1; w < kExThreads / 32; w++)
+                r = combine(r, red[w]);
+            red[0] = r;
+        }
+        __syncthreads();
+        const Best3 r = red[0];
+        if (tid < kGroup) {
+            const float w = ws[tid];
+            const float s = half_value(r.j);
+            const int aq = abs_code(fabsf(w), s, w < 0.0f ? 8 : 7);
+            const int q = (w < 0.0f) ? -aq : aq;
+            nib[tid] = static_cast<uint32_t>((q + 8) & 0xF);
+        }
+        __syncthreads();
+        if (tid < 16) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int t = 0; t < 8; t++)
+                word |= nib[8 * tid + t] << (4 * t);
+            p.out_codes[g * 16 + tid] = word;
+        }
+        if (tid == 0) {
+            p.out_scales[g] = static_cast<uint16_t>(r.j);
+            if (p.out_obj)
+                p.out_obj[g] = r.best;
+            const bool near = near_tie(r.best, r.second, p.flag_rel_gap);
+            if (p.out_flags)
+                p.out_flags[g] = CQ_FLAG_FALLBACK | (near ? CQ_FLAG_NEAR_TIE : 0);
+            if (near)
+                atomicAdd(&p.counters[CQ_CNT_NEAR_TIE], 1u);
+        }
+        __syncthreads();
+    }
+}
+
+// ---- host side ---------------------------------------------------------------
+
+constexpr size_t kHeaderBytes = 256;
+
+size_t workspace_bytes(int64_t G)
+{
+    const size_t q = static_cast<size_t>(G < 0 ? 0 : G) * sizeof(uint32_t);
+    return kHeaderBytes + ((q + 255) / 256) * 256;
+}
+
+struct DeviceInfo {
+    int sms = 0;
+    bool init = false;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[64];
+cudaMemPool_t g_pool[64];
+bool g_pool_init[64];
+
+int sm_count(int dev)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (dev < 0 || dev >= 64)
+        return 148;
+    if (!g_dev[dev].init) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        g_dev[dev].sms = n;
+        g_dev[dev].init = true;
+    }
+    return g_dev[dev].sms;
+}
+
+// Library-private stream-ordered pool, so the caller's default pool settings
+// are left alone and freed blocks are kept for the next call.
+cudaError_t pool_alloc(void **ptr, size_t bytes, cudaStream_t st)
+{
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess)
+        return err;
+    if (dev < 0 || dev >= 64)
+        return cudaErrorInvalidDevice;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_pool_init[dev]) {
+            cudaMemPoolProps props;
+            memset(&props, 0, sizeof(props));
+            props.allocType = cudaMemAllocationTypePinned;
+            props.handleTypes = cudaMemHandleTypeNone;
+            props.location.type = cudaMemLocationTypeDevice;
+            props.location.id = dev;
+            err = cudaMemPoolCreate(&g_pool[dev], &props);
+            if (err != cudaSuccess)
+                return err;
+            uint64_t keep = UINT64_MAX;
+            cudaMemPoolSetAttribute(g_pool[dev], cudaMemPoolAttrReleaseThreshold, &keep);
+            g_pool_init[dev] = true;
+        }
+    }
+    return cudaMallocFromPoolAsync(ptr, bytes, g_pool[dev], st);
+}
+
+template <int E>
+cudaError_t launch(const Params &p, cudaStream_t st)
+{
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess)
+        return err;
+    const int sms = sm_count(dev);
+    const size_t smem = sizeof(WarpSmem<E>) * kWarps;
+    err = cudaFuncSetAttribute(select_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    if (err != cudaSuccess)
+        return err;
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel<E>, kWarps * 32, smem);
+    if (err != cudaSuccess)
+        return err;
+    if (per_sm < 1)
+        per_sm = 1;
+    const int64_t need = (p.G + kWarps - 1) / kWarps;
+    const int64_t grid = need < static_cast<int64_t>(sms) * per_sm ? need : static_cast<int64_t>(sms) * per_sm;
+    if (p.ev_begin && (err = cudaEventRecord(p.ev_begin, st)) != cudaSuccess)
+        return err;
+    select_kernel<E><<<static_cast<unsigned>(grid), kWarps * 32, smem, st>>>(p);
+    err = cudaGetLastError();
+    if (err != cudaSuccess)
+        return err;
+    if (p.ev_end && (err = cudaEventRecord(p.ev_end, st)) != cudaSuccess)
+        return err;
+    exhaustive_kernel<E><<<static_cast<unsigned>(2 * sms), kExThreads, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t dispatch(int E, const Params &p, cudaStream_t st)
+{
+    switch (E) {
+    case 1: return launch<1>(p, st);
+    case 2: return launch<2>(p, st);
+    case 3: return launch<3>(p, st);
+    case 4: return launch<4>(p, st);
+    case 5: return launch<5>(p, st);
+    case 6: return launch<6>(p, st);
+    case 7: return launch<7>(p, st);
+    case 8: return launch<8>(p, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+bool aligned(const void *ptr, size_t a)
+{
+    return (reinterpret_cast<uintptr_t>(ptr) % a) == 0;
+}
+
+cq_status validate(const uint16_t *W, int64_t G, const float *D, int E, int64_t K, const uint16_t *out_scales,
+                   const uint32_t *out_codes)
+{
+    if (G < 0 || K < 0)
+        return CQ_ERR_INVALID_ARG;
+    if (E < 1)
+        return CQ_ERR_INVALID_ARG;
+    if (E > CQ_MAX_E)
+        return CQ_ERR_UNSUPPORTED;
+    if (G >= (static_cast<int64_t>(1) << 32))
+        return CQ_ERR_UNSUPPORTED;
+    if (K > 0) {
+        if (K % kGroup != 0)
+            return CQ_ERR_INVALID_ARG;
+        if (G % (K / kGroup) != 0)
+            return CQ_ERR_INVALID_ARG;
+    }
+    if (G == 0)
+        return CQ_OK;
+    if (!W || !D || !out_scales || !out_codes)
+        return CQ_ERR_INVALID_ARG;
+    if (!aligned(W, 16) || !aligned(D, 16) || !aligned(out_codes, 4) || !aligned(out_scales, 2))
+        return CQ_ERR_INVALID_ARG;
+    return CQ_OK;
+}
+
+}  // namespace cq
+
+using namespace cq;
+
+extern "C" {
+
+size_t cq_workspace_bytes(int64_t G, int E)
+{
+    (void)E;
+    return workspace_bytes(G);
+}
+
+cq_status cq_select_scales_ex(const uint16_t *W, int64_t G, const float *D, int E, int64_t K,
+                              uint16_t *out_scales, uint32_t *out_codes, void *stream, const cq_opts *opts,
+                              void *workspace, size_t ws_bytes, double *out_objective, uint8_t *out_flags)
+{
+    cq_status st = validate(W, G, D, E, K, out_scales, out_codes);
+    if (st != CQ_OK)
+        return st;
+    if (!workspace || ws_bytes < workspace_bytes(G) || !aligned(workspace, 256))
+        return CQ_ERR_WORKSPACE;
+    if ((out_objective && !aligned(out_objective, 8)))
+        return CQ_ERR_INVALID_ARG;
+    Params p;
+    p.W = W;
+    p.D = D;
+    p.G = G;
+    p.K = K;
+    p.gpr = K > 0 ? K / kGroup : 1;
+    p.out_scales = out_scales;
+    p.out_codes = out_codes;
+    p.out_obj = out_objective;
+    p.out_flags = out_flags;
+    p.counters = static_cast<uint32_t *>(workspace);
+    p.queue = reinterpret_cast<uint32_t *>(static_cast<unsigned char *>(workspace) + kHeaderBytes);
+    p.finalist_cap = kDefaultFinalists;
+    p.force_exhaustive = 0;
+    p.flag_rel_gap = 1e-12;
+    p.ev_begin = nullptr;
+    p.ev_end = nullptr;
+    if (opts) {
+        p.ev_begin = static_cast<cudaEvent_t>(opts->ev_main_begin);
+        p.ev_end = static_cast<cudaEvent_t>(opts->ev_main_end);
+        if (opts->finalist_cap < 0 || opts->finalist_cap > kMaxFinalists)
+            return CQ_ERR_INVALID_ARG;
+        if (opts->finalist_cap > 0)
+            p.finalist_cap = opts->finalist_cap;
+        p.force_exhaustive = opts->force_exhaustive != 0;
+        if (opts->flag_rel_gap < 0.0 || !(opts->flag_rel_gap == opts->flag_rel_gap))
+            return CQ_ERR_INVALID_ARG;
+        if (opts->flag_rel_gap > 0.0)
+            p.flag_rel_gap = opts->flag_rel_gap;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(workspace, 0, kHeaderBytes, s) != cudaSuccess)
+        return CQ_ERR_CUDA;
+    if (G == 0)
+        return CQ_OK;
+    if (dispatch(E, p, s) != cudaSuccess)
+        return CQ_ERR_CUDA;
+    return CQ_OK;
+}
+
+cq_status cq_select_scales(const uint16_t *W, int64_t G, const float *D, int E, int64_t K, uint16_t *out_scales,
+                           uint32_t *out_codes, void *stream)
+{
+    cq_status st = validate(W, G, D, E, K, out_scales, out_codes);
+    if (st != CQ_OK || G == 0)
+        return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    void *ws = nullptr;
+    const size_t bytes = workspace_bytes(G);
+    if (pool_alloc(&ws, bytes, s) != cudaSuccess)
+        return CQ_ERR_CUDA;
+    st = cq_select_scales_ex(W, G, D, E, K, out_scales, out_codes, stream, nullptr, ws, bytes, nullptr, nullptr);
+    if (cudaFreeAsync(ws, s) != cudaSuccess && st == CQ_OK)
+        st = CQ_ERR_CUDA;
+    return st;
+}
+
+cq_status cq_select_scales_host(const uint16_t *W_host, int64_t G, const float *D_host, int E, int64_t K,
+                                uint16_t *out_scales_host, uint32_t *out_codes_host, void *stream)
+{
+    cq_status st = validate(W_host, G, D_host, E, K, out_scales_host, out_codes_host);
+    if (st != CQ_OK || G == 0)
+        return st;
+    cudaStream_t user = static_cast<cudaStream_t>(stream);
+    const int64_t gpr = K > 0 ? K / kGroup : 1;
+    int64_t chunk = (static_cast<int64_t>(1) << 19) / gpr * gpr;
+    if (chunk < gpr)
+        chunk = gpr;
+    if (chunk > G)
+        chunk = G;
+    const int64_t nchunks = (G + chunk - 1) / chunk;
+    const int nslots = nchunks > 1 ? 2 : 1;
+
+    cudaStream_t ss[2] = {nullptr, nullptr};
+    cudaEvent_t ev_start = nullptr, ev_d = nullptr;
+    void *dW[2] = {nullptr, nullptr}, *dD[2] = {nullptr, nullptr}, *dS[2] = {nullptr, nullptr},
+         *dC[2] = {nullptr, nullptr}, *dWs[2] = {nullptr, nullptr};
+    void *dDcol = nullptr;
+    cudaError_t err = cudaSuccess;
+    const size_t wsb = workspace_bytes(chunk);
+    const size_t dcol_bytes = K > 0 ? static_cast<size_t>(E) * K * sizeof(float) : 0;
+    const size_t dgrp_bytes = K > 0 ? 0 : static_cast<size_t>(E) * chunk * kGroup * sizeof(float);
+
+#define CQ_TRY(x)              \
+    do {                       \
+        err = (x);             \
+        if (err != cudaSuccess) \
+            goto done;         \
+    } while (0)
+
+    CQ_TRY(cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming));
+    CQ_TRY(cudaEventCreateWithFlags(&ev_d, cudaEventDisableTiming));
+    for (int k = 0; k < nslots; k++)
+        CQ_TRY(cudaStreamCreateWithFlags(&ss[k], cudaStreamNonBlocking));
+    CQ_TRY(cudaEventRecord(ev_start, user));
+    for (int k = 0; k < nslots; k++) {
+        CQ_TRY(cudaStreamWaitEvent(ss[k], ev_start, 0));
+        CQ_TRY(pool_alloc(&dW[k], static_cast<size_t>(chunk) * kGroup * sizeof(uint16_t), ss[k]));
+        CQ_TRY(pool_alloc(&dS[k], static_cast<size_t>(chunk) * sizeof(uint16_t) + 256, ss[k]));
+        CQ_TRY(pool_alloc(&dC[k], static_cast<size_t>(chunk) * CQ_WORDS * sizeof(uint32_t), ss[k]));
+        CQ_TRY(pool_alloc(&dWs[k], wsb, ss[k]));
+        if (dgrp_bytes)
+            CQ_TRY(pool_alloc(&dD[k], dgrp_bytes, ss[k]));
+    }
+    if (dcol_bytes) {
+        CQ_TRY(pool_alloc(&dDcol, dcol_bytes, ss[0]));
+        CQ_TRY(cudaMemcpyAsync(dDcol, D_host, dcol_bytes, cudaMemcpyHostToDevice, ss[0]));
+        CQ_TRY(cudaEventRecord(ev_d, ss[0]));
+        if (nslots > 1)
+            CQ_TRY(cudaStreamWaitEvent(ss[1], ev_d, 0));
+    }
+    for (int64_t c = 0; c < nchunks; c++) {
+        const int k = static_cast<int>(c % nslots);
+        cudaStream_t s = ss[k];
+        const int64_t g0 = c * chunk;
+        const int64_t n = (G - g0) < chunk ? (G - g0) : chunk;
+        CQ_TRY(cudaMemcpyAsync(dW[k], W_host + g0 * kGroup, static_cast<size_t>(n) * kGroup * sizeof(uint16_t),
+                               cudaMemcpyHostToDevice, s));
+        const float *dptr = static_cast<const float *>(dDcol);
+        if (!dcol_bytes) {
+            for (int e = 0; e < E; e++)
+                CQ_TRY(cudaMemcpyAsync(static_cast<float *>(dD[k]) + static_cast<size_t>(e) * n * kGroup,
+                                       D_host + (static_cast<size_t>(e) * G + g0) * kGroup,
+                                       static_cast<size_t>(n) * kGroup * sizeof(float), cudaMemcpyHostToDevice, s));
+            dptr = static_cast<const float *>(dD[k]);
+        }
+        st = cq_select_scales_ex(static_cast<const uint16_t *>(dW[k]), n, dptr, E, K,
+                                 static_cast<uint16_t *>(dS[k]), static_cast<uint32_t *>(dC[k]), s, nullptr, dWs[k],
+                                 wsb, nullptr, nullptr);
+        if (st != CQ_OK)
+            goto done;
+        CQ_TRY(cudaMemcpyAsync(out_scales_host + g0, dS[k], static_cast<size_t>(n) * sizeof(uint16_t),
+                               cudaMemcpyDeviceToHost, s));
+        CQ_TRY(cudaMemcpyAsync(out_codes_host + g0 * CQ_WORDS, dC[k],
+                               static_cast<size_t>(n) * CQ_WORDS * sizeof(uint32_t), cudaMemcpyDeviceToHost, s));
+    }
+done:
+    for (int k = 0; k < nslots; k++) {
+        if (!ss[k])
+            continue;
+        void *bufs[5] = {dW[k], dS[k], dC[k], dWs[k], dD[k]};
+        for (void *b : bufs)
+            if (b)
+                cudaFreeAsync(b, ss[k]);
+    }
+    if (dDcol)
+        cudaFreeAsync(dDcol, ss[0]);
+    for (int k = 0; k < nslots; k++) {
+        if (ss[k]) {
+            if (cudaStreamSynchronize(ss[k]) != cudaSuccess && err == cudaSuccess)
+                err = cudaErrorUnknown;
+            cudaStreamDestroy(ss[k]);
+        }
+    }
+    if (ev_start)
+        cudaEventDestroy(ev_start);
+    if (ev_d)
+        cudaEventDestroy(ev_d);
+#undef CQ_TRY
+    if (st != CQ_OK)
+        return st;
+    return err == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
+}
+
+cq_status cq_read_counters(const void *workspace, uint32_t *host_counters, void *stream)
+{
+    if (!workspace || !host_counters)
+        return CQ_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(host_counters, workspace, CQ_NUM_COUNTERS * sizeof(uint32_t), cudaMemcpyDeviceToHost, s) !=
+        cudaSuccess)
+        return CQ_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess)
+        return CQ_ERR_CUDA;
+    return host_counters[CQ_CNT_NONFINITE] ? CQ_ERR_NONFINITE : CQ_OK;
+}
+
+const char *cq_status_string(cq_status status)
+{
+    switch (status) {
+    case CQ_OK: return "CQ_OK";
+    case CQ_ERR_INVALID_ARG: return "CQ_ERR_INVALID_ARG: null pointer, bad size, layout or alignment";
+    case CQ_ERR_UNSUPPORTED: return "CQ_ERR_UNSUPPORTED: E above 8 or G at or above 2^32";
+    case CQ_ERR_CUDA: return "CQ_ERR_CUDA: a CUDA runtime call failed";
+    case CQ_ERR_NONFINITE: return "CQ_ERR_NONFINITE: non-finite or negative input in some group";
+    case CQ_ERR_WORKSPACE: return "CQ_ERR_WORKSPACE: workspace missing, too small or misaligned";
+    default: return "unknown cq_status";
+    }
+}
+
+int cq_version(void)
+{
+    return 100;
+}
+
+}  // extern "C"

@@ -1,0 +1,103 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/cq.h declares, and rejects bad arguments before enqueuing anything."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "cq.h")
+
+
+@pytest.fixture(scope="module")
+def cq():
+    from minimax_scale_search_b200 import build
+    build.build()
+    from minimax_scale_search_b200 import cq as mod
+    return mod
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(cq_\w+)\s*\(", src, flags=re.M)
+
+
+def test_header_declares_expected_entry_points(cq):
+    names = declared_functions()
+    assert set(names) == set(cq.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(cq):
+    out = subprocess.run(["nm", "-D", "--defined-only", cq.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if ln.strip()}
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(cq.lib, name)
+
+
+def test_status_strings_and_version(cq):
+    assert cq.status_string(0) == "CQ_OK"
+    for st in range(1, 6):
+        assert cq.status_string(st).startswith("CQ_ERR_")
+    assert "unknown" in cq.status_string(99)
+    assert cq.version() >= 100
+
+
+def test_workspace_size(cq):
+    assert cq.workspace_bytes(0, 4) == 256
+    assert cq.workspace_bytes(1, 4) == 512
+    assert cq.workspace_bytes(3883008, 4) == 256 + 3883008 * 4
+
+
+FAKE = 0x10000  # 16-byte aligned fake device address: every call below fails validation first
+
+
+def call_ex(cq, W=FAKE, G=8, D=FAKE, E=4, K=0, S=FAKE, C=FAKE, opts=None, ws=FAKE, wsb=1 << 20):
+    vp = ctypes.c_void_p
+    return cq.lib.cq_select_scales_ex(vp(W), G, vp(D), E, K, vp(S), vp(C), vp(None),
+                                      ctypes.byref(opts) if opts is not None else None, vp(ws), wsb,
+                                      vp(None), vp(None))
+
+
+def test_argument_errors_are_synchronous(cq):
+    assert call_ex(cq, E=0) == cq.CQ_ERR_INVALID_ARG
+    assert call_ex(cq, E=9) == cq.CQ_ERR_UNSUPPORTED
+    assert call_ex(cq, G=-1) == cq.CQ_ERR_INVALID_ARG
+    assert call_ex(cq, K=-128) == cq.CQ_ERR_INVALID_ARG
+    assert call_ex(cq, K=100) == cq.CQ_ERR_INVALID_ARG          # K % 128 != 0
+    assert call_ex(cq, G=9, K=256) == cq.CQ_ERR_INVALID_ARG     # G not whole rows of K/128 groups
+    assert call_ex(cq, G=1 << 32) == cq.CQ_ERR_UNSUPPORTED
+    assert call_ex(cq, W=0) == cq.CQ_ERR_INVALID_ARG
+    assert call_ex(cq, D=0) == cq.CQ_ERR_INVALID_ARG
+    assert call_ex(cq, S=0) == cq.CQ_ERR_INVALID_ARG
+    assert call_ex(cq, C=0) == cq.CQ_ERR_INVALID_ARG
+    assert call_ex(cq, W=FAKE + 8) == cq.CQ_ERR_INVALID_ARG     # W not 16-byte aligned
+    assert call_ex(cq, D=FAKE + 4) == cq.CQ_ERR_INVALID_ARG
+    assert call_ex(cq, C=FAKE + 2) == cq.CQ_ERR_INVALID_ARG
+    assert call_ex(cq, ws=0) == cq.CQ_ERR_WORKSPACE
+    assert call_ex(cq, wsb=100) == cq.CQ_ERR_WORKSPACE
+    assert call_ex(cq, ws=FAKE + 16) == cq.CQ_ERR_WORKSPACE     # not 256-byte aligned
+    assert call_ex(cq, opts=cq.Opts(65, 0, 0.0, None, None)) == cq.CQ_ERR_INVALID_ARG
+    assert call_ex(cq, opts=cq.Opts(-1, 0, 0.0, None, None)) == cq.CQ_ERR_INVALID_ARG
+    assert call_ex(cq, opts=cq.Opts(0, 0, -1.0, None, None)) == cq.CQ_ERR_INVALID_ARG
+
+
+def test_plain_and_host_entry_points_validate(cq):
+    vp = ctypes.c_void_p
+    assert cq.lib.cq_select_scales(vp(FAKE), 8, vp(FAKE), 0, 0, vp(FAKE), vp(FAKE), vp(None)) == \
+        cq.CQ_ERR_INVALID_ARG
+    assert cq.lib.cq_select_scales(vp(None), 0, vp(None), 4, 0, vp(None), vp(None), vp(None)) == cq.CQ_OK
+    assert cq.lib.cq_select_scales_host(vp(None), 8, vp(FAKE), 4, 0, vp(FAKE), vp(FAKE), vp(None)) == \
+        cq.CQ_ERR_INVALID_ARG
+    assert cq.lib.cq_select_scales_host(vp(None), 0, vp(None), 4, 0, vp(None), vp(None), vp(None)) == cq.CQ_OK
+    assert cq.lib.cq_read_counters(vp(None), vp(FAKE), vp(None)) == cq.CQ_ERR_INVALID_ARG
+
+
+def test_no_cpu_fallback_in_binding():
+    """The binding refuses to run without its CUDA library."""
+    src = open(os.path.join(ROOT, "minimax_scale_search_b200", "cq.py")).read()
+    assert "import oracle" not in src and "from oracle" not in src
+    assert "raise ImportError" in src
