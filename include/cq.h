@@ -67,7 +67,7 @@ enum {
     CQ_CNT_FINALISTS = 4,    /* total fp64-rescored candidate scales */
     CQ_CNT_UNCERTAIN = 5,    /* runs whose screen could not be certified */
     CQ_CNT_QUEUE = 6,        /* internal: fallback queue length */
-    CQ_CNT_RESERVED = 7
+    CQ_CNT_SURVIVORS = 7     /* runs that passed the fp32 screen (summed over groups) */
 };
 
 /* Per-group flag bits written to out_flags. */

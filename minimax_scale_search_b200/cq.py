@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libcq.so")
 
 CQ_OK, CQ_ERR_INVALID_ARG, CQ_ERR_UNSUPPORTED, CQ_ERR_CUDA, CQ_ERR_NONFINITE, CQ_ERR_WORKSPACE = range(6)
 CQ_NUM_COUNTERS = 8
-COUNTER_NAMES = ("fallback", "near_tie", "nonfinite", "trivial", "finalists", "uncertain", "queue", "reserved")
+COUNTER_NAMES = ("fallback", "near_tie", "nonfinite", "trivial", "finalists", "uncertain", "queue", "survivors")
 FLAG_TRIVIAL, FLAG_FALLBACK, FLAG_NEAR_TIE, FLAG_NONFINITE = 0x01, 0x02, 0x04, 0x08
 GROUP = 128
 WORDS = 16

@@ -54,11 +54,12 @@ namespace cq {
 constexpr int kGroup = 128;
 constexpr uint32_t kLast = 0x7BFFu;    // largest finite binary16 pattern (65504)
 constexpr uint32_t kBeyond = 0x7C00u;  // one past the grid
-constexpr int kWarps = 8;              // warps (groups in flight) per CTA of the main kernel
+constexpr int kWarps = 4;              // warps (groups in flight) per CTA of the main kernel
 constexpr int kKeys = 1024;            // 128 weights x up to 8 transitions
 constexpr uint32_t kInvalidKey = 0xFFFFFFFFu;
 constexpr int kMaxFinalists = 64;
 constexpr int kDefaultFinalists = 32;
+constexpr int kMaxSurvivors = 128;  // runs passing the fp32 screen before the exhaustive fallback
 constexpr uint32_t kUncertainBit = 0x8000u;
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
@@ -149,48 +150,86 @@ __device__ __forceinline__ T warp_sum(T v)
     return v;
 }
 
+__device__ __forceinline__ void cx_asc(uint32_t &a, uint32_t &b)
+{
+    const uint32_t lo = min(a, b);
+    b = max(a, b);
+    a = lo;
+}
+
 // Ascending bitonic sort of 1024 keys, blocked layout: lane L holds positions
-// 32L .. 32L+31 in key[0..31].
+// 32L .. 32L+31 in key[0..31].  Blocks of up to 16 keys sort inside a lane with
+// compile-time directions.  For the larger block sizes the lanes whose block
+// runs descending complement their keys (an order-reversing bijection), so
+// every compare-exchange of the level is ascending, and complement back after.
 __device__ __forceinline__ void bitonic_sort_1024(uint32_t (&key)[32], int lane)
 {
 #pragma unroll
-    for (int k = 2; k <= kKeys; k <<= 1) {
+    for (int k = 2; k <= 16; k <<= 1) {
 #pragma unroll
         for (int j = k >> 1; j > 0; j >>= 1) {
-            if (j >= 32) {
-                const int lm = j >> 5;
-                const bool upper = (lane & lm) != 0;
-                const bool asc = ((32 * lane) & k) == 0;
-                const bool keep_min = (asc != upper);
 #pragma unroll
-                for (int x = 0; x < 32; x++) {
-                    const uint32_t other = __shfl_xor_sync(kFull, key[x], lm);
-                    key[x] = keep_min ? min(key[x], other) : max(key[x], other);
-                }
-            } else {
-#pragma unroll
-                for (int x = 0; x < 32; x++) {
-                    const int y = x ^ j;
-                    if (y > x) {
-                        const bool asc = (k >= 32) ? (((32 * lane) & k) == 0) : ((x & k) == 0);
-                        const uint32_t a = key[x], b = key[y];
-                        const uint32_t lo = min(a, b), hi = max(a, b);
-                        key[x] = asc ? lo : hi;
-                        key[y] = asc ? hi : lo;
-                    }
+            for (int x = 0; x < 32; x++) {
+                const int y = x ^ j;
+                if (y > x) {
+                    if ((x & k) == 0)
+                        cx_asc(key[x], key[y]);
+                    else
+                        cx_asc(key[y], key[x]);
                 }
             }
         }
     }
+#pragma unroll 1
+    for (int k = 32; k <= kKeys; k <<= 1) {
+        const uint32_t flip = (((32 * lane) & k) != 0) ? 0xFFFFFFFFu : 0u;
+#pragma unroll
+        for (int x = 0; x < 32; x++)
+            key[x] ^= flip;
+#pragma unroll 1
+        for (int lm = k >> 6; lm > 0; lm >>= 1) {
+            const bool upper = (lane & lm) != 0;
+#pragma unroll
+            for (int x = 0; x < 32; x++) {
+                const uint32_t o = __shfl_xor_sync(kFull, key[x], lm);
+                key[x] = upper ? max(key[x], o) : min(key[x], o);
+            }
+        }
+#pragma unroll
+        for (int j = 16; j > 0; j >>= 1) {
+#pragma unroll
+            for (int x = 0; x < 32; x++) {
+                const int y = x ^ j;
+                if (y > x)
+                    cx_asc(key[x], key[y]);
+            }
+        }
+#pragma unroll
+        for (int x = 0; x < 32; x++)
+            key[x] ^= flip;
+    }
 }
+
+// Coefficients of one surviving run, handed from the lane that owns its
+// position to the lane that searches it.
+template <int E>
+struct SurvEntry {
+    double B[E];
+    double C[E];
+    uint32_t ja, jb;
+};
 
 template <int E>
 struct WarpSmem {
     float d[E][kGroup];
     float w[kGroup];
     uint32_t keys[kKeys];
-    float lb[kKeys + 1];          // certified lower bound of each run's minimum
-    uint16_t jf[kKeys + 2];       // each run's minimiser | kUncertainBit
+    union {
+        float lb[kKeys + 1];          // fp32-screen lower bound of each run's minimum
+        SurvEntry<E> ent[32];         // one batch of surviving runs
+    } u;
+    float res_lb[kMaxSurvivors];      // certified lower bound of each survivor's minimum
+    uint16_t res_j[kMaxSurvivors];    // its minimiser | kUncertainBit
     int fin[kMaxFinalists];
 };
 
@@ -277,6 +316,40 @@ __device__ RunResult solve_run(const double (&A)[E], const double (&B)[E], const
     return r;
 }
 
+// fp32 screen of one run [ja, jb]: a lower bound of min_s max_e F_e (the max
+// over e of each environment's minimum, at its clamped vertex B/C) and an
+// upper bound (max_e F_e at the grid point nearest the binding vertex), each
+// widened by 2^-16 of max_e (A + 2Bs + Cs^2) at the run's right end.  The
+// coefficients carry at most ~40 fp32 roundings of relative size 2^-24 and
+// the evaluation three more, so the true values lie inside the widened bounds.
+template <int E>
+__device__ __forceinline__ void screen_run32(const float (&A)[E], const float (&B)[E], const float (&C)[E],
+                                             uint32_t ja, uint32_t jb, float &lbm, float &ubm)
+{
+    const float sa = half_value(ja), sb = half_value(jb);
+    float L = -INFINITY, vstar = sa, P = 0.0f;
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        const float v = fminf(fmaxf(__fdividef(B[e], C[e]), sa), sb);
+        const float f = fmaf(fmaf(C[e], v, -2.0f * B[e]), v, A[e]);
+        if (f > L) {
+            L = f;
+            vstar = v;
+        }
+        P = fmaxf(P, fmaf(fmaf(C[e], sb, 2.0f * B[e]), sb, A[e]));
+    }
+    uint32_t jc = __half_as_ushort(__float2half_rn(vstar));
+    jc = min(max(jc, ja), jb);
+    const float s = half_value(jc);
+    float U = fmaf(fmaf(C[0], s, -2.0f * B[0]), s, A[0]);
+#pragma unroll
+    for (int e = 1; e < E; e++)
+        U = fmaxf(U, fmaf(fmaf(C[e], s, -2.0f * B[e]), s, A[e]));
+    const float m = P * 0x1p-16f;
+    lbm = L - m;
+    ubm = U + m;
+}
+
 // Best two objectives within rel of each other (an exact tie always counts).
 __device__ __forceinline__ bool near_tie(double best, double second, double rel)
 {
@@ -319,6 +392,34 @@ __device__ __forceinline__ void enqueue(const Params &p, int64_t g, int lane)
         const uint32_t at = atomicAdd(&p.counters[CQ_CNT_QUEUE], 1u);
         p.queue[at] = static_cast<uint32_t>(g);
         atomicAdd(&p.counters[CQ_CNT_FALLBACK], 1u);
+    }
+}
+
+template <int E>
+__device__ __forceinline__ void add_delta(const WarpSmem<E> &sm, uint32_t kk, double (&RB)[E], double (&RC)[E])
+{
+    const int i = (kk >> 3) & 127;
+    const double aw = fabs(static_cast<double>(sm.w[i]));
+    const double c = static_cast<double>(2 * (kk & 7) + 1);
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        const double dd = sm.d[e][i];
+        RB[e] += dd * aw;  // exact terms: 24-bit d times 11-bit |w|, 24-bit d times odd <= 15
+        RC[e] += dd * c;
+    }
+}
+
+template <int E>
+__device__ __forceinline__ void add_delta32(const WarpSmem<E> &sm, uint32_t kk, float (&RB)[E], float (&RC)[E])
+{
+    const int i = (kk >> 3) & 127;
+    const float aw = fabsf(sm.w[i]);
+    const float c = static_cast<float>(2 * (kk & 7) + 1);
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        const float dd = sm.d[e][i];
+        RB[e] = fmaf(dd, aw, RB[e]);
+        RC[e] = fmaf(dd, c, RC[e]);
     }
 }
 
@@ -368,6 +469,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
 
     // ---- 2. A_e = sum d w^2 (exact terms) -------------------------------
     double A[E];
+    float Af[E];
 #pragma unroll
     for (int e = 0; e < E; e++) {
         double a = 0.0;
@@ -375,6 +477,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         for (int m = 0; m < 4; m++)
             a += static_cast<double>(dr[e][m]) * (static_cast<double>(wf[m]) * static_cast<double>(wf[m]));
         A[e] = warp_sum(a);
+        Af[e] = static_cast<float>(A[e]);
     }
 
     // ---- 3. transitions -------------------------------------------------
@@ -393,38 +496,27 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
 
     // ---- 4. order -------------------------------------------------------
     bitonic_sort_1024(key, lane);
+#pragma unroll
+    for (int x = 0; x < 32; x++)
+        sm.keys[swz(32 * lane + x)] = key[x];
+    __syncwarp();
 
     // ---- 5. coefficient scan: lane totals, then suffix across lanes ----
-    double TB[E], TC[E];
+    double RB0[E], RC0[E];
 #pragma unroll
     for (int e = 0; e < E; e++) {
-        TB[e] = 0.0;
-        TC[e] = 0.0;
+        RB0[e] = 0.0;
+        RC0[e] = 0.0;
     }
-#pragma unroll
-    for (int x = 0; x < 32; x++) {
-        sm.keys[swz(32 * lane + x)] = key[x];
-    }
-    __syncwarp();
 #pragma unroll 4
     for (int x = 0; x < 32; x++) {
         const uint32_t kk = sm.keys[swz(32 * lane + x)];
-        if (kk != kInvalidKey) {
-            const int i = (kk >> 3) & 127;
-            const double aw = fabs(static_cast<double>(sm.w[i]));
-            const double c = static_cast<double>(2 * (kk & 7) + 1);
-#pragma unroll
-            for (int e = 0; e < E; e++) {
-                const double dd = sm.d[e][i];
-                TB[e] += dd * aw;
-                TC[e] += dd * c;
-            }
-        }
+        if (kk != kInvalidKey)
+            add_delta<E>(sm, kk, RB0, RC0);
     }
-    double RB[E], RC[E];
 #pragma unroll
     for (int e = 0; e < E; e++) {
-        double vb = TB[e], vc = TC[e];
+        double vb = RB0[e], vc = RC0[e];
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const double ub = __shfl_down_sync(kFull, vb, o);
@@ -436,109 +528,183 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         }
         const double xb = __shfl_down_sync(kFull, vb, 1);
         const double xc = __shfl_down_sync(kFull, vc, 1);
-        RB[e] = (lane == 31) ? 0.0 : xb;
-        RC[e] = (lane == 31) ? 0.0 : xc;
+        RB0[e] = (lane == 31) ? 0.0 : xb;  // sum over every position after this lane's chunk
+        RC0[e] = (lane == 31) ? 0.0 : xc;
     }
-
-    // ---- 6. runs ----------------------------------------------------------
-    uint32_t next_t = kBeyond;
+    uint32_t t_after = kBeyond;  // t of the first position after this lane's chunk
     {
         const uint32_t kn = (lane < 31) ? sm.keys[swz(32 * lane + 32)] : kInvalidKey;
         if (kn != kInvalidKey)
-            next_t = kn >> 10;
+            t_after = kn >> 10;
     }
-    double ub_min = INFINITY;
+
+    // ---- 6. fp32 screen of every run ----------------------------------
+    float rbf[E], rcf[E];
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        rbf[e] = static_cast<float>(RB0[e]);
+        rcf[e] = static_cast<float>(RC0[e]);
+    }
+    float ub_lane = INFINITY;
+    uint32_t next_t = t_after;
     for (int x = 31; x >= 0; --x) {
         const int pos = 32 * lane + x;
         const uint32_t kk = sm.keys[swz(pos)];
         float lbv = INFINITY;
-        uint32_t jv = 0;
         if (kk != kInvalidKey) {
             const uint32_t t = kk >> 10;
             if (t <= kLast && t != next_t) {
-                const RunResult rr = solve_run<E>(A, RB, RC, t, min(next_t, kBeyond) - 1u);
-                lbv = rr.lb;
-                jv = rr.j | (rr.uncertain ? kUncertainBit : 0u);
-                ub_min = fmin(ub_min, rr.ub);
+                float ubv;
+                screen_run32<E>(Af, rbf, rcf, t, min(next_t, kBeyond) - 1u, lbv, ubv);
+                ub_lane = fminf(ub_lane, ubv);
             }
-            const int i = (kk >> 3) & 127;
-            const double aw = fabs(static_cast<double>(sm.w[i]));
-            const double c = static_cast<double>(2 * (kk & 7) + 1);
-#pragma unroll
-            for (int e = 0; e < E; e++) {
-                const double dd = sm.d[e][i];
-                RB[e] += dd * aw;
-                RC[e] += dd * c;
-            }
+            add_delta32<E>(sm, kk, rbf, rcf);
             next_t = t;
         }
-        sm.lb[swz(pos)] = lbv;
-        sm.jf[swz(pos)] = static_cast<uint16_t>(jv);
+        sm.u.lb[swz(pos)] = lbv;
     }
+    const uint32_t t_first = next_t;  // lane 0: t of position 0
     if (lane == 0) {
-        // the run below every transition: [1, t_0 - 1], all transitions active
         float lbv = INFINITY;
-        uint32_t jv = 0;
-        if (next_t > 1u) {
-            const RunResult rr = solve_run<E>(A, RB, RC, 1u, min(next_t, kBeyond) - 1u);
-            lbv = rr.lb;
-            jv = rr.j | (rr.uncertain ? kUncertainBit : 0u);
+        if (t_first > 1u) {
+            float ubv;
+            screen_run32<E>(Af, rbf, rcf, 1u, min(t_first, kBeyond) - 1u, lbv, ubv);
+            ub_lane = fminf(ub_lane, ubv);
+        }
+        sm.u.lb[kKeys] = lbv;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        ub_lane = fminf(ub_lane, __shfl_xor_sync(kFull, ub_lane, o));
+    // survivors: runs whose screened lower bound reaches the best screened upper bound
+    const float U = ub_lane * (1.0f + 0x1p-20f);
+    __syncwarp();
+    uint32_t smask = 0;
+    for (int x = 0; x < 32; x++)
+        smask |= (sm.u.lb[swz(32 * lane + x)] <= U ? 1u : 0u) << x;
+    const bool init_surv = (lane == 0) && (sm.u.lb[kKeys] <= U);
+    const int my_surv = __popc(smask) + (init_surv ? 1 : 0);
+    int excl = my_surv;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(kFull, excl, o);
+        if (lane >= o)
+            excl += v;
+    }
+    const int n_surv = __shfl_sync(kFull, excl, 31);
+    excl -= my_surv;
+    if (n_surv > kMaxSurvivors) {
+        enqueue(p, g, lane);
+        return;
+    }
+    __syncwarp();
+
+    // ---- 7. certified fp64 search of the survivors, 32 at a time -------
+    double ub_min = INFINITY;
+    for (int base = 0; base < n_surv; base += 32) {
+        if (my_surv > 0 && excl < base + 32 && excl + my_surv > base) {
+            double RB[E], RC[E];
+#pragma unroll
+            for (int e = 0; e < E; e++) {
+                RB[e] = RB0[e];
+                RC[e] = RC0[e];
+            }
+            int r = excl;
+            uint32_t nt = t_after;
+            for (int x = 31; x >= 0; --x) {
+                const uint32_t kk = sm.keys[swz(32 * lane + x)];
+                if (kk == kInvalidKey)
+                    continue;
+                const uint32_t t = kk >> 10;
+                if ((smask >> x) & 1u) {
+                    if (r >= base && r < base + 32) {
+                        SurvEntry<E> &en = sm.u.ent[r - base];
+#pragma unroll
+                        for (int e = 0; e < E; e++) {
+                            en.B[e] = RB[e];
+                            en.C[e] = RC[e];
+                        }
+                        en.ja = t;
+                        en.jb = min(nt, kBeyond) - 1u;
+                    }
+                    r++;
+                }
+                add_delta<E>(sm, kk, RB, RC);
+                nt = t;
+            }
+            if (init_surv && r >= base && r < base + 32) {
+                SurvEntry<E> &en = sm.u.ent[r - base];
+#pragma unroll
+                for (int e = 0; e < E; e++) {
+                    en.B[e] = RB[e];
+                    en.C[e] = RC[e];
+                }
+                en.ja = 1u;
+                en.jb = min(t_first, kBeyond) - 1u;
+            }
+        }
+        __syncwarp();
+        const int me = base + lane;
+        if (me < n_surv) {
+            const SurvEntry<E> &en = sm.u.ent[lane];
+            double Bv[E], Cv[E];
+#pragma unroll
+            for (int e = 0; e < E; e++) {
+                Bv[e] = en.B[e];
+                Cv[e] = en.C[e];
+            }
+            const RunResult rr = solve_run<E>(A, Bv, Cv, en.ja, en.jb);
+            sm.res_lb[me] = rr.lb;
+            sm.res_j[me] = static_cast<uint16_t>(rr.j | (rr.uncertain ? kUncertainBit : 0u));
             ub_min = fmin(ub_min, rr.ub);
         }
-        sm.lb[kKeys] = lbv;
-        sm.jf[kKeys] = static_cast<uint16_t>(jv);
+        __syncwarp();
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
         ub_min = fmin(ub_min, __shfl_xor_sync(kFull, ub_min, o));
     const float T = __double2float_ru(ub_min * (1.0 + 0x1p-40));
-    __syncwarp();
 
-    // ---- 7. finalists -----------------------------------------------------
+    // ---- 8. finalists ---------------------------------------------------
     int cnt = 0;
     bool unc_comp = false, unc_any = false;
-    for (int x = 0; x < 33; x++) {
-        if (x == 32 && lane != 0)
-            break;
-        const int at = (x == 32) ? kKeys : swz(32 * lane + x);
-        const uint32_t jv = sm.jf[at];
-        unc_any |= (jv & kUncertainBit) != 0u && sm.lb[at] < INFINITY;
-        if (sm.lb[at] <= T) {
+    for (int me = lane; me < n_surv; me += 32) {
+        const uint32_t jv = sm.res_j[me];
+        const bool in = sm.res_lb[me] <= T;
+        unc_any |= (jv & kUncertainBit) != 0u;
+        if (in) {
             if (jv & kUncertainBit)
                 unc_comp = true;
             else
                 cnt++;
         }
     }
+    if (lane == 0) {
+        atomicAdd(&p.counters[CQ_CNT_SURVIVORS], static_cast<uint32_t>(n_surv));
+    }
     if (__any_sync(kFull, unc_any) && lane == 0)
         atomicAdd(&p.counters[CQ_CNT_UNCERTAIN], 1u);
     unc_comp = __any_sync(kFull, unc_comp);
-    int excl = cnt;
+    int fx = cnt;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(kFull, excl, o);
+        const int u = __shfl_up_sync(kFull, fx, o);
         if (lane >= o)
-            excl += u;
+            fx += u;
     }
-    const int total = __shfl_sync(kFull, excl, 31);
-    excl -= cnt;
+    const int total = __shfl_sync(kFull, fx, 31);
+    fx -= cnt;
     if (unc_comp || total > p.finalist_cap || total == 0) {
         enqueue(p, g, lane);
         return;
     }
-    {
-        int o = excl;
-        for (int x = 0; x < 33; x++) {
-            if (x == 32 && lane != 0)
-                break;
-            const int at = (x == 32) ? kKeys : swz(32 * lane + x);
-            if (sm.lb[at] <= T && !(sm.jf[at] & kUncertainBit))
-                sm.fin[o++] = sm.jf[at];
-        }
+    for (int me = lane; me < n_surv; me += 32) {
+        if (sm.res_lb[me] <= T && !(sm.res_j[me] & kUncertainBit))
+            sm.fin[fx++] = sm.res_j[me];
     }
     __syncwarp();
 
-    // ---- 8. fp64 rescoring of the finalists -------------------------------
+    // ---- 9. fp64 rescoring of the finalists -------------------------------
     int Kc[4];
 #pragma unroll
     for (int m = 0; m < 4; m++)
@@ -576,7 +742,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         }
     }
 
-    // ---- 9. pack and store ------------------------------------------------
+    // ---- 10. pack and store -------------------------------------------------
     const float s = half_value(bj);
     int q[4];
 #pragma unroll
@@ -601,7 +767,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
 }
 
 template <int E>
-__global__ void __launch_bounds__(kWarps * 32) select_kernel(Params p)
+__global__ void __launch_bounds__(kWarps * 32, (E <= 4 ? 4 : 2)) select_kernel(Params p)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int lane = threadIdx.x & 31;
