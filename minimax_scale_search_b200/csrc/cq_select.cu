@@ -55,11 +55,11 @@ constexpr int kGroup = 128;
 constexpr uint32_t kLast = 0x7BFFu;    // largest finite binary16 pattern (65504)
 constexpr uint32_t kBeyond = 0x7C00u;  // one past the grid
 constexpr int kWarps = 4;              // warps (groups in flight) per CTA of the main kernel
-constexpr int kKeys = 1024;            // 128 weights x up to 8 transitions
 constexpr uint32_t kInvalidKey = 0xFFFFFFFFu;
 constexpr int kMaxFinalists = 64;
 constexpr int kDefaultFinalists = 32;
 constexpr int kMaxSurvivors = 128;  // runs passing the fp32 screen before the exhaustive fallback
+constexpr int kWalkMax = 16;        // longest delta walk between survivors before a direct sum
 constexpr uint32_t kUncertainBit = 0x8000u;
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
@@ -85,6 +85,18 @@ struct Params {
 __device__ __forceinline__ float half_value(uint32_t bits)
 {
     return __half2float(__ushort_as_half(static_cast<unsigned short>(bits)));
+}
+
+// Value of a positive binary16 pattern j in [1, 0x7C00] (0x7C00 gives 65536),
+// built from bits without a conversion instruction: for j >= 0x400 the fp32
+// pattern is (j << 13) + 0x38000000; for subnormal halves the same construction
+// with the exponent one higher gives 2^-14 + j 2^-24, and 2^-14 is subtracted
+// exactly.
+__device__ __forceinline__ float grid_value(uint32_t j)
+{
+    const bool sub = j < 0x400u;
+    const float v = __uint_as_float((j << 13) + (sub ? 0x38800000u : 0x38000000u));
+    return sub ? v - 0x1p-14f : v;
 }
 
 __device__ __forceinline__ const float *diag_ptr(const Params &p, int64_t g, int e)
@@ -115,30 +127,27 @@ __device__ __forceinline__ int abs_code(float aw, float s, int K)
     return min(n, K);
 }
 
+// 1 / (k + 1/2), k = 0..7 (only an estimate's accuracy is needed).
+__constant__ float c_inv_half[8] = {2.0f, 2.0f / 3.0f, 2.0f / 5.0f, 2.0f / 7.0f,
+                                    2.0f / 9.0f, 2.0f / 11.0f, 2.0f / 13.0f, 2.0f / 15.0f};
+
 // Smallest grid index j in [1, kBeyond] with |q(s_j)| <= k, kBeyond meaning
 // "still above k at 65504".  The fp32 estimate |w|/(k+1/2) rounded up to
-// binary16 is at most one pattern away from the answer.
-template <int k>
-__device__ __forceinline__ uint32_t transition_index(float aw)
+// binary16 is at most one pattern away from the answer, which the exact
+// threshold tests then fix.
+__device__ __forceinline__ uint32_t transition_index(float aw, int k)
 {
-    constexpr float inv = 2.0f / static_cast<float>(2 * k + 1);
-    const float x = aw * inv;
+    const float x = aw * c_inv_half[k];
     uint32_t j0 = __half_as_ushort(__float2half_ru(x));
     if (j0 > kBeyond)
         j0 = kBeyond;
     if (j0 < 1u)
         j0 = 1u;
-    if (j0 > 1u && !code_at_least(aw, half_value(j0 - 1), k + 1))
+    if (j0 > 1u && !code_at_least(aw, grid_value(j0 - 1), k + 1))
         return j0 - 1;
-    if (j0 == kBeyond || !code_at_least(aw, half_value(j0), k + 1))
+    if (j0 == kBeyond || !code_at_least(aw, grid_value(j0), k + 1))
         return j0;
     return j0 + 1;
-}
-
-// Bank-conflict-free placement of position p = 32*lane + x in a per-warp array.
-__device__ __forceinline__ int swz(int p)
-{
-    return (p & ~31) | ((p ^ (p >> 5)) & 31);
 }
 
 template <typename T>
@@ -157,80 +166,107 @@ __device__ __forceinline__ void cx_asc(uint32_t &a, uint32_t &b)
     a = lo;
 }
 
-// Ascending bitonic sort of 1024 keys, blocked layout: lane L holds positions
-// 32L .. 32L+31 in key[0..31].  Blocks of up to 16 keys sort inside a lane with
-// compile-time directions.  For the larger block sizes the lanes whose block
-// runs descending complement their keys (an order-reversing bijection), so
-// every compare-exchange of the level is ascending, and complement back after.
-__device__ __forceinline__ void bitonic_sort_1024(uint32_t (&key)[32], int lane)
+// Ascending bitonic sort of 128 keys, blocked layout: lane L holds positions
+// 4L .. 4L+3 in key[0..3].  Block size 2 sorts inside a lane with compile-time
+// directions; for larger blocks the lanes whose block runs descending
+// complement their keys (an order-reversing bijection), so every
+// compare-exchange of the level is ascending, and complement back after.
+__device__ __forceinline__ void bitonic_sort_128(uint32_t (&key)[4], int lane)
 {
+    cx_asc(key[0], key[1]);
+    cx_asc(key[3], key[2]);
 #pragma unroll
-    for (int k = 2; k <= 16; k <<= 1) {
+    for (int k = 4; k <= kGroup; k <<= 1) {
+        const uint32_t flip = (((4 * lane) & k) != 0) ? 0xFFFFFFFFu : 0u;
 #pragma unroll
-        for (int j = k >> 1; j > 0; j >>= 1) {
-#pragma unroll
-            for (int x = 0; x < 32; x++) {
-                const int y = x ^ j;
-                if (y > x) {
-                    if ((x & k) == 0)
-                        cx_asc(key[x], key[y]);
-                    else
-                        cx_asc(key[y], key[x]);
-                }
-            }
-        }
-    }
-#pragma unroll 1
-    for (int k = 32; k <= kKeys; k <<= 1) {
-        const uint32_t flip = (((32 * lane) & k) != 0) ? 0xFFFFFFFFu : 0u;
-#pragma unroll
-        for (int x = 0; x < 32; x++)
+        for (int x = 0; x < 4; x++)
             key[x] ^= flip;
-#pragma unroll 1
-        for (int lm = k >> 6; lm > 0; lm >>= 1) {
+#pragma unroll
+        for (int lm = k >> 3; lm > 0; lm >>= 1) {
             const bool upper = (lane & lm) != 0;
 #pragma unroll
-            for (int x = 0; x < 32; x++) {
+            for (int x = 0; x < 4; x++) {
                 const uint32_t o = __shfl_xor_sync(kFull, key[x], lm);
                 key[x] = upper ? max(key[x], o) : min(key[x], o);
             }
         }
+        cx_asc(key[0], key[2]);
+        cx_asc(key[1], key[3]);
+        cx_asc(key[0], key[1]);
+        cx_asc(key[2], key[3]);
 #pragma unroll
-        for (int j = 16; j > 0; j >>= 1) {
-#pragma unroll
-            for (int x = 0; x < 32; x++) {
-                const int y = x ^ j;
-                if (y > x)
-                    cx_asc(key[x], key[y]);
-            }
-        }
-#pragma unroll
-        for (int x = 0; x < 32; x++)
+        for (int x = 0; x < 4; x++)
             key[x] ^= flip;
     }
 }
 
-// Coefficients of one surviving run, handed from the lane that owns its
-// position to the lane that searches it.
-template <int E>
+// Merge path: number of elements of A among the first d outputs of the merge
+// of ascending A[0..a) and B[0..b) (all keys distinct).
+__device__ __forceinline__ int merge_split(const uint32_t *A, int a, const uint32_t *B, int b, int d)
+{
+    int lo = max(0, d - b), hi = min(d, a);
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (A[mid] < B[d - 1 - mid])
+            lo = mid + 1;
+        else
+            hi = mid;
+    }
+    return lo;
+}
+
+// Outputs [d0, d1) of the merge of A and B (each followed by a kInvalidKey
+// sentinel) written to C[d0 .. d1).
+__device__ __forceinline__ void merge_range(const uint32_t *A, int a, const uint32_t *B, int b, uint32_t *C,
+                                            int d0, int d1)
+{
+    if (d0 >= d1)
+        return;
+    int i = merge_split(A, a, B, b, d0);
+    int j = d0 - i;
+    uint32_t va = A[i], vb = B[j];
+    for (int o = d0; o < d1; o++) {
+        const bool ta = va < vb;
+        C[o] = ta ? va : vb;
+        if (ta)
+            va = A[++i];
+        else
+            vb = B[++j];
+    }
+}
+
+// Grid range [ja, jb] of one surviving run.
 struct SurvEntry {
-    double B[E];
-    double C[E];
     uint32_t ja, jb;
+    int pos;   // sorted-key position of the run's first transition; -1: the run below all
+    int pad;
 };
+
+constexpr int kLayerStride = 130;   // 128 codes + sentinel, per transition layer
+constexpr int kBufWords = 8 * kLayerStride;  // 1040: 8 layers, 4 x 257 or 2 x 513 merge lists, 1024 keys
 
 template <int E>
 struct WarpSmem {
-    float d[E][kGroup];
-    float w[kGroup];
-    uint32_t keys[kKeys];
-    union {
-        float lb[kKeys + 1];          // fp32-screen lower bound of each run's minimum
-        SurvEntry<E> ent[32];         // one batch of surviving runs
-    } u;
-    float res_lb[kMaxSurvivors];      // certified lower bound of each survivor's minimum
-    uint16_t res_j[kMaxSurvivors];    // its minimiser | kUncertainBit
-    int fin[kMaxFinalists];
+    float d[E][kGroup];       // diagonals by rank in ascending |w|
+    float w[kGroup];          // signed weights by rank in ascending |w|
+    // A: transition layers -> level-2 lists -> per-run fp32 lower bounds ->
+    //    survivor ranges + survivor results
+    alignas(16) uint32_t bufA[kBufWords];
+    // B: weight keys -> level-1 lists -> sorted keys (element x of lane L at
+    //    x*32+L) -> finalists
+    alignas(16) uint32_t bufB[kBufWords];
+
+    __device__ float *lb() { return reinterpret_cast<float *>(bufA); }
+    __device__ SurvEntry *ent() { return reinterpret_cast<SurvEntry *>(bufA); }
+    __device__ float *res_lb() { return reinterpret_cast<float *>(bufA + 4 * kMaxSurvivors); }
+    __device__ uint16_t *res_j() { return reinterpret_cast<uint16_t *>(bufA + 5 * kMaxSurvivors); }
+    __device__ int *fin() { return reinterpret_cast<int *>(bufB); }
+};
+
+// Per-warp event counts, flushed to the device counters once per warp.
+struct Tally {
+    uint32_t fallback = 0, near_tie = 0, nonfinite = 0, trivial = 0, finalists = 0, uncertain = 0,
+             survivors = 0;
 };
 
 struct RunResult {
@@ -273,7 +309,7 @@ __device__ RunResult solve_run(const double (&A)[E], const double (&B)[E], const
         r.uncertain = false;
         return r;
     }
-    const double sa = half_value(ja), sb = half_value(jb);
+    const double sa = grid_value(ja), sb = grid_value(jb);
     double P = 0.0, nb2[E];
 #pragma unroll
     for (int e = 0; e < E; e++) {
@@ -285,8 +321,8 @@ __device__ RunResult solve_run(const double (&A)[E], const double (&B)[E], const
     bool unc = false;
     while (lo < hi) {
         const uint32_t mid = (lo + hi) >> 1;
-        const double S0 = screen<E>(A, nb2, C, half_value(mid));
-        const double S1 = screen<E>(A, nb2, C, half_value(mid + 1));
+        const double S0 = screen<E>(A, nb2, C, grid_value(mid));
+        const double S1 = screen<E>(A, nb2, C, grid_value(mid + 1));
         const double Dd = S1 - S0;
         if (fabs(Dd) <= 2.0 * delta + 0x1p-40 * fmax(fabs(S0), fabs(S1)))
             unc = true;
@@ -295,7 +331,7 @@ __device__ RunResult solve_run(const double (&A)[E], const double (&B)[E], const
         else
             lo = mid + 1;
     }
-    const double Sf = screen<E>(A, nb2, C, half_value(lo));
+    const double Sf = screen<E>(A, nb2, C, grid_value(lo));
     r.j = lo;
     r.ub = Sf + delta;
     r.uncertain = unc;
@@ -326,7 +362,7 @@ template <int E>
 __device__ __forceinline__ void screen_run32(const float (&A)[E], const float (&B)[E], const float (&C)[E],
                                              uint32_t ja, uint32_t jb, float &lbm, float &ubm)
 {
-    const float sa = half_value(ja), sb = half_value(jb);
+    const float sa = grid_value(ja), sb = grid_value(jb);
     float L = -INFINITY, vstar = sa, P = 0.0f;
 #pragma unroll
     for (int e = 0; e < E; e++) {
@@ -340,7 +376,7 @@ __device__ __forceinline__ void screen_run32(const float (&A)[E], const float (&
     }
     uint32_t jc = __half_as_ushort(__float2half_rn(vstar));
     jc = min(max(jc, ja), jb);
-    const float s = half_value(jc);
+    const float s = grid_value(jc);
     float U = fmaf(fmaf(C[0], s, -2.0f * B[0]), s, A[0]);
 #pragma unroll
     for (int e = 1; e < E; e++)
@@ -371,8 +407,7 @@ __device__ __forceinline__ uint32_t pack_lane_codes(const int (&q)[4], int lane)
     return h | (up << 16);  // valid on even lanes: codes 8*(lane/2) .. +7
 }
 
-__device__ __forceinline__ void write_constant_group(const Params &p, int64_t g, int lane, uint8_t flag,
-                                                     int counter)
+__device__ __forceinline__ void write_constant_group(const Params &p, int64_t g, int lane, uint8_t flag)
 {
     if (lane < 16)
         p.out_codes[g * 16 + lane] = 0x88888888u;
@@ -382,186 +417,302 @@ __device__ __forceinline__ void write_constant_group(const Params &p, int64_t g,
             p.out_obj[g] = 0.0;
         if (p.out_flags)
             p.out_flags[g] = flag;
-        atomicAdd(&p.counters[counter], 1u);
     }
 }
 
-__device__ __forceinline__ void enqueue(const Params &p, int64_t g, int lane)
+__device__ __forceinline__ void enqueue(const Params &p, int64_t g, int lane, Tally &tl)
 {
     if (lane == 0) {
         const uint32_t at = atomicAdd(&p.counters[CQ_CNT_QUEUE], 1u);
         p.queue[at] = static_cast<uint32_t>(g);
-        atomicAdd(&p.counters[CQ_CNT_FALLBACK], 1u);
     }
+    tl.fallback++;
 }
 
-template <int E>
-__device__ __forceinline__ void add_delta(const WarpSmem<E> &sm, uint32_t kk, double (&RB)[E], double (&RC)[E])
-{
-    const int i = (kk >> 3) & 127;
-    const double aw = fabs(static_cast<double>(sm.w[i]));
-    const double c = static_cast<double>(2 * (kk & 7) + 1);
-#pragma unroll
-    for (int e = 0; e < E; e++) {
-        const double dd = sm.d[e][i];
-        RB[e] += dd * aw;  // exact terms: 24-bit d times 11-bit |w|, 24-bit d times odd <= 15
-        RC[e] += dd * c;
-    }
-}
-
+// Key layout: t (grid index of the transition) << 10 | r (rank of the weight
+// in ascending |w|) << 3 | k (the transition |q|: k+1 -> k).
 template <int E>
 __device__ __forceinline__ void add_delta32(const WarpSmem<E> &sm, uint32_t kk, float (&RB)[E], float (&RC)[E])
 {
-    const int i = (kk >> 3) & 127;
-    const float aw = fabsf(sm.w[i]);
+    const int r = (kk >> 3) & 127;
+    const float aw = fabsf(sm.w[r]);
     const float c = static_cast<float>(2 * (kk & 7) + 1);
 #pragma unroll
     for (int e = 0; e < E; e++) {
-        const float dd = sm.d[e][i];
+        const float dd = sm.d[e][r];
         RB[e] = fmaf(dd, aw, RB[e]);
         RC[e] = fmaf(dd, c, RC[e]);
     }
 }
 
+// Exact fp64 coefficient deltas of one transition (products of a 24-bit d with
+// an 11-bit |w| or an odd number <= 15 are exact in fp64).
 template <int E>
-__device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int lane)
+__device__ __forceinline__ void add_delta64(const WarpSmem<E> &sm, uint32_t kk, double (&RB)[E], double (&RC)[E])
 {
-    // ---- 1. load -------------------------------------------------------
-    const uint2 wv = *reinterpret_cast<const uint2 *>(p.W + g * kGroup + 4 * lane);
-    const uint32_t wb[4] = {wv.x & 0xFFFFu, wv.x >> 16, wv.y & 0xFFFFu, wv.y >> 16};
-    float wf[4];
-    float dr[E][4];
-    bool bad = false, nonzero = false;
+    const int r = (kk >> 3) & 127;
+    const double aw = fabsf(sm.w[r]);
+    const double c = static_cast<double>(2 * (kk & 7) + 1);
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        const double dd = sm.d[e][r];
+        RB[e] = fma(dd, aw, RB[e]);
+        RC[e] = fma(dd, c, RC[e]);
+    }
+}
+
+// B_e = sum_i d |w| |q_i(s)| and C_e = sum_i d q_i(s)^2 summed directly over
+// the group (lane L takes ranks 32m + L); every lane gets the same totals.
+template <int E>
+__device__ __forceinline__ void direct_coefficients(const WarpSmem<E> &sm, float s, int lane, double (&B)[E],
+                                                    double (&C)[E])
+{
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        B[e] = 0.0;
+        C[e] = 0.0;
+    }
 #pragma unroll
     for (int m = 0; m < 4; m++) {
-        wf[m] = half_value(wb[m]);
+        const int r = 32 * m + lane;
+        const float wv = sm.w[r];
+        const int aq = abs_code(fabsf(wv), s, wv < 0.0f ? 8 : 7);
+        const double bw = static_cast<double>(fabsf(wv)) * static_cast<double>(aq);  // exact
+        const double cq = static_cast<double>(aq * aq);
+#pragma unroll
+        for (int e = 0; e < E; e++) {
+            const double dd = sm.d[e][r];
+            B[e] = fma(dd, bw, B[e]);  // exact products (<= 39 bits)
+            C[e] = fma(dd, cq, C[e]);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        B[e] = warp_sum(B[e]);
+        C[e] = warp_sum(C[e]);
+    }
+}
+
+template <int E>
+__device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int lane, Tally &tl)
+{
+    // ---- 1. load ---------------------------------------------------------
+    const uint2 wv = *reinterpret_cast<const uint2 *>(p.W + g * kGroup + 4 * lane);
+    const uint32_t wb[4] = {wv.x & 0xFFFFu, wv.x >> 16, wv.y & 0xFFFFu, wv.y >> 16};
+    bool bad = false, nonzero = false;
+    double A[E];
+#pragma unroll
+    for (int m = 0; m < 4; m++) {
         bad |= (wb[m] & 0x7C00u) == 0x7C00u;
         nonzero |= (wb[m] & 0x7FFFu) != 0u;
-        sm.w[4 * lane + m] = wf[m];
     }
 #pragma unroll
     for (int e = 0; e < E; e++) {
         const float4 dv = *reinterpret_cast<const float4 *>(diag_ptr(p, g, e) + 4 * lane);
-        dr[e][0] = dv.x;
-        dr[e][1] = dv.y;
-        dr[e][2] = dv.z;
-        dr[e][3] = dv.w;
+        const float dq[4] = {dv.x, dv.y, dv.z, dv.w};
+        double a = 0.0;
 #pragma unroll
         for (int m = 0; m < 4; m++) {
-            bad |= !(dr[e][m] >= 0.0f && dr[e][m] <= FLT_MAX);
-            sm.d[e][4 * lane + m] = dr[e][m];
+            bad |= !(dq[m] >= 0.0f && dq[m] <= FLT_MAX);
+            const double wd = half_value(wb[m]);
+            a += static_cast<double>(dq[m]) * (wd * wd);  // exact: 24-bit d times 22-bit w^2
         }
+        A[e] = a;
     }
     bad = __any_sync(kFull, bad);
     nonzero = __any_sync(kFull, nonzero);
     if (bad) {
-        write_constant_group(p, g, lane, CQ_FLAG_NONFINITE, CQ_CNT_NONFINITE);
+        write_constant_group(p, g, lane, CQ_FLAG_NONFINITE);
+        tl.nonfinite++;
         return;
     }
     if (!nonzero) {
-        write_constant_group(p, g, lane, CQ_FLAG_TRIVIAL, CQ_CNT_TRIVIAL);
+        write_constant_group(p, g, lane, CQ_FLAG_TRIVIAL);
+        tl.trivial++;
         return;
     }
     if (p.force_exhaustive) {
-        enqueue(p, g, lane);
+        enqueue(p, g, lane, tl);
         return;
     }
-
-    // ---- 2. A_e = sum d w^2 (exact terms) -------------------------------
-    double A[E];
     float Af[E];
 #pragma unroll
     for (int e = 0; e < E; e++) {
-        double a = 0.0;
-#pragma unroll
-        for (int m = 0; m < 4; m++)
-            a += static_cast<double>(dr[e][m]) * (static_cast<double>(wf[m]) * static_cast<double>(wf[m]));
-        A[e] = warp_sum(a);
+        A[e] = warp_sum(A[e]);
         Af[e] = static_cast<float>(A[e]);
     }
 
-    // ---- 3. transitions -------------------------------------------------
-    uint32_t key[32];
+    // ---- 2. order the weights by |w|; stage w and d by rank ----------------
+    // After the sort lane L owns ranks r = 32m + L (m = 0..3).
+    {
+        uint32_t wk[4];
+#pragma unroll
+        for (int m = 0; m < 4; m++)
+            wk[m] = ((wb[m] & 0x7FFFu) << 7) | static_cast<uint32_t>(4 * lane + m);
+        bitonic_sort_128(wk, lane);
+#pragma unroll
+        for (int m = 0; m < 4; m++)
+            sm.bufB[4 * lane + m] = wk[m];
+    }
+    __syncwarp();
+    int z = 0, n7 = 0, negbase[4];
+    bool negm[4];
 #pragma unroll
     for (int m = 0; m < 4; m++) {
-        const float aw = fabsf(wf[m]);
-        const int Kc = ((wb[m] & 0x7FFFu) == 0u) ? 0 : ((wb[m] & 0x8000u) ? 8 : 7);
-        const uint32_t ib = static_cast<uint32_t>(4 * lane + m) << 3;
-#define CQ_T(kk)                                                                                     \
-    key[8 * m + kk] = (kk < Kc) ? ((transition_index<kk>(aw) << 10) | ib | static_cast<uint32_t>(kk)) \
-                                : kInvalidKey;
-        CQ_T(0) CQ_T(1) CQ_T(2) CQ_T(3) CQ_T(4) CQ_T(5) CQ_T(6) CQ_T(7)
-#undef CQ_T
-    }
-
-    // ---- 4. order -------------------------------------------------------
-    bitonic_sort_1024(key, lane);
+        const uint32_t k = sm.bufB[32 * m + lane];
+        const int i = k & 127;
+        const uint32_t bits = p.W[g * kGroup + i];
+        const int r = 32 * m + lane;
+        sm.w[r] = half_value(bits);
 #pragma unroll
-    for (int x = 0; x < 32; x++)
-        sm.keys[swz(32 * lane + x)] = key[x];
+        for (int e = 0; e < E; e++)
+            sm.d[e][r] = diag_ptr(p, g, e)[i];
+        const bool isz = (k >> 7) == 0u;
+        negm[m] = !isz && (bits & 0x8000u) != 0u;
+        const unsigned bz = __ballot_sync(kFull, isz), bn = __ballot_sync(kFull, negm[m]);
+        z += __popc(bz);
+        negbase[m] = n7 + __popc(bn & ((1u << lane) - 1u));
+        n7 += __popc(bn);
+    }
+    const int n = kGroup - z;
     __syncwarp();
 
-    // ---- 5. coefficient scan: lane totals, then suffix across lanes ----
-    double RB0[E], RC0[E];
+    // ---- 3. transitions, one ascending list per code layer k ---------------
+    // Layer k holds t_{r,k} for every nonzero weight in ascending |w| (k = 7:
+    // negative weights only); t is nondecreasing in |w| so each layer is sorted.
+    uint32_t *layer = sm.bufA;
+#pragma unroll
+    for (int m = 0; m < 4; m++) {
+        const int r = 32 * m + lane;
+        if (r >= z) {
+            const float aw = fabsf(sm.w[r]);
+            const uint32_t rb = static_cast<uint32_t>(r) << 3;
+#pragma unroll 1
+            for (int k = 0; k < 7; k++)
+                layer[k * kLayerStride + (r - z)] = (transition_index(aw, k) << 10) | rb | static_cast<uint32_t>(k);
+            if (negm[m])
+                layer[7 * kLayerStride + negbase[m]] = (transition_index(aw, 7) << 10) | rb | 7u;
+        }
+    }
+    if (lane < 7)
+        layer[lane * kLayerStride + n] = kInvalidKey;
+    if (lane == 7)
+        layer[7 * kLayerStride + n7] = kInvalidKey;
+    __syncwarp();
+
+    // ---- 4. merge the eight layers: 4 x 8 lanes, 2 x 16 lanes, 32 lanes ---
+    {
+        const int mg = lane >> 3, sl = lane & 7;
+        const uint32_t *La = layer + (2 * mg) * kLayerStride;
+        const uint32_t *Lb = layer + (2 * mg + 1) * kLayerStride;
+        const int nb = (mg == 3) ? n7 : n;
+        uint32_t *out = sm.bufB + mg * 260;
+        const int tot = n + nb, ch = (tot + 7) >> 3;
+        merge_range(La, n, Lb, nb, out, min(sl * ch, tot), min(sl * ch + ch, tot));
+        if (sl == 0)
+            out[tot] = kInvalidKey;
+    }
+    __syncwarp();
+    {
+        const int mg = lane >> 4, sl = lane & 15;
+        const uint32_t *La = sm.bufB + (2 * mg) * 260;
+        const uint32_t *Lb = sm.bufB + (2 * mg + 1) * 260;
+        const int na = 2 * n, nb = (mg == 1) ? n + n7 : 2 * n;
+        uint32_t *out = sm.bufA + mg * 520;
+        const int tot = na + nb, ch = (tot + 15) >> 4;
+        merge_range(La, na, Lb, nb, out, min(sl * ch, tot), min(sl * ch + ch, tot));
+        if (sl == 0)
+            out[tot] = kInvalidKey;
+    }
+    __syncwarp();
+    // final level: lane L produces outputs [L*c, L*c + c), stores element x at
+    // bufB[x*32 + L] and sums its outputs' coefficient deltas (fp32)
+    const int T = 7 * n + n7;
+    const int c = (T + 31) >> 5;
+    float rbf[E], rcf[E];
 #pragma unroll
     for (int e = 0; e < E; e++) {
-        RB0[e] = 0.0;
-        RC0[e] = 0.0;
+        rbf[e] = 0.0f;
+        rcf[e] = 0.0f;
     }
-#pragma unroll 4
-    for (int x = 0; x < 32; x++) {
-        const uint32_t kk = sm.keys[swz(32 * lane + x)];
-        if (kk != kInvalidKey)
-            add_delta<E>(sm, kk, RB0, RC0);
+    {
+        const uint32_t *La = sm.bufA;
+        const uint32_t *Lb = sm.bufA + 520;
+        const int na = 4 * n, nb = 3 * n + n7;
+        const int d0 = min(lane * c, T), d1 = min(lane * c + c, T);
+        int x = 0;
+        if (d0 < d1) {
+            int i = merge_split(La, na, Lb, nb, d0);
+            int j = d0 - i;
+            uint32_t va = La[i], vb = Lb[j];
+            for (; x < d1 - d0; x++) {
+                const bool ta = va < vb;
+                const uint32_t kk = ta ? va : vb;
+                if (ta)
+                    va = La[++i];
+                else
+                    vb = Lb[++j];
+                sm.bufB[x * 32 + lane] = kk;
+                add_delta32<E>(sm, kk, rbf, rcf);
+            }
+        }
+        for (; x < c; x++)
+            sm.bufB[x * 32 + lane] = kInvalidKey;
     }
+    __syncwarp();
+    const uint32_t *keys = sm.bufB;
+
+    // ---- 5. suffix across lanes: sums over every position after this lane --
 #pragma unroll
     for (int e = 0; e < E; e++) {
-        double vb = RB0[e], vc = RC0[e];
+        float vb = rbf[e], vc = rcf[e];
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const double ub = __shfl_down_sync(kFull, vb, o);
-            const double uc = __shfl_down_sync(kFull, vc, o);
+            const float ub = __shfl_down_sync(kFull, vb, o);
+            const float uc = __shfl_down_sync(kFull, vc, o);
             if (lane + o < 32) {
                 vb += ub;
                 vc += uc;
             }
         }
-        const double xb = __shfl_down_sync(kFull, vb, 1);
-        const double xc = __shfl_down_sync(kFull, vc, 1);
-        RB0[e] = (lane == 31) ? 0.0 : xb;  // sum over every position after this lane's chunk
-        RC0[e] = (lane == 31) ? 0.0 : xc;
+        const float xb = __shfl_down_sync(kFull, vb, 1);
+        const float xc = __shfl_down_sync(kFull, vc, 1);
+        rbf[e] = (lane == 31) ? 0.0f : xb;
+        rcf[e] = (lane == 31) ? 0.0f : xc;
     }
     uint32_t t_after = kBeyond;  // t of the first position after this lane's chunk
     {
-        const uint32_t kn = (lane < 31) ? sm.keys[swz(32 * lane + 32)] : kInvalidKey;
+        const uint32_t kn = (lane < 31 && c > 0) ? keys[lane + 1] : kInvalidKey;
         if (kn != kInvalidKey)
             t_after = kn >> 10;
     }
 
-    // ---- 6. fp32 screen of every run ----------------------------------
-    float rbf[E], rcf[E];
-#pragma unroll
-    for (int e = 0; e < E; e++) {
-        rbf[e] = static_cast<float>(RB0[e]);
-        rcf[e] = static_cast<float>(RC0[e]);
-    }
+    // ---- 6. fp32 screen of every run ----------------------------------------
     float ub_lane = INFINITY;
     uint32_t next_t = t_after;
-    for (int x = 31; x >= 0; --x) {
-        const int pos = 32 * lane + x;
-        const uint32_t kk = sm.keys[swz(pos)];
-        float lbv = INFINITY;
-        if (kk != kInvalidKey) {
-            const uint32_t t = kk >> 10;
-            if (t <= kLast && t != next_t) {
-                float ubv;
-                screen_run32<E>(Af, rbf, rcf, t, min(next_t, kBeyond) - 1u, lbv, ubv);
-                ub_lane = fminf(ub_lane, ubv);
-            }
-            add_delta32<E>(sm, kk, rbf, rcf);
-            next_t = t;
+    float *lbs = sm.lb();
+#pragma unroll 1
+    for (int x = c - 1; x >= 0; --x) {
+        const uint32_t kk = keys[x * 32 + lane];
+        const bool valid = kk != kInvalidKey;
+        const uint32_t t = valid ? (kk >> 10) : kBeyond;
+        const bool run = t <= kLast && t != next_t;
+        const uint32_t ja = run ? t : 1u;
+        const uint32_t jb = run ? min(next_t, kBeyond) - 1u : 1u;
+        float lbv, ubv;
+        screen_run32<E>(Af, rbf, rcf, ja, jb, lbv, ubv);
+        lbs[x * 32 + lane] = run ? lbv : INFINITY;
+        ub_lane = run ? fminf(ub_lane, ubv) : ub_lane;
+        const int r = (kk >> 3) & 127;
+        const float aw = valid ? fabsf(sm.w[r]) : 0.0f;
+        const float cc = valid ? static_cast<float>(2 * (kk & 7) + 1) : 0.0f;
+#pragma unroll
+        for (int e = 0; e < E; e++) {
+            const float dd = sm.d[e][r];
+            rbf[e] = fmaf(dd, aw, rbf[e]);
+            rcf[e] = fmaf(dd, cc, rcf[e]);
         }
-        sm.u.lb[swz(pos)] = lbv;
+        next_t = valid ? t : next_t;
     }
     const uint32_t t_first = next_t;  // lane 0: t of position 0
     if (lane == 0) {
@@ -571,7 +722,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
             screen_run32<E>(Af, rbf, rcf, 1u, min(t_first, kBeyond) - 1u, lbv, ubv);
             ub_lane = fminf(ub_lane, ubv);
         }
-        sm.u.lb[kKeys] = lbv;
+        lbs[1024] = lbv;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
@@ -580,9 +731,10 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     const float U = ub_lane * (1.0f + 0x1p-20f);
     __syncwarp();
     uint32_t smask = 0;
-    for (int x = 0; x < 32; x++)
-        smask |= (sm.u.lb[swz(32 * lane + x)] <= U ? 1u : 0u) << x;
-    const bool init_surv = (lane == 0) && (sm.u.lb[kKeys] <= U);
+#pragma unroll 1
+    for (int x = 0; x < c; x++)
+        smask |= (lbs[x * 32 + lane] <= U ? 1u : 0u) << x;
+    const bool init_surv = (lane == 0) && (lbs[1024] <= U);
     const int my_surv = __popc(smask) + (init_surv ? 1 : 0);
     int excl = my_surv;
 #pragma unroll
@@ -593,97 +745,113 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     }
     const int n_surv = __shfl_sync(kFull, excl, 31);
     excl -= my_surv;
+    tl.survivors += n_surv;
     if (n_surv > kMaxSurvivors) {
-        enqueue(p, g, lane);
+        enqueue(p, g, lane, tl);
         return;
     }
     __syncwarp();
 
-    // ---- 7. certified fp64 search of the survivors, 32 at a time -------
+    // ---- 7. survivors: exact fp64 coefficients, certified search -------------
+    // Survivors are ranked by descending position (lane 31 first, x descending;
+    // the run below every transition last).  The highest one gets its exact
+    // coefficients from a direct sum over the weights; each next one adds the
+    // exact fp64 deltas of the transitions in between, walked by the whole warp
+    // in lockstep, or is summed directly again when the gap is long.
+    SurvEntry *ent = sm.ent();
+    float *res_lb = sm.res_lb();
+    uint16_t *res_j = sm.res_j();
+    int above = my_surv;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_down_sync(kFull, above, o);
+        if (lane + o < 32)
+            above += v;
+    }
+    above -= my_surv;  // survivors of higher lanes
+    if (my_surv > 0) {
+        int rk = above;
+        uint32_t nt = t_after;
+#pragma unroll 1
+        for (int x = c - 1; x >= 0; --x) {
+            const uint32_t kk = keys[x * 32 + lane];
+            if (kk == kInvalidKey)
+                continue;
+            const uint32_t t = kk >> 10;
+            if ((smask >> x) & 1u)
+                ent[rk++] = SurvEntry{t, min(nt, kBeyond) - 1u, lane * c + x, 0};
+            nt = t;
+        }
+        if (init_surv)
+            ent[rk] = SurvEntry{1u, min(t_first, kBeyond) - 1u, -1, 0};
+    }
+    __syncwarp();
     double ub_min = INFINITY;
+    double Bc[E], Cc[E];
+    int cur = -2;  // position whose run the coefficients Bc, Cc belong to
+#pragma unroll 1
     for (int base = 0; base < n_surv; base += 32) {
-        if (my_surv > 0 && excl < base + 32 && excl + my_surv > base) {
-            double RB[E], RC[E];
+        const int nb = min(32, n_surv - base);
+        double myB[E], myC[E];
 #pragma unroll
-            for (int e = 0; e < E; e++) {
-                RB[e] = RB0[e];
-                RC[e] = RC0[e];
-            }
-            int r = excl;
-            uint32_t nt = t_after;
-            for (int x = 31; x >= 0; --x) {
-                const uint32_t kk = sm.keys[swz(32 * lane + x)];
-                if (kk == kInvalidKey)
-                    continue;
-                const uint32_t t = kk >> 10;
-                if ((smask >> x) & 1u) {
-                    if (r >= base && r < base + 32) {
-                        SurvEntry<E> &en = sm.u.ent[r - base];
-#pragma unroll
-                        for (int e = 0; e < E; e++) {
-                            en.B[e] = RB[e];
-                            en.C[e] = RC[e];
-                        }
-                        en.ja = t;
-                        en.jb = min(nt, kBeyond) - 1u;
+        for (int e = 0; e < E; e++) {
+            myB[e] = 0.0;
+            myC[e] = 0.0;
+        }
+#pragma unroll 1
+        for (int si = 0; si < nb; si++) {
+            const SurvEntry en = ent[base + si];
+            if (cur == -2 || cur - en.pos > kWalkMax) {
+                direct_coefficients<E>(sm, grid_value(en.ja), lane, Bc, Cc);
+            } else {
+                // add the deltas of positions cur, cur-1, ..., en.pos+1
+                int lp = cur / c, x = cur - lp * c;
+#pragma unroll 1
+                for (int q = cur; q > en.pos; --q) {
+                    add_delta64<E>(sm, keys[x * 32 + lp], Bc, Cc);
+                    if (--x < 0) {
+                        x = c - 1;
+                        --lp;
                     }
-                    r++;
                 }
-                add_delta<E>(sm, kk, RB, RC);
-                nt = t;
             }
-            if (init_surv && r >= base && r < base + 32) {
-                SurvEntry<E> &en = sm.u.ent[r - base];
+            cur = en.pos;
+            if (lane == si) {
 #pragma unroll
                 for (int e = 0; e < E; e++) {
-                    en.B[e] = RB[e];
-                    en.C[e] = RC[e];
+                    myB[e] = Bc[e];
+                    myC[e] = Cc[e];
                 }
-                en.ja = 1u;
-                en.jb = min(t_first, kBeyond) - 1u;
             }
         }
-        __syncwarp();
-        const int me = base + lane;
-        if (me < n_surv) {
-            const SurvEntry<E> &en = sm.u.ent[lane];
-            double Bv[E], Cv[E];
-#pragma unroll
-            for (int e = 0; e < E; e++) {
-                Bv[e] = en.B[e];
-                Cv[e] = en.C[e];
-            }
-            const RunResult rr = solve_run<E>(A, Bv, Cv, en.ja, en.jb);
-            sm.res_lb[me] = rr.lb;
-            sm.res_j[me] = static_cast<uint16_t>(rr.j | (rr.uncertain ? kUncertainBit : 0u));
+        if (lane < nb) {
+            const SurvEntry en = ent[base + lane];
+            const RunResult rr = solve_run<E>(A, myB, myC, en.ja, en.jb);
+            res_lb[base + lane] = rr.lb;
+            res_j[base + lane] = static_cast<uint16_t>(rr.j | (rr.uncertain ? kUncertainBit : 0u));
             ub_min = fmin(ub_min, rr.ub);
         }
-        __syncwarp();
     }
+    __syncwarp();
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
         ub_min = fmin(ub_min, __shfl_xor_sync(kFull, ub_min, o));
-    const float T = __double2float_ru(ub_min * (1.0 + 0x1p-40));
+    const float Tf = __double2float_ru(ub_min * (1.0 + 0x1p-40));
 
-    // ---- 8. finalists ---------------------------------------------------
+    // ---- 8. finalists ---------------------------------------------------------
     int cnt = 0;
     bool unc_comp = false, unc_any = false;
     for (int me = lane; me < n_surv; me += 32) {
-        const uint32_t jv = sm.res_j[me];
-        const bool in = sm.res_lb[me] <= T;
+        const uint32_t jv = res_j[me];
         unc_any |= (jv & kUncertainBit) != 0u;
-        if (in) {
+        if (res_lb[me] <= Tf) {
             if (jv & kUncertainBit)
                 unc_comp = true;
             else
                 cnt++;
         }
     }
-    if (lane == 0) {
-        atomicAdd(&p.counters[CQ_CNT_SURVIVORS], static_cast<uint32_t>(n_surv));
-    }
-    if (__any_sync(kFull, unc_any) && lane == 0)
-        atomicAdd(&p.counters[CQ_CNT_UNCERTAIN], 1u);
+    tl.uncertain += __any_sync(kFull, unc_any) ? 1u : 0u;
     unc_comp = __any_sync(kFull, unc_comp);
     int fx = cnt;
 #pragma unroll
@@ -695,25 +863,23 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     const int total = __shfl_sync(kFull, fx, 31);
     fx -= cnt;
     if (unc_comp || total > p.finalist_cap || total == 0) {
-        enqueue(p, g, lane);
+        enqueue(p, g, lane, tl);
         return;
     }
+    int *fin = sm.fin();
     for (int me = lane; me < n_surv; me += 32) {
-        if (sm.res_lb[me] <= T && !(sm.res_j[me] & kUncertainBit))
-            sm.fin[fx++] = sm.res_j[me];
+        if (res_lb[me] <= Tf && !(res_j[me] & kUncertainBit))
+            fin[fx++] = res_j[me];
     }
     __syncwarp();
 
-    // ---- 9. fp64 rescoring of the finalists -------------------------------
-    int Kc[4];
-#pragma unroll
-    for (int m = 0; m < 4; m++)
-        Kc[m] = (wb[m] & 0x8000u) ? 8 : 7;
+    // ---- 9. fp64 rescoring of the finalists (lane L takes ranks 32m + L) -------
     double best = INFINITY, second = INFINITY;
     uint32_t bj = 0;
+#pragma unroll 1
     for (int f = 0; f < total; f++) {
-        const uint32_t j = static_cast<uint32_t>(sm.fin[f]);
-        const float s = half_value(j);
+        const uint32_t j = static_cast<uint32_t>(fin[f]);
+        const float s = grid_value(j);
         const double sd = s;
         double acc[E];
 #pragma unroll
@@ -721,13 +887,14 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
             acc[e] = 0.0;
 #pragma unroll
         for (int m = 0; m < 4; m++) {
-            const int aq = abs_code(fabsf(wf[m]), s, Kc[m]);
-            const double q = (wb[m] & 0x8000u) ? -static_cast<double>(aq) : static_cast<double>(aq);
-            const double r = static_cast<double>(wf[m]) - sd * q;  // exact
-            const double rr = __dmul_rn(r, r);
+            const int r = 32 * m + lane;
+            const float wv = sm.w[r];
+            const int aq = abs_code(fabsf(wv), s, wv < 0.0f ? 8 : 7);
+            const double r_ = static_cast<double>(fabsf(wv)) - sd * static_cast<double>(aq);  // exact
+            const double rr = __dmul_rn(r_, r_);
 #pragma unroll
             for (int e = 0; e < E; e++)
-                acc[e] = __dadd_rn(acc[e], __dmul_rn(static_cast<double>(dr[e][m]), rr));
+                acc[e] = __dadd_rn(acc[e], __dmul_rn(static_cast<double>(sm.d[e][r]), rr));
         }
         double v = -INFINITY;
 #pragma unroll
@@ -742,41 +909,53 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         }
     }
 
-    // ---- 10. pack and store -------------------------------------------------
-    const float s = half_value(bj);
+    // ---- 10. pack and store ---------------------------------------------------
+    const float s = grid_value(bj);
     int q[4];
 #pragma unroll
     for (int m = 0; m < 4; m++) {
-        const int aq = abs_code(fabsf(wf[m]), s, Kc[m]);
+        const int aq = abs_code(half_value(wb[m] & 0x7FFFu), s, (wb[m] & 0x8000u) ? 8 : 7);
         q[m] = (wb[m] & 0x8000u) ? -aq : aq;
     }
     const uint32_t word = pack_lane_codes(q, lane);
     if ((lane & 1) == 0)
         p.out_codes[g * 16 + (lane >> 1)] = word;
+    const bool near = near_tie(best, second, p.flag_rel_gap);
     if (lane == 0) {
         p.out_scales[g] = static_cast<uint16_t>(bj);
         if (p.out_obj)
             p.out_obj[g] = best;
-        const bool near = near_tie(best, second, p.flag_rel_gap);
         if (p.out_flags)
             p.out_flags[g] = near ? CQ_FLAG_NEAR_TIE : 0;
-        if (near)
-            atomicAdd(&p.counters[CQ_CNT_NEAR_TIE], 1u);
-        atomicAdd(&p.counters[CQ_CNT_FINALISTS], static_cast<uint32_t>(total));
     }
+    tl.near_tie += near ? 1u : 0u;
+    tl.finalists += static_cast<uint32_t>(total);
 }
 
 template <int E>
-__global__ void __launch_bounds__(kWarps * 32, (E <= 4 ? 4 : 2)) select_kernel(Params p)
+__global__ void __launch_bounds__(kWarps * 32, (E <= 4 ? 5 : 4)) select_kernel(Params p)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int lane = threadIdx.x & 31;
     const int wib = threadIdx.x >> 5;
     WarpSmem<E> &sm = reinterpret_cast<WarpSmem<E> *>(smem_raw)[wib];
+    Tally tl;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * kWarps;
     for (int64_t g = static_cast<int64_t>(blockIdx.x) * kWarps + wib; g < p.G; g += stride) {
-        process_group<E>(p, sm, g, lane);
+        if (lane < 2 && g + stride < p.G)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(p.W + (g + stride) * kGroup + 64 * lane));
+        process_group<E>(p, sm, g, lane, tl);
         __syncwarp();
+    }
+    if (lane == 0) {
+        const uint32_t v[7] = {tl.fallback, tl.near_tie, tl.nonfinite, tl.trivial, tl.finalists, tl.uncertain,
+                               tl.survivors};
+        const int at[7] = {CQ_CNT_FALLBACK, CQ_CNT_NEAR_TIE, CQ_CNT_NONFINITE, CQ_CNT_TRIVIAL, CQ_CNT_FINALISTS,
+                           CQ_CNT_UNCERTAIN, CQ_CNT_SURVIVORS};
+#pragma unroll
+        for (int k = 0; k < 7; k++)
+            if (v[k])
+                atomicAdd(&p.counters[at[k]], v[k]);
     }
 }
 
@@ -819,7 +998,7 @@ __global__ void __launch_bounds__(kExThreads) exhaustive_kernel(Params p)
         __syncthreads();
         Best3 b{INFINITY, INFINITY, 0u};
         for (uint32_t j = 1u + tid; j <= kLast; j += kExThreads) {
-            const float s = half_value(j);
+            const float s = grid_value(j);
             const double sd = s;
             double acc[E];
 #pragma unroll
@@ -869,7 +1048,7 @@ __global__ void __launch_bounds__(kExThreads) exhaustive_kernel(Params p)
         const Best3 r = red[0];
         if (tid < kGroup) {
             const float w = ws[tid];
-            const float s = half_value(r.j);
+            const float s = grid_value(r.j);
             const int aq = abs_code(fabsf(w), s, w < 0.0f ? 8 : 7);
             const int q = (w < 0.0f) ? -aq : aq;
             nib[tid] = static_cast<uint32_t>((q + 8) & 0xF);
