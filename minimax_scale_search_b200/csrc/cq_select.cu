@@ -249,6 +249,8 @@ template <int E>
 struct WarpSmem {
     float d[E][kGroup];       // diagonals by rank in ascending |w|
     float w[kGroup];          // signed weights by rank in ascending |w|
+    uint8_t negpre[kGroup + 4];  // number of negative weights below each rank
+    int lay[16];                 // window rank range of each transition layer
     // A: transition layers -> level-2 lists -> per-run fp32 lower bounds ->
     //    survivor ranges + survivor results
     alignas(16) uint32_t bufA[kBufWords];
@@ -555,8 +557,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
             sm.bufB[4 * lane + m] = wk[m];
     }
     __syncwarp();
-    int z = 0, n7 = 0, negbase[4];
-    bool negm[4];
+    int n7 = 0;
 #pragma unroll
     for (int m = 0; m < 4; m++) {
         const uint32_t k = sm.bufB[32 * m + lane];
@@ -567,48 +568,223 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
 #pragma unroll
         for (int e = 0; e < E; e++)
             sm.d[e][r] = diag_ptr(p, g, e)[i];
-        const bool isz = (k >> 7) == 0u;
-        negm[m] = !isz && (bits & 0x8000u) != 0u;
-        const unsigned bz = __ballot_sync(kFull, isz), bn = __ballot_sync(kFull, negm[m]);
-        z += __popc(bz);
-        negbase[m] = n7 + __popc(bn & ((1u << lane) - 1u));
+        const bool neg = (k >> 7) != 0u && (bits & 0x8000u) != 0u;
+        const unsigned bn = __ballot_sync(kFull, neg);
+        sm.negpre[r] = static_cast<uint8_t>(n7 + __popc(bn & ((1u << lane) - 1u)));
         n7 += __popc(bn);
     }
-    const int n = kGroup - z;
+    if (lane == 0)
+        sm.negpre[kGroup] = static_cast<uint8_t>(n7);
     __syncwarp();
 
-    // ---- 3. transitions, one ascending list per code layer k ---------------
-    // Layer k holds t_{r,k} for every nonzero weight in ascending |w| (k = 7:
-    // negative weights only); t is nondecreasing in |w| so each layer is sorted.
+    // ---- 3. a rigorous upper bound U of the minimum -----------------------
+    // The fp32 objective at three grid scales near the AbsMax scale |w|max/7,
+    // widened by 2^-18 (>= 12 fp32 roundings of nonnegative terms).
+    const float amax = fabsf(sm.w[kGroup - 1]);
+    const uint32_t ja0 = min(max(static_cast<uint32_t>(__half_as_ushort(__float2half_rn(amax * (1.0f / 7.0f)))), 1u),
+                             kLast);
+    float U;
+    {
+        const uint32_t jc[3] = {ja0, min(max(static_cast<uint32_t>(
+                                              __half_as_ushort(__float2half_rn(amax * (0.9f / 7.0f)))), 1u), kLast),
+                                min(max(static_cast<uint32_t>(
+                                        __half_as_ushort(__float2half_rn(amax * (0.8f / 7.0f)))), 1u), kLast)};
+        float acc[3][E];
+#pragma unroll
+        for (int c = 0; c < 3; c++)
+#pragma unroll
+            for (int e = 0; e < E; e++)
+                acc[c][e] = 0.0f;
+#pragma unroll
+        for (int m = 0; m < 4; m++) {
+            const int r = 32 * m + lane;
+            const float wv = sm.w[r];
+            const float aw = fabsf(wv);
+            const int K = wv < 0.0f ? 8 : 7;
+#pragma unroll
+            for (int c = 0; c < 3; c++) {
+                const float s = grid_value(jc[c]);
+                const float res = fmaf(-s, static_cast<float>(abs_code(aw, s, K)), aw);
+                const float rr = res * res;
+#pragma unroll
+                for (int e = 0; e < E; e++)
+                    acc[c][e] = fmaf(sm.d[e][r], rr, acc[c][e]);
+            }
+        }
+        U = INFINITY;
+#pragma unroll
+        for (int c = 0; c < 3; c++) {
+            float f = 0.0f;
+#pragma unroll
+            for (int e = 0; e < E; e++)
+                f = fmaxf(f, warp_sum(acc[c][e]));
+            U = fminf(U, f);
+        }
+        U *= 1.0f + 0x1p-18f;
+    }
+
+    // ---- 4. window [J0, J1] of grid indices that can hold the minimum -----
+    // Below: the clipping error of the 8 largest weights, sum d (|w| - K s)_+^2,
+    // is a lower bound of every F_e that decreases in s.  Above: weights with
+    // |w| <= s/2 quantise to 0, so sum over them of d w^2 is a lower bound that
+    // increases in s.  Lane j tests the scales 128 j patterns below / above
+    // the AbsMax scale; each bound is shrunk by 2^-18 for its fp32 roundings.
+    uint32_t J0 = 1u, J1 = kLast;
+    {
+        // prefix sums over ranks of d w^2 (fp32), ph[e][c] = sum over ranks < c
+        float *ph = reinterpret_cast<float *>(sm.bufB);  // [E][kGroup + 1]
+        float carry[E];
+#pragma unroll
+        for (int e = 0; e < E; e++)
+            carry[e] = 0.0f;
+        if (lane == 0) {
+#pragma unroll
+            for (int e = 0; e < E; e++)
+                ph[e * (kGroup + 1)] = 0.0f;
+        }
+#pragma unroll
+        for (int m = 0; m < 4; m++) {
+            const int r = 32 * m + lane;
+            const float wv = sm.w[r];
+            const float w2 = wv * wv;
+#pragma unroll
+            for (int e = 0; e < E; e++) {
+                float v = sm.d[e][r] * w2;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float u = __shfl_up_sync(kFull, v, o);
+                    if (lane >= o)
+                        v += u;
+                }
+                ph[e * (kGroup + 1) + r + 1] = carry[e] + v;
+                carry[e] += __shfl_sync(kFull, v, 31);
+            }
+        }
+        // lower end: clip bound of the top 8 weights at scale ja0 - 128 * lane
+        const uint32_t jl = ja0 > 128u * lane ? ja0 - 128u * lane : 1u;
+        const float sl = grid_value(jl);
+        float L = 0.0f;
+        {
+            float le[E];
+#pragma unroll
+            for (int e = 0; e < E; e++)
+                le[e] = 0.0f;
+#pragma unroll
+            for (int r = kGroup - 8; r < kGroup; r++) {
+                const float wv = sm.w[r];
+                const float ex = fmaxf(fmaf(-(wv < 0.0f ? 8.0f : 7.0f), sl, fabsf(wv)), 0.0f);
+                const float e2 = ex * ex;
+#pragma unroll
+                for (int e = 0; e < E; e++)
+                    le[e] = fmaf(sm.d[e][r], e2, le[e]);
+            }
+#pragma unroll
+            for (int e = 0; e < E; e++)
+                L = fmaxf(L, le[e]);
+        }
+        const unsigned cut_lo = __ballot_sync(kFull, L * (1.0f - 0x1p-18f) > U);
+        if (cut_lo) {
+            const int j0 = __ffs(cut_lo) - 1;  // largest excluded scale
+            J0 = __shfl_sync(kFull, jl, j0) + 1u;
+        }
+        __syncwarp();
+        // upper end: round-to-zero bound at scale ja0 + 128 * lane
+        const uint32_t jh = min(ja0 + 128u * lane, kLast);
+        const float half_s = 0.5f * grid_value(jh);
+        int lo = 0, hi = kGroup;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (fabsf(sm.w[mid]) <= half_s)
+                lo = mid + 1;
+            else
+                hi = mid;
+        }
+        float H = 0.0f;
+#pragma unroll
+        for (int e = 0; e < E; e++)
+            H = fmaxf(H, ph[e * (kGroup + 1) + lo]);
+        const unsigned cut_hi = __ballot_sync(kFull, H * (1.0f - 0x1p-18f) > U);
+        if (cut_hi) {
+            const int j1 = __ffs(cut_hi) - 1;  // smallest excluded scale
+            J1 = __shfl_sync(kFull, jh, j1) - 1u;
+        }
+        if (J0 > J1) {  // cannot happen for valid bounds; keep the whole grid
+            J0 = 1u;
+            J1 = kLast;
+        }
+    }
+    const uint32_t jend = J1 + 1u;
+    const float sJ0 = grid_value(J0), sJ1 = grid_value(J1);
+    __syncwarp();
+
+    // ---- 3'. transitions inside the window, one ascending list per layer k --
+    // Weight r has |q| >= k+1 at s_J0 and <= k at s_J1 exactly when its
+    // transition k+1 -> k lies in (J0, J1]; with ranks in ascending |w| those
+    // weights form one rank range [F0_k, F1_k) (layer 7: negative weights, by
+    // their rank among negatives).  Transitions above J1 are active on the
+    // whole window and only enter the coefficients, in closed form.
     uint32_t *layer = sm.bufA;
+    if (lane < 16) {
+        const int k = lane & 7;
+        const float sx = (lane < 8) ? sJ0 : sJ1;
+        int lo = 0, hi = kGroup;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (!code_at_least(fabsf(sm.w[mid]), sx, k + 1))
+                lo = mid + 1;
+            else
+                hi = mid;
+        }
+        sm.lay[lane] = (k == 7) ? sm.negpre[lo] : lo;  // lanes 0..7: F0_k, lanes 8..15: F1_k
+    }
+    __syncwarp();
+    const int *off = sm.lay;  // layer k holds ranks [off[k], off[k + 8]) (layer 7: negative ranks)
+    float rbf[E], rcf[E];
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        rbf[e] = 0.0f;
+        rcf[e] = 0.0f;
+    }
+    float bb[E], bc[E];  // this lane's share of the coefficients above the window
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        bb[e] = 0.0f;
+        bc[e] = 0.0f;
+    }
 #pragma unroll
     for (int m = 0; m < 4; m++) {
         const int r = 32 * m + lane;
-        if (r >= z) {
-            const float aw = fabsf(sm.w[r]);
-            const uint32_t rb = static_cast<uint32_t>(r) << 3;
-#pragma unroll 1
-            for (int k = 0; k < 7; k++)
-                layer[k * kLayerStride + (r - z)] = (transition_index(aw, k) << 10) | rb | static_cast<uint32_t>(k);
-            if (negm[m])
-                layer[7 * kLayerStride + negbase[m]] = (transition_index(aw, 7) << 10) | rb | 7u;
+        const float wv = sm.w[r];
+        const float aw = fabsf(wv);
+        const int K = wv < 0.0f ? 8 : 7;
+        const int ktop = abs_code(aw, sJ1, K);
+        const int kbot = abs_code(aw, sJ0, K);
+        const float fk = static_cast<float>(ktop);
+#pragma unroll
+        for (int e = 0; e < E; e++) {
+            const float dd = sm.d[e][r];
+            bb[e] = fmaf(dd, aw * fk, bb[e]);
+            bc[e] = fmaf(dd, fk * fk, bc[e]);
+        }
+        const uint32_t rb = static_cast<uint32_t>(r) << 3;
+        for (int k = ktop; k < kbot; k++) {
+            const int at = (k == 7) ? static_cast<int>(sm.negpre[r]) - off[7] : r - off[k];
+            layer[k * kLayerStride + at] = (transition_index(aw, k) << 10) | rb | static_cast<uint32_t>(k);
         }
     }
-    if (lane < 7)
-        layer[lane * kLayerStride + n] = kInvalidKey;
-    if (lane == 7)
-        layer[7 * kLayerStride + n7] = kInvalidKey;
+    if (lane < 8)
+        layer[lane * kLayerStride + off[lane + 8] - off[lane]] = kInvalidKey;
     __syncwarp();
 
-    // ---- 4. merge the eight layers: 4 x 8 lanes, 2 x 16 lanes, 32 lanes ---
+    // ---- 4'. merge the eight layers: 4 x 8 lanes, 2 x 16 lanes, 32 lanes ---
     {
         const int mg = lane >> 3, sl = lane & 7;
         const uint32_t *La = layer + (2 * mg) * kLayerStride;
         const uint32_t *Lb = layer + (2 * mg + 1) * kLayerStride;
-        const int nb = (mg == 3) ? n7 : n;
+        const int na = off[2 * mg + 8] - off[2 * mg], nb = off[2 * mg + 9] - off[2 * mg + 1];
         uint32_t *out = sm.bufB + mg * 260;
-        const int tot = n + nb, ch = (tot + 7) >> 3;
-        merge_range(La, n, Lb, nb, out, min(sl * ch, tot), min(sl * ch + ch, tot));
+        const int tot = na + nb, ch = (tot + 7) >> 3;
+        merge_range(La, na, Lb, nb, out, min(sl * ch, tot), min(sl * ch + ch, tot));
         if (sl == 0)
             out[tot] = kInvalidKey;
     }
@@ -617,7 +793,8 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         const int mg = lane >> 4, sl = lane & 15;
         const uint32_t *La = sm.bufB + (2 * mg) * 260;
         const uint32_t *Lb = sm.bufB + (2 * mg + 1) * 260;
-        const int na = 2 * n, nb = (mg == 1) ? n + n7 : 2 * n;
+        const int na = off[4 * mg + 8] - off[4 * mg] + off[4 * mg + 9] - off[4 * mg + 1];
+        const int nb = off[4 * mg + 10] - off[4 * mg + 2] + off[4 * mg + 11] - off[4 * mg + 3];
         uint32_t *out = sm.bufA + mg * 520;
         const int tot = na + nb, ch = (tot + 15) >> 4;
         merge_range(La, na, Lb, nb, out, min(sl * ch, tot), min(sl * ch + ch, tot));
@@ -627,22 +804,21 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     __syncwarp();
     // final level: lane L produces outputs [L*c, L*c + c), stores element x at
     // bufB[x*32 + L] and sums its outputs' coefficient deltas (fp32)
-    const int T = 7 * n + n7;
-    const int c = (T + 31) >> 5;
-    float rbf[E], rcf[E];
+    int na3 = 0, nb3 = 0;
 #pragma unroll
-    for (int e = 0; e < E; e++) {
-        rbf[e] = 0.0f;
-        rcf[e] = 0.0f;
+    for (int k = 0; k < 4; k++) {
+        na3 += off[k + 8] - off[k];
+        nb3 += off[k + 12] - off[k + 4];
     }
+    const int T = na3 + nb3;
+    const int c = (T + 31) >> 5;
     {
         const uint32_t *La = sm.bufA;
         const uint32_t *Lb = sm.bufA + 520;
-        const int na = 4 * n, nb = 3 * n + n7;
         const int d0 = min(lane * c, T), d1 = min(lane * c + c, T);
         int x = 0;
         if (d0 < d1) {
-            int i = merge_split(La, na, Lb, nb, d0);
+            int i = merge_split(La, na3, Lb, nb3, d0);
             int j = d0 - i;
             uint32_t va = La[i], vb = Lb[j];
             for (; x < d1 - d0; x++) {
@@ -662,7 +838,8 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     __syncwarp();
     const uint32_t *keys = sm.bufB;
 
-    // ---- 5. suffix across lanes: sums over every position after this lane --
+    // ---- 5. suffix across lanes: sums over every position after this lane,
+    //         plus the transitions above the window ---------------------------
 #pragma unroll
     for (int e = 0; e < E; e++) {
         float vb = rbf[e], vc = rcf[e];
@@ -677,17 +854,17 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         }
         const float xb = __shfl_down_sync(kFull, vb, 1);
         const float xc = __shfl_down_sync(kFull, vc, 1);
-        rbf[e] = (lane == 31) ? 0.0f : xb;
-        rcf[e] = (lane == 31) ? 0.0f : xc;
+        rbf[e] = ((lane == 31) ? 0.0f : xb) + warp_sum(bb[e]);
+        rcf[e] = ((lane == 31) ? 0.0f : xc) + warp_sum(bc[e]);
     }
-    uint32_t t_after = kBeyond;  // t of the first position after this lane's chunk
+    uint32_t t_after = jend;  // t of the first position after this lane's chunk
     {
         const uint32_t kn = (lane < 31 && c > 0) ? keys[lane + 1] : kInvalidKey;
         if (kn != kInvalidKey)
             t_after = kn >> 10;
     }
 
-    // ---- 6. fp32 screen of every run ----------------------------------------
+    // ---- 6. fp32 screen of every run in the window --------------------------
     float ub_lane = INFINITY;
     uint32_t next_t = t_after;
     float *lbs = sm.lb();
@@ -695,10 +872,10 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     for (int x = c - 1; x >= 0; --x) {
         const uint32_t kk = keys[x * 32 + lane];
         const bool valid = kk != kInvalidKey;
-        const uint32_t t = valid ? (kk >> 10) : kBeyond;
-        const bool run = t <= kLast && t != next_t;
-        const uint32_t ja = run ? t : 1u;
-        const uint32_t jb = run ? min(next_t, kBeyond) - 1u : 1u;
+        const uint32_t t = valid ? (kk >> 10) : jend;
+        const bool run = t <= J1 && t != next_t;
+        const uint32_t ja = run ? t : J0;
+        const uint32_t jb = run ? min(next_t, jend) - 1u : J0;
         float lbv, ubv;
         screen_run32<E>(Af, rbf, rcf, ja, jb, lbv, ubv);
         lbs[x * 32 + lane] = run ? lbv : INFINITY;
@@ -714,12 +891,12 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         }
         next_t = valid ? t : next_t;
     }
-    const uint32_t t_first = next_t;  // lane 0: t of position 0
+    const uint32_t t_first = next_t;  // lane 0: t of position 0 (jend if none)
     if (lane == 0) {
         float lbv = INFINITY;
-        if (t_first > 1u) {
+        if (t_first > J0) {
             float ubv;
-            screen_run32<E>(Af, rbf, rcf, 1u, min(t_first, kBeyond) - 1u, lbv, ubv);
+            screen_run32<E>(Af, rbf, rcf, J0, min(t_first, jend) - 1u, lbv, ubv);
             ub_lane = fminf(ub_lane, ubv);
         }
         lbs[1024] = lbv;
@@ -728,13 +905,13 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     for (int o = 16; o > 0; o >>= 1)
         ub_lane = fminf(ub_lane, __shfl_xor_sync(kFull, ub_lane, o));
     // survivors: runs whose screened lower bound reaches the best screened upper bound
-    const float U = ub_lane * (1.0f + 0x1p-20f);
+    const float Us = fminf(ub_lane, U) * (1.0f + 0x1p-20f);
     __syncwarp();
     uint32_t smask = 0;
-#pragma unroll 1
+#pragma unroll 4
     for (int x = 0; x < c; x++)
-        smask |= (lbs[x * 32 + lane] <= U ? 1u : 0u) << x;
-    const bool init_surv = (lane == 0) && (lbs[1024] <= U);
+        smask |= (lbs[x * 32 + lane] <= Us ? 1u : 0u) << x;
+    const bool init_surv = (lane == 0) && (lbs[1024] <= Us);
     const int my_surv = __popc(smask) + (init_surv ? 1 : 0);
     int excl = my_surv;
 #pragma unroll
@@ -744,7 +921,6 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
             excl += v;
     }
     const int n_surv = __shfl_sync(kFull, excl, 31);
-    excl -= my_surv;
     tl.survivors += n_surv;
     if (n_surv > kMaxSurvivors) {
         enqueue(p, g, lane, tl);
@@ -779,11 +955,11 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
                 continue;
             const uint32_t t = kk >> 10;
             if ((smask >> x) & 1u)
-                ent[rk++] = SurvEntry{t, min(nt, kBeyond) - 1u, lane * c + x, 0};
+                ent[rk++] = SurvEntry{t, min(nt, jend) - 1u, lane * c + x, 0};
             nt = t;
         }
         if (init_surv)
-            ent[rk] = SurvEntry{1u, min(t_first, kBeyond) - 1u, -1, 0};
+            ent[rk] = SurvEntry{J0, min(t_first, jend) - 1u, -1, 0};
     }
     __syncwarp();
     double ub_min = INFINITY;
