@@ -250,7 +250,7 @@ struct WarpSmem {
     float d[E][kGroup];       // diagonals by rank in ascending |w|
     float w[kGroup];          // signed weights by rank in ascending |w|
     uint8_t negpre[kGroup + 4];  // number of negative weights below each rank
-    int lay[16];                 // window rank range of each transition layer
+    int lay[32];                 // window rank range of each transition layer; rank thresholds
     // A: transition layers -> level-2 lists -> per-run fp32 lower bounds ->
     //    survivor ranges + survivor results
     alignas(16) uint32_t bufA[kBufWords];
@@ -293,7 +293,7 @@ __device__ __forceinline__ double screen(const double (&A)[E], const double (&nb
 // indices [ja, jb], with a certified bracket (see the file comment, step 5).
 template <int E>
 __device__ RunResult solve_run(const double (&A)[E], const double (&B)[E], const double (&C)[E],
-                               uint32_t ja, uint32_t jb)
+                               uint32_t ja, uint32_t jb, uint32_t guess)
 {
     RunResult r;
     double cmax = C[0], amax = A[0];
@@ -319,6 +319,28 @@ __device__ RunResult solve_run(const double (&A)[E], const double (&B)[E], const
         P = fmax(P, fma(fma(C[e], sb, 2.0 * B[e]), sb, A[e]));
     }
     const double delta = P * 0x1p-44;  // >= |screen - exact| anywhere on the run
+    // A certified strict local minimum at the guess is the run's unique
+    // minimiser (convexity); otherwise fall back to the binary search.
+    {
+        const uint32_t j = min(max(guess, ja), jb);
+        const double Sj = screen<E>(A, nb2, C, grid_value(j));
+        bool ok = true;
+        if (j > ja) {
+            const double Sl = screen<E>(A, nb2, C, grid_value(j - 1));
+            ok = Sl - Sj > 2.0 * delta + 0x1p-40 * fmax(fabs(Sl), fabs(Sj));
+        }
+        if (ok && j < jb) {
+            const double Sr = screen<E>(A, nb2, C, grid_value(j + 1));
+            ok = Sr - Sj > 2.0 * delta + 0x1p-40 * fmax(fabs(Sr), fabs(Sj));
+        }
+        if (ok) {
+            r.j = j;
+            r.ub = Sj + delta;
+            r.lb = __double2float_rd(Sj - delta);
+            r.uncertain = false;
+            return r;
+        }
+    }
     uint32_t lo = ja, hi = jb;
     bool unc = false;
     while (lo < hi) {
@@ -604,7 +626,10 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
 #pragma unroll
             for (int c = 0; c < 3; c++) {
                 const float s = grid_value(jc[c]);
-                const float res = fmaf(-s, static_cast<float>(abs_code(aw, s, K)), aw);
+                // any codes in range give an objective >= the one of the exact
+                // codes at s, so an uncorrected estimate keeps U an upper bound
+                const float qe = fminf(rintf(__fdividef(aw, s)), static_cast<float>(K));
+                const float res = fmaf(-s, qe, aw);
                 const float rr = res * res;
 #pragma unroll
                 for (int e = 0; e < E; e++)
@@ -736,6 +761,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
                 hi = mid;
         }
         sm.lay[lane] = (k == 7) ? sm.negpre[lo] : lo;  // lanes 0..7: F0_k, lanes 8..15: F1_k
+        sm.lay[16 + lane] = lo;                         // the same as rank thresholds
     }
     __syncwarp();
     const int *off = sm.lay;  // layer k holds ranks [off[k], off[k + 8]) (layer 7: negative ranks)
@@ -756,9 +782,14 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         const int r = 32 * m + lane;
         const float wv = sm.w[r];
         const float aw = fabsf(wv);
-        const int K = wv < 0.0f ? 8 : 7;
-        const int ktop = abs_code(aw, sJ1, K);
-        const int kbot = abs_code(aw, sJ0, K);
+        // |q| at s_J0 and s_J1: the layers whose rank threshold r has passed
+        int ktop = (wv < 0.0f && r >= sm.lay[16 + 15]) ? 1 : 0;
+        int kbot = (wv < 0.0f && r >= sm.lay[16 + 7]) ? 1 : 0;
+#pragma unroll
+        for (int k = 0; k < 7; k++) {
+            ktop += r >= sm.lay[16 + 8 + k];
+            kbot += r >= sm.lay[16 + k];
+        }
         const float fk = static_cast<float>(ktop);
 #pragma unroll
         for (int e = 0; e < E; e++) {
@@ -1002,7 +1033,22 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         }
         if (lane < nb) {
             const SurvEntry en = ent[base + lane];
-            const RunResult rr = solve_run<E>(A, myB, myC, en.ja, en.jb);
+            // starting guess: the grid point nearest the clamped vertex of the
+            // environment whose own minimum on the run is largest
+            const float sa = grid_value(en.ja), sb = grid_value(en.jb);
+            float L = -INFINITY, vstar = sa;
+#pragma unroll
+            for (int e = 0; e < E; e++) {
+                const float Bf = static_cast<float>(myB[e]), Cf = static_cast<float>(myC[e]);
+                const float v = fminf(fmaxf(__fdividef(Bf, Cf), sa), sb);
+                const float f = fmaf(fmaf(Cf, v, -2.0f * Bf), v, Af[e]);
+                if (f > L) {
+                    L = f;
+                    vstar = v;
+                }
+            }
+            const uint32_t guess = __half_as_ushort(__float2half_rn(vstar));
+            const RunResult rr = solve_run<E>(A, myB, myC, en.ja, en.jb, guess);
             res_lb[base + lane] = rr.lb;
             res_j[base + lane] = static_cast<uint16_t>(rr.j | (rr.uncertain ? kUncertainBit : 0u));
             ub_min = fmin(ub_min, rr.ub);
