@@ -175,13 +175,13 @@ __device__ __forceinline__ void bitonic_sort_128(uint32_t (&key)[4], int lane)
 {
     cx_asc(key[0], key[1]);
     cx_asc(key[3], key[2]);
-#pragma unroll
+#pragma unroll 1
     for (int k = 4; k <= kGroup; k <<= 1) {
         const uint32_t flip = (((4 * lane) & k) != 0) ? 0xFFFFFFFFu : 0u;
 #pragma unroll
         for (int x = 0; x < 4; x++)
             key[x] ^= flip;
-#pragma unroll
+#pragma unroll 1
         for (int lm = k >> 3; lm > 0; lm >>= 1) {
             const bool upper = (lane & lm) != 0;
 #pragma unroll
@@ -362,16 +362,18 @@ __device__ RunResult solve_run(const double (&A)[E], const double (&B)[E], const
     if (!unc) {
         r.lb = __double2float_rd(Sf - delta);
     } else {
-        // max_e of each environment's own minimum over [sa, sb]: a lower bound
+        // max_e of a lower bound of each environment's minimum over [sa, sb]:
+        // a convex quadratic with curvature C lies at most C (sb - sa)^2 / 4
+        // below the smaller of its end values anywhere between them
+        const double h = sb - sa;
         double L = -INFINITY;
 #pragma unroll
         for (int e = 0; e < E; e++) {
-            double v = sb;
-            if (C[e] > 0.0)
-                v = fmin(fmax(B[e] / C[e], sa), sb);
-            L = fmax(L, fma(fma(C[e], v, nb2[e]), v, A[e]));
+            const double Fa = fma(fma(C[e], sa, nb2[e]), sa, A[e]);
+            const double Fb = fma(fma(C[e], sb, nb2[e]), sb, A[e]);
+            L = fmax(L, fmin(Fa, Fb) - 0.25 * C[e] * h * h);
         }
-        r.lb = __double2float_rd(L - delta);
+        r.lb = __double2float_rd(L - 2.0 * delta);
     }
     return r;
 }
@@ -496,7 +498,7 @@ __device__ __forceinline__ void direct_coefficients(const WarpSmem<E> &sm, float
         B[e] = 0.0;
         C[e] = 0.0;
     }
-#pragma unroll
+#pragma unroll 1
     for (int m = 0; m < 4; m++) {
         const int r = 32 * m + lane;
         const float wv = sm.w[r];
@@ -580,7 +582,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     }
     __syncwarp();
     int n7 = 0;
-#pragma unroll
+#pragma unroll 1
     for (int m = 0; m < 4; m++) {
         const uint32_t k = sm.bufB[32 * m + lane];
         const int i = k & 127;
@@ -617,7 +619,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
 #pragma unroll
             for (int e = 0; e < E; e++)
                 acc[c][e] = 0.0f;
-#pragma unroll
+#pragma unroll 1
         for (int m = 0; m < 4; m++) {
             const int r = 32 * m + lane;
             const float wv = sm.w[r];
@@ -667,7 +669,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
             for (int e = 0; e < E; e++)
                 ph[e * (kGroup + 1)] = 0.0f;
         }
-#pragma unroll
+#pragma unroll 1
         for (int m = 0; m < 4; m++) {
             const int r = 32 * m + lane;
             const float wv = sm.w[r];
@@ -694,7 +696,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
 #pragma unroll
             for (int e = 0; e < E; e++)
                 le[e] = 0.0f;
-#pragma unroll
+#pragma unroll 1
             for (int r = kGroup - 8; r < kGroup; r++) {
                 const float wv = sm.w[r];
                 const float ex = fmaxf(fmaf(-(wv < 0.0f ? 8.0f : 7.0f), sl, fabsf(wv)), 0.0f);
@@ -777,7 +779,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         bb[e] = 0.0f;
         bc[e] = 0.0f;
     }
-#pragma unroll
+#pragma unroll 1
     for (int m = 0; m < 4; m++) {
         const int r = 32 * m + lane;
         const float wv = sm.w[r];
@@ -808,33 +810,9 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     __syncwarp();
 
     // ---- 4'. merge the eight layers: 4 x 8 lanes, 2 x 16 lanes, 32 lanes ---
-    {
-        const int mg = lane >> 3, sl = lane & 7;
-        const uint32_t *La = layer + (2 * mg) * kLayerStride;
-        const uint32_t *Lb = layer + (2 * mg + 1) * kLayerStride;
-        const int na = off[2 * mg + 8] - off[2 * mg], nb = off[2 * mg + 9] - off[2 * mg + 1];
-        uint32_t *out = sm.bufB + mg * 260;
-        const int tot = na + nb, ch = (tot + 7) >> 3;
-        merge_range(La, na, Lb, nb, out, min(sl * ch, tot), min(sl * ch + ch, tot));
-        if (sl == 0)
-            out[tot] = kInvalidKey;
-    }
-    __syncwarp();
-    {
-        const int mg = lane >> 4, sl = lane & 15;
-        const uint32_t *La = sm.bufB + (2 * mg) * 260;
-        const uint32_t *Lb = sm.bufB + (2 * mg + 1) * 260;
-        const int na = off[4 * mg + 8] - off[4 * mg] + off[4 * mg + 9] - off[4 * mg + 1];
-        const int nb = off[4 * mg + 10] - off[4 * mg + 2] + off[4 * mg + 11] - off[4 * mg + 3];
-        uint32_t *out = sm.bufA + mg * 520;
-        const int tot = na + nb, ch = (tot + 15) >> 4;
-        merge_range(La, na, Lb, nb, out, min(sl * ch, tot), min(sl * ch + ch, tot));
-        if (sl == 0)
-            out[tot] = kInvalidKey;
-    }
-    __syncwarp();
-    // final level: lane L produces outputs [L*c, L*c + c), stores element x at
-    // bufB[x*32 + L] and sums its outputs' coefficient deltas (fp32)
+    // Level 0 merges layer pairs into bufB, level 1 pairs of those into bufA,
+    // level 2 the last pair into bufB with element x of lane L at x*32 + L,
+    // where lane L produces outputs [L*c, L*c + c) and sums their deltas.
     int na3 = 0, nb3 = 0;
 #pragma unroll
     for (int k = 0; k < 4; k++) {
@@ -843,30 +821,67 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     }
     const int T = na3 + nb3;
     const int c = (T + 31) >> 5;
-    {
-        const uint32_t *La = sm.bufA;
-        const uint32_t *Lb = sm.bufA + 520;
-        const int d0 = min(lane * c, T), d1 = min(lane * c + c, T);
-        int x = 0;
+#pragma unroll 1
+    for (int level = 0; level < 3; level++) {
+        const uint32_t *La, *Lb;
+        int na, nb, d0, d1, obase, ostride;
+        uint32_t *out;
+        if (level == 0) {
+            const int mg = lane >> 3, sl = lane & 7;
+            La = layer + (2 * mg) * kLayerStride;
+            Lb = layer + (2 * mg + 1) * kLayerStride;
+            na = off[2 * mg + 8] - off[2 * mg];
+            nb = off[2 * mg + 9] - off[2 * mg + 1];
+            out = sm.bufB + mg * 260;
+            const int tot = na + nb, ch = (tot + 7) >> 3;
+            d0 = min(sl * ch, tot);
+            d1 = min(sl * ch + ch, tot);
+            if (sl == 0)
+                out[tot] = kInvalidKey;
+        } else if (level == 1) {
+            const int mg = lane >> 4, sl = lane & 15;
+            La = sm.bufB + (2 * mg) * 260;
+            Lb = sm.bufB + (2 * mg + 1) * 260;
+            na = off[4 * mg + 8] - off[4 * mg] + off[4 * mg + 9] - off[4 * mg + 1];
+            nb = off[4 * mg + 10] - off[4 * mg + 2] + off[4 * mg + 11] - off[4 * mg + 3];
+            out = sm.bufA + mg * 520;
+            const int tot = na + nb, ch = (tot + 15) >> 4;
+            d0 = min(sl * ch, tot);
+            d1 = min(sl * ch + ch, tot);
+            if (sl == 0)
+                out[tot] = kInvalidKey;
+        } else {
+            La = sm.bufA;
+            Lb = sm.bufA + 520;
+            na = na3;
+            nb = nb3;
+            out = sm.bufB;
+            d0 = min(lane * c, T);
+            d1 = min(lane * c + c, T);
+        }
+        obase = (level == 2) ? lane - 32 * d0 : 0;
+        ostride = (level == 2) ? 32 : 1;
         if (d0 < d1) {
-            int i = merge_split(La, na3, Lb, nb3, d0);
+            int i = merge_split(La, na, Lb, nb, d0);
             int j = d0 - i;
             uint32_t va = La[i], vb = Lb[j];
-            for (; x < d1 - d0; x++) {
+            for (int o = d0; o < d1; o++) {
                 const bool ta = va < vb;
                 const uint32_t kk = ta ? va : vb;
                 if (ta)
                     va = La[++i];
                 else
                     vb = Lb[++j];
-                sm.bufB[x * 32 + lane] = kk;
-                add_delta32<E>(sm, kk, rbf, rcf);
+                out[obase + o * ostride] = kk;
+                if (level == 2)
+                    add_delta32<E>(sm, kk, rbf, rcf);
             }
         }
-        for (; x < c; x++)
-            sm.bufB[x * 32 + lane] = kInvalidKey;
+        if (level == 2)
+            for (int x = d1 - d0; x < c; x++)
+                sm.bufB[x * 32 + lane] = kInvalidKey;
+        __syncwarp();
     }
-    __syncwarp();
     const uint32_t *keys = sm.bufB;
 
     // ---- 5. suffix across lanes: sums over every position after this lane,
@@ -899,17 +914,19 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     float ub_lane = INFINITY;
     uint32_t next_t = t_after;
     float *lbs = sm.lb();
+    // x = -1 (lane 0 only) is the run below every window transition: [J0, t_0 - 1]
 #pragma unroll 1
-    for (int x = c - 1; x >= 0; --x) {
-        const uint32_t kk = keys[x * 32 + lane];
+    for (int x = c - 1; x >= -1; --x) {
+        const uint32_t kk = (x >= 0) ? keys[x * 32 + lane] : kInvalidKey;
         const bool valid = kk != kInvalidKey;
-        const uint32_t t = valid ? (kk >> 10) : jend;
+        const uint32_t t = valid ? (kk >> 10) : ((x >= 0 || lane != 0) ? jend : J0);
         const bool run = t <= J1 && t != next_t;
         const uint32_t ja = run ? t : J0;
         const uint32_t jb = run ? min(next_t, jend) - 1u : J0;
         float lbv, ubv;
         screen_run32<E>(Af, rbf, rcf, ja, jb, lbv, ubv);
-        lbs[x * 32 + lane] = run ? lbv : INFINITY;
+        if (x >= 0 || lane == 0)
+            lbs[x >= 0 ? x * 32 + lane : 1024] = run ? lbv : INFINITY;
         ub_lane = run ? fminf(ub_lane, ubv) : ub_lane;
         const int r = (kk >> 3) & 127;
         const float aw = valid ? fabsf(sm.w[r]) : 0.0f;
@@ -920,18 +937,10 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
             rbf[e] = fmaf(dd, aw, rbf[e]);
             rcf[e] = fmaf(dd, cc, rcf[e]);
         }
-        next_t = valid ? t : next_t;
+        if (valid)
+            next_t = t;
     }
     const uint32_t t_first = next_t;  // lane 0: t of position 0 (jend if none)
-    if (lane == 0) {
-        float lbv = INFINITY;
-        if (t_first > J0) {
-            float ubv;
-            screen_run32<E>(Af, rbf, rcf, J0, min(t_first, jend) - 1u, lbv, ubv);
-            ub_lane = fminf(ub_lane, ubv);
-        }
-        lbs[1024] = lbv;
-    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
         ub_lane = fminf(ub_lane, __shfl_xor_sync(kFull, ub_lane, o));
@@ -1107,7 +1116,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
 #pragma unroll
         for (int e = 0; e < E; e++)
             acc[e] = 0.0;
-#pragma unroll
+#pragma unroll 1
         for (int m = 0; m < 4; m++) {
             const int r = 32 * m + lane;
             const float wv = sm.w[r];
