@@ -88,7 +88,7 @@ typedef struct {
 } cq_opts;
 
 /* Bytes of device workspace cq_select_scales_ex needs for G groups.  The
- * workspace holds the counters and the fallback queue (4 bytes per group). */
+ * workspace holds the counters and the fallback queue (8 bytes per group). */
 size_t cq_workspace_bytes(int64_t G, int E);
 
 /* Select scales and codes for G groups.

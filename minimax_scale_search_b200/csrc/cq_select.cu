@@ -74,7 +74,7 @@ struct Params {
     double *out_obj;
     uint8_t *out_flags;
     uint32_t *counters;
-    uint32_t *queue;
+    uint2 *queue;  // fallback entries: group, then J0 | J1 << 16 (the grid range to scan)
     int finalist_cap;
     int force_exhaustive;
     double flag_rel_gap;
@@ -446,11 +446,14 @@ __device__ __forceinline__ void write_constant_group(const Params &p, int64_t g,
     }
 }
 
-__device__ __forceinline__ void enqueue(const Params &p, int64_t g, int lane, Tally &tl)
+// Queue group g for the exhaustive pass over grid indices [j0, j1] (a range
+// outside of which no scale can reach the minimum).
+__device__ __forceinline__ void enqueue(const Params &p, int64_t g, int lane, Tally &tl, uint32_t j0 = 1u,
+                                        uint32_t j1 = kLast)
 {
     if (lane == 0) {
         const uint32_t at = atomicAdd(&p.counters[CQ_CNT_QUEUE], 1u);
-        p.queue[at] = static_cast<uint32_t>(g);
+        p.queue[at] = make_uint2(static_cast<uint32_t>(g), j0 | (j1 << 16));
     }
     tl.fallback++;
 }
@@ -963,7 +966,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     const int n_surv = __shfl_sync(kFull, excl, 31);
     tl.survivors += n_surv;
     if (n_surv > kMaxSurvivors) {
-        enqueue(p, g, lane, tl);
+        enqueue(p, g, lane, tl, J0, J1);
         return;
     }
     __syncwarp();
@@ -1094,7 +1097,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     const int total = __shfl_sync(kFull, fx, 31);
     fx -= cnt;
     if (unc_comp || total > p.finalist_cap || total == 0) {
-        enqueue(p, g, lane, tl);
+        enqueue(p, g, lane, tl, J0, J1);
         return;
     }
     int *fin = sm.fin();
@@ -1213,22 +1216,26 @@ template <int E>
 __global__ void __launch_bounds__(kExThreads) exhaustive_kernel(Params p)
 {
     __shared__ float ws[kGroup];
-    __shared__ float ds[E][kGroup];
+    __shared__ double wsd[kGroup];
+    __shared__ double ds[E][kGroup];
     __shared__ Best3 red[kExThreads / 32];
     __shared__ uint32_t nib[kGroup];
     const int tid = threadIdx.x;
     const uint32_t count = p.counters[CQ_CNT_QUEUE];
     for (uint32_t qi = blockIdx.x; qi < count; qi += gridDim.x) {
-        const int64_t g = p.queue[qi];
+        const uint2 qe = p.queue[qi];
+        const int64_t g = qe.x;
+        const uint32_t j0 = qe.y & 0xFFFFu, j1 = qe.y >> 16;
         if (tid < kGroup) {
             ws[tid] = half_value(p.W[g * kGroup + tid]);
+            wsd[tid] = ws[tid];
 #pragma unroll
             for (int e = 0; e < E; e++)
                 ds[e][tid] = diag_ptr(p, g, e)[tid];
         }
         __syncthreads();
         Best3 b{INFINITY, INFINITY, 0u};
-        for (uint32_t j = 1u + tid; j <= kLast; j += kExThreads) {
+        for (uint32_t j = j0 + tid; j <= j1; j += kExThreads) {
             const float s = grid_value(j);
             const double sd = s;
             double acc[E];
@@ -1240,11 +1247,11 @@ __global__ void __launch_bounds__(kExThreads) exhaustive_kernel(Params p)
                 const float w = ws[i];
                 const int aq = abs_code(fabsf(w), s, w < 0.0f ? 8 : 7);
                 const double q = (w < 0.0f) ? -static_cast<double>(aq) : static_cast<double>(aq);
-                const double r = static_cast<double>(w) - sd * q;
+                const double r = wsd[i] - sd * q;
                 const double rr = __dmul_rn(r, r);
 #pragma unroll
                 for (int e = 0; e < E; e++)
-                    acc[e] = __dadd_rn(acc[e], __dmul_rn(static_cast<double>(ds[e][i]), rr));
+                    acc[e] = __dadd_rn(acc[e], __dmul_rn(ds[e][i], rr));
             }
             double v = acc[0];
 #pragma unroll
@@ -1312,7 +1319,7 @@ constexpr size_t kHeaderBytes = 256;
 
 size_t workspace_bytes(int64_t G)
 {
-    const size_t q = static_cast<size_t>(G < 0 ? 0 : G) * sizeof(uint32_t);
+    const size_t q = static_cast<size_t>(G < 0 ? 0 : G) * sizeof(uint2);
     return kHeaderBytes + ((q + 255) / 256) * 256;
 }
 
@@ -1484,7 +1491,7 @@ cq_status cq_select_scales_ex(const uint16_t *W, int64_t G, const float *D, int 
     p.out_obj = out_objective;
     p.out_flags = out_flags;
     p.counters = static_cast<uint32_t *>(workspace);
-    p.queue = reinterpret_cast<uint32_t *>(static_cast<unsigned char *>(workspace) + kHeaderBytes);
+    p.queue = reinterpret_cast<uint2 *>(static_cast<unsigned char *>(workspace) + kHeaderBytes);
     p.finalist_cap = kDefaultFinalists;
     p.force_exhaustive = 0;
     p.flag_rel_gap = 1e-12;

@@ -49,7 +49,7 @@ def test_status_strings_and_version(cq):
 def test_workspace_size(cq):
     assert cq.workspace_bytes(0, 4) == 256
     assert cq.workspace_bytes(1, 4) == 512
-    assert cq.workspace_bytes(3883008, 4) == 256 + 3883008 * 4
+    assert cq.workspace_bytes(3883008, 4) == 256 + 3883008 * 8
 
 
 FAKE = 0x10000  # 16-byte aligned fake device address: every call below fails validation first
