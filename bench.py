@@ -135,6 +135,26 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(inside)}
 
 
+def rank_matrix(rank: int) -> int:
+    """Each rank solves its own matrix of the workload (weak scaling, no data exchange)."""
+    return rank
+
+
+def max_over_ranks(values, dist=None, device=None):
+    """Elementwise max of per-rank timings (the job's time is its slowest rank)."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def job_rate(world: int, groups_per_rank: int, seconds: float) -> float:
+    """Whole-job groups per second: every rank's groups over the slowest rank's time."""
+    return world * groups_per_rank / seconds
+
+
 def gpu_index_for(local_rank: int) -> str:
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     if vis:
@@ -233,8 +253,8 @@ def main():
     dev = torch.device("cuda", local)
 
     from minimax_scale_search_b200 import cq
-    W = synth.make_weights(WORKLOAD, matrix=rank)
-    D = synth.make_diagonals(WORKLOAD, matrix=rank)
+    W = synth.make_weights(WORKLOAD, matrix=rank_matrix(rank))
+    D = synth.make_diagonals(WORKLOAD, matrix=rank_matrix(rank))
     Wg = W.reshape(-1, 128)
     G = Wg.shape[0]
     f32, f64 = counted_flops(Wg, wl.E)
@@ -274,12 +294,9 @@ def main():
     clocks = sampler.stop(w0, w1)
     ms_total = t_start.elapsed_time(t_end)
     kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
-    if dist:
-        t = torch.tensor([ms_total, kernel_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total, kernel_ms = float(t[0]), float(t[1])
+    ms_total, kernel_ms = max_over_ranks([ms_total, kernel_ms], dist, dev)
     ms_step = ms_total / args.steps
-    value = world * G / (ms_step / 1e3)
+    value = job_rate(world, G, ms_step / 1e3)
 
     # ---- end to end through the host-buffer entry point (pinned host memory)
     e2e = None
@@ -297,14 +314,10 @@ def main():
         t0 = time.perf_counter()
         for _ in range(n_e2e):
             cq.select_scales_host(Wn, Dn, out_scales=sn, out_codes=cn)
-        e2e_s = (time.perf_counter() - t0) / n_e2e
-        if dist:
-            t = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_s = float(t[0])
+        e2e_s = max_over_ranks([(time.perf_counter() - t0) / n_e2e], dist, dev)[0]
         dev_s = out_s.cpu().numpy().view(np.uint16)
         assert np.array_equal(dev_s, sn), "host entry point disagrees with the device entry point"
-        e2e = {"value": world * G / e2e_s, "unit": "groups/s", "h2d_bytes_per_step": int(W.nbytes + D.nbytes),
+        e2e = {"value": job_rate(world, G, e2e_s), "unit": "groups/s", "h2d_bytes_per_step": int(W.nbytes + D.nbytes),
                "d2h_bytes_per_step": int(sn.nbytes + cn.nbytes), "ms_per_step": 1e3 * e2e_s, "steps": n_e2e}
 
     p32, p64, mhz, psrc = peaks()
