@@ -55,7 +55,8 @@ typedef enum {
     CQ_ERR_UNSUPPORTED = 2,      /* E > CQ_MAX_E, or G >= 2^32 */
     CQ_ERR_CUDA = 3,             /* a CUDA runtime call failed */
     CQ_ERR_NONFINITE = 4,        /* (cq_read_counters) some group had non-finite/negative input */
-    CQ_ERR_WORKSPACE = 5         /* workspace missing, too small or misaligned */
+    CQ_ERR_WORKSPACE = 5,        /* workspace missing, too small or misaligned */
+    CQ_ERR_TOO_LARGE = 6         /* (cq_select_scales_noalloc) G above CQ_NOALLOC_MAX_GROUPS */
 } cq_status;
 
 /* Indices into the device counters kept in the workspace. */
@@ -125,6 +126,34 @@ cq_status cq_select_scales_ex(const uint16_t *W, int64_t G, const float *D, int 
 cq_status cq_select_scales_host(const uint16_t *W_host, int64_t G, const float *D_host, int E,
                                 int64_t K, uint16_t *out_scales_host, uint32_t *out_codes_host,
                                 void *stream);
+
+/* Largest G that cq_select_scales_noalloc accepts. */
+#define CQ_NOALLOC_MAX_GROUPS (1 << 20)
+
+/* Allocation-free variant of cq_select_scales, for callers that cannot
+ * allocate device memory at call time: code running inside an allocator
+ * callback or under an external memory budget, an embedded runtime whose
+ * device memory is planned up front, or a host thread that must not touch
+ * the CUDA allocator.  It has no counterpart on the method's pages; it is a
+ * property of this library.
+ *
+ * Same arguments, layouts and results as cq_select_scales.  The selection
+ * kernel's scratch (its counters and the exhaustive-fallback queue) lives in
+ * one fixed array of 256 + 8 * CQ_NOALLOC_MAX_GROUPS bytes (about 8 MiB)
+ * compiled into the library, which every GPU that loads the library keeps
+ * until the process exits.  Nothing is allocated or freed: no cudaMalloc, no
+ * cudaFree, no pool or library allocation.
+ *  - G > CQ_NOALLOC_MAX_GROUPS returns CQ_ERR_TOO_LARGE before anything is
+ *    enqueued.
+ *  - The first call on a device looks up that device's address of the array
+ *    (cudaGetSymbolAddress) and keeps it; make that first call before any
+ *    stream capture on the device.
+ *  - Every call uses the same array; the counters in it are cleared on
+ *    `stream` at the start of each call.  Calls whose work overlaps on the
+ *    GPU (on different streams, or from different host threads without
+ *    ordering) race on the array: order them on one stream or otherwise. */
+cq_status cq_select_scales_noalloc(const uint16_t *W, int64_t G, const float *D, int E, int64_t K,
+                                   uint16_t *out_scales, uint32_t *out_codes, void *stream);
 
 /* Copy the workspace counters to host_counters[CQ_NUM_COUNTERS] (host
  * memory).  Synchronises `stream`.  Returns CQ_ERR_NONFINITE when the last

@@ -16,7 +16,8 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libcq.so")
 
-CQ_OK, CQ_ERR_INVALID_ARG, CQ_ERR_UNSUPPORTED, CQ_ERR_CUDA, CQ_ERR_NONFINITE, CQ_ERR_WORKSPACE = range(6)
+CQ_OK, CQ_ERR_INVALID_ARG, CQ_ERR_UNSUPPORTED, CQ_ERR_CUDA, CQ_ERR_NONFINITE, CQ_ERR_WORKSPACE, CQ_ERR_TOO_LARGE = range(7)
+NOALLOC_MAX_GROUPS = 1 << 20
 CQ_NUM_COUNTERS = 8
 COUNTER_NAMES = ("fallback", "near_tie", "nonfinite", "trivial", "finalists", "uncertain", "queue", "survivors")
 FLAG_TRIVIAL, FLAG_FALLBACK, FLAG_NEAR_TIE, FLAG_NONFINITE = 0x01, 0x02, 0x04, 0x08
@@ -26,7 +27,7 @@ MAX_E = 8
 
 # Symbols the C header declares, in declaration order.
 EXPORTS = ("cq_workspace_bytes", "cq_select_scales", "cq_select_scales_ex", "cq_select_scales_host",
-           "cq_read_counters", "cq_status_string", "cq_version")
+           "cq_select_scales_noalloc", "cq_read_counters", "cq_status_string", "cq_version")
 
 
 class CQError(RuntimeError):
@@ -55,6 +56,8 @@ def _load():
                                       ctypes.c_size_t, vp, vp]
     L.cq_select_scales_host.restype = i32
     L.cq_select_scales_host.argtypes = [vp, i64, vp, i32, i64, vp, vp, vp]
+    L.cq_select_scales_noalloc.restype = i32
+    L.cq_select_scales_noalloc.argtypes = [vp, i64, vp, i32, i64, vp, vp, vp]
     L.cq_read_counters.restype = i32
     L.cq_read_counters.argtypes = [vp, vp, vp]
     L.cq_status_string.restype = ctypes.c_char_p
@@ -186,6 +189,23 @@ def select_scales_plain(W, D, K: int | None = None, *, stream=None, out_scales=N
     st = lib.cq_select_scales(_ptr(W), G, _ptr(D), E, K, _ptr(out_scales), _ptr(out_codes),
                               _stream_handle(stream))
     _check(st, "cq_select_scales")
+    return out_scales, out_codes
+
+
+def select_scales_noalloc(W, D, K: int | None = None, *, stream=None, out_scales=None, out_codes=None):
+    """The allocation-free entry point: the library allocates nothing (its
+    scratch is a fixed array inside libcq.so, up to NOALLOC_MAX_GROUPS groups).
+    The outputs are allocated here only when not passed in.  Calls that
+    overlap on the GPU share that scratch and must be ordered on one stream."""
+    import torch
+    G, E, K = _shapes(W, D, K)
+    if out_scales is None:
+        out_scales = torch.empty(G, dtype=torch.int16, device=W.device)
+    if out_codes is None:
+        out_codes = torch.empty((G, WORDS), dtype=torch.int32, device=W.device)
+    st = lib.cq_select_scales_noalloc(_ptr(W), G, _ptr(D), E, K, _ptr(out_scales), _ptr(out_codes),
+                                      _stream_handle(stream))
+    _check(st, "cq_select_scales_noalloc")
     return out_scales, out_codes
 
 

@@ -1457,6 +1457,32 @@ cq_status validate(const uint16_t *W, int64_t G, const float *D, int E, int64_t 
     return CQ_OK;
 }
 
+// Fixed scratch of cq_select_scales_noalloc: counters + fallback queue for up
+// to CQ_NOALLOC_MAX_GROUPS groups.  Host code must not use the symbol as an
+// address; noalloc_scratch() looks up the device address once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kHeaderBytes + CQ_NOALLOC_MAX_GROUPS * sizeof(uint2)];
+void *g_noalloc_ptr[64];
+
+cudaError_t noalloc_scratch(void **ptr)
+{
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess)
+        return err;
+    if (dev < 0 || dev >= 64)
+        return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (err != cudaSuccess)
+            return err;
+        g_noalloc_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_ptr[dev];
+    return cudaSuccess;
+}
+
 }  // namespace cq
 
 using namespace cq;
@@ -1644,6 +1670,21 @@ done:
     return err == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
 }
 
+cq_status cq_select_scales_noalloc(const uint16_t *W, int64_t G, const float *D, int E, int64_t K,
+                                   uint16_t *out_scales, uint32_t *out_codes, void *stream)
+{
+    cq_status st = validate(W, G, D, E, K, out_scales, out_codes);
+    if (st != CQ_OK || G == 0)
+        return st;
+    if (G > CQ_NOALLOC_MAX_GROUPS)
+        return CQ_ERR_TOO_LARGE;
+    void *ws = nullptr;
+    if (noalloc_scratch(&ws) != cudaSuccess)
+        return CQ_ERR_CUDA;
+    return cq_select_scales_ex(W, G, D, E, K, out_scales, out_codes, stream, nullptr, ws, workspace_bytes(G), nullptr,
+                               nullptr);
+}
+
 cq_status cq_read_counters(const void *workspace, uint32_t *host_counters, void *stream)
 {
     if (!workspace || !host_counters)
@@ -1666,6 +1707,7 @@ const char *cq_status_string(cq_status status)
     case CQ_ERR_CUDA: return "CQ_ERR_CUDA: a CUDA runtime call failed";
     case CQ_ERR_NONFINITE: return "CQ_ERR_NONFINITE: non-finite or negative input in some group";
     case CQ_ERR_WORKSPACE: return "CQ_ERR_WORKSPACE: workspace missing, too small or misaligned";
+    case CQ_ERR_TOO_LARGE: return "CQ_ERR_TOO_LARGE: G above the fixed scratch of cq_select_scales_noalloc";
     default: return "unknown cq_status";
     }
 }
