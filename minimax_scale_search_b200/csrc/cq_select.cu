@@ -381,12 +381,12 @@ __device__ RunResult solve_run(const double (&A)[E], const double (&B)[E], const
 // fp32 screen of one run [ja, jb]: a lower bound of min_s max_e F_e (the max
 // over e of each environment's minimum, at its clamped vertex B/C) and an
 // upper bound (max_e F_e at the grid point nearest the binding vertex), each
-// widened by 2^-16 of max_e (A + 2Bs + Cs^2) at the run's right end.  The
-// coefficients carry at most ~40 fp32 roundings of relative size 2^-24 and
-// the evaluation three more, so the true values lie inside the widened bounds.
+// widened by `rel` times max_e (A + 2Bs + Cs^2) at the run's right end.  With
+// every term nonnegative, an fp32 value that passed through n roundings errs
+// by at most n 2^-24 of that sum; `rel` is twice the caller's count.
 template <int E>
 __device__ __forceinline__ void screen_run32(const float (&A)[E], const float (&B)[E], const float (&C)[E],
-                                             uint32_t ja, uint32_t jb, float &lbm, float &ubm)
+                                             uint32_t ja, uint32_t jb, float rel, float &lbm, float &ubm)
 {
     const float sa = grid_value(ja), sb = grid_value(jb);
     float L = -INFINITY, vstar = sa, P = 0.0f;
@@ -407,7 +407,7 @@ __device__ __forceinline__ void screen_run32(const float (&A)[E], const float (&
 #pragma unroll
     for (int e = 1; e < E; e++)
         U = fmaxf(U, fmaf(fmaf(C[e], s, -2.0f * B[e]), s, A[e]));
-    const float m = P * 0x1p-16f;
+    const float m = P * rel;
     lbm = L - m;
     ubm = U + m;
 }
@@ -914,6 +914,10 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     }
 
     // ---- 6. fp32 screen of every run in the window --------------------------
+    // Rounding count of a screened value: the coefficients above the window
+    // (4 per lane + 5 levels), this lane's suffix (c + 5 levels + 1), the
+    // running sum (c), A's conversion (1) and the evaluation (3): 2c + 19.
+    const float rel = static_cast<float>(2 * (2 * c + 19)) * 0x1p-24f;
     float ub_lane = INFINITY;
     uint32_t next_t = t_after;
     float *lbs = sm.lb();
@@ -927,7 +931,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         const uint32_t ja = run ? t : J0;
         const uint32_t jb = run ? min(next_t, jend) - 1u : J0;
         float lbv, ubv;
-        screen_run32<E>(Af, rbf, rcf, ja, jb, lbv, ubv);
+        screen_run32<E>(Af, rbf, rcf, ja, jb, rel, lbv, ubv);
         if (x >= 0 || lane == 0)
             lbs[x >= 0 ? x * 32 + lane : 1024] = run ? lbv : INFINITY;
         ub_lane = run ? fminf(ub_lane, ubv) : ub_lane;
