@@ -99,6 +99,19 @@ __device__ __forceinline__ float grid_value(uint32_t j)
     return sub ? v - 0x1p-14f : v;
 }
 
+// Diagonals of group g: environment e's 128 values start at base + e * stride.
+struct DiagView {
+    const float *base;
+    int64_t stride;
+};
+
+__device__ __forceinline__ DiagView diag_view(const Params &p, int64_t g)
+{
+    if (p.K > 0)
+        return DiagView{p.D + (g % p.gpr) * kGroup, p.K};
+    return DiagView{p.D + g * kGroup, p.G * kGroup};
+}
+
 __device__ __forceinline__ const float *diag_ptr(const Params &p, int64_t g, int e)
 {
     if (p.K > 0)
@@ -386,10 +399,11 @@ __device__ RunResult solve_run(const double (&A)[E], const double (&B)[E], const
 // by at most n 2^-24 of that sum; `rel` is twice the caller's count.
 template <int E>
 __device__ __forceinline__ void screen_run32(const float (&A)[E], const float (&B)[E], const float (&C)[E],
-                                             uint32_t ja, uint32_t jb, float rel, float &lbm, float &ubm)
+                                             uint32_t ja, uint32_t jb, float rel, float amax2, float &lbm,
+                                             float &ubm)
 {
     const float sa = grid_value(ja), sb = grid_value(jb);
-    float L = -INFINITY, vstar = sa, P = 0.0f;
+    float L = -INFINITY, vstar = sa, cmax = C[0];
 #pragma unroll
     for (int e = 0; e < E; e++) {
         const float v = fminf(fmaxf(__fdividef(B[e], C[e]), sa), sb);
@@ -398,7 +412,7 @@ __device__ __forceinline__ void screen_run32(const float (&A)[E], const float (&
             L = f;
             vstar = v;
         }
-        P = fmaxf(P, fmaf(fmaf(C[e], sb, 2.0f * B[e]), sb, A[e]));
+        cmax = fmaxf(cmax, C[e]);
     }
     uint32_t jc = __half_as_ushort(__float2half_rn(vstar));
     jc = min(max(jc, ja), jb);
@@ -407,7 +421,8 @@ __device__ __forceinline__ void screen_run32(const float (&A)[E], const float (&
 #pragma unroll
     for (int e = 1; e < E; e++)
         U = fmaxf(U, fmaf(fmaf(C[e], s, -2.0f * B[e]), s, A[e]));
-    const float m = P * rel;
+    // A + 2Bs + Cs^2 <= 2A + 2Cs^2 for every environment (2Bs <= A + Cs^2 term by term)
+    const float m = fmaf(2.0f * sb * sb, cmax, amax2) * rel;
     lbm = L - m;
     ubm = U + m;
 }
@@ -526,6 +541,7 @@ template <int E>
 __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int lane, Tally &tl)
 {
     // ---- 1. load ---------------------------------------------------------
+    const DiagView dv_g = diag_view(p, g);
     const uint2 wv = *reinterpret_cast<const uint2 *>(p.W + g * kGroup + 4 * lane);
     const uint32_t wb[4] = {wv.x & 0xFFFFu, wv.x >> 16, wv.y & 0xFFFFu, wv.y >> 16};
     bool bad = false, nonzero = false;
@@ -537,7 +553,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     }
 #pragma unroll
     for (int e = 0; e < E; e++) {
-        const float4 dv = *reinterpret_cast<const float4 *>(diag_ptr(p, g, e) + 4 * lane);
+        const float4 dv = *reinterpret_cast<const float4 *>(dv_g.base + e * dv_g.stride + 4 * lane);
         const float dq[4] = {dv.x, dv.y, dv.z, dv.w};
         double a = 0.0;
 #pragma unroll
@@ -594,7 +610,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         sm.w[r] = half_value(bits);
 #pragma unroll
         for (int e = 0; e < E; e++)
-            sm.d[e][r] = diag_ptr(p, g, e)[i];
+            sm.d[e][r] = dv_g.base[e * dv_g.stride + i];
         const bool neg = (k >> 7) != 0u && (bits & 0x8000u) != 0u;
         const unsigned bn = __ballot_sync(kFull, neg);
         sm.negpre[r] = static_cast<uint8_t>(n7 + __popc(bn & ((1u << lane) - 1u)));
@@ -782,18 +798,22 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         bb[e] = 0.0f;
         bc[e] = 0.0f;
     }
+    int th[16];
+#pragma unroll
+    for (int k = 0; k < 16; k++)
+        th[k] = sm.lay[16 + k];
 #pragma unroll 1
     for (int m = 0; m < 4; m++) {
         const int r = 32 * m + lane;
         const float wv = sm.w[r];
         const float aw = fabsf(wv);
         // |q| at s_J0 and s_J1: the layers whose rank threshold r has passed
-        int ktop = (wv < 0.0f && r >= sm.lay[16 + 15]) ? 1 : 0;
-        int kbot = (wv < 0.0f && r >= sm.lay[16 + 7]) ? 1 : 0;
+        int ktop = (wv < 0.0f && r >= th[15]) ? 1 : 0;
+        int kbot = (wv < 0.0f && r >= th[7]) ? 1 : 0;
 #pragma unroll
         for (int k = 0; k < 7; k++) {
-            ktop += r >= sm.lay[16 + 8 + k];
-            kbot += r >= sm.lay[16 + k];
+            ktop += r >= th[8 + k];
+            kbot += r >= th[k];
         }
         const float fk = static_cast<float>(ktop);
 #pragma unroll
@@ -918,6 +938,11 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     // (4 per lane + 5 levels), this lane's suffix (c + 5 levels + 1), the
     // running sum (c), A's conversion (1) and the evaluation (3): 2c + 19.
     const float rel = static_cast<float>(2 * (2 * c + 19)) * 0x1p-24f;
+    float amax2 = Af[0];
+#pragma unroll
+    for (int e = 1; e < E; e++)
+        amax2 = fmaxf(amax2, Af[e]);
+    amax2 *= 2.0f;
     float ub_lane = INFINITY;
     uint32_t next_t = t_after;
     float *lbs = sm.lb();
@@ -931,7 +956,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         const uint32_t ja = run ? t : J0;
         const uint32_t jb = run ? min(next_t, jend) - 1u : J0;
         float lbv, ubv;
-        screen_run32<E>(Af, rbf, rcf, ja, jb, rel, lbv, ubv);
+        screen_run32<E>(Af, rbf, rcf, ja, jb, rel, amax2, lbv, ubv);
         if (x >= 0 || lane == 0)
             lbs[x >= 0 ? x * 32 + lane : 1024] = run ? lbv : INFINITY;
         ub_lane = run ? fminf(ub_lane, ubv) : ub_lane;
