@@ -72,8 +72,11 @@ def peaks():
 
 
 def kernel_source_hash() -> str:
-    p = os.path.join(ROOT, "minimax_scale_search_b200", "csrc", "cq_select.cu")
-    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+    """Hash of the main kernel's sources (its file and the device header it includes)."""
+    h = hashlib.sha256()
+    for name in ("cq_select.cu", "cq_device.cuh"):
+        h.update(open(os.path.join(ROOT, "minimax_scale_search_b200", "csrc", name), "rb").read())
+    return h.hexdigest()[:16]
 
 
 def recorded_traffic(groups: int):
@@ -220,6 +223,124 @@ def run_reference(args, wl):
     print(json.dumps(line), flush=True)
 
 
+def hbm_peak():
+    """(GB/s, source): the measured copy bandwidth, else the recipe's fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "of measured (MEASURED_PEAKS.json hbm_gbs)"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "of fallback (6.65 TB/s)"
+
+
+def time_calls(fn, steps: int, warmup: int, stream):
+    """Mean device ms per call of fn() (CUDA events on the launching stream)."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps
+
+
+def bench_policies(args, wl, W, D, Wd, Dd, dev):
+    """One JSON line per comparison-policy kernel on the same workload: AbsMax
+    (HBM-bound), Pooled-WMSE (pooling + the search at E = 1), the objective of
+    given scales (HBM-bound) and the three-policy reconstruction proxy on its
+    own 4,096-group input."""
+    import torch
+    from minimax_scale_search_b200 import cq, synth
+    stream = torch.cuda.current_stream()
+    G = W.size // 128
+    hbm, hsrc = hbm_peak()
+    p32, p64, _, psrc = peaks()
+    base = {"n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "data": "synthetic",
+            "config": {"workload": wl.name, "groups": G, "E": wl.E, "K": wl.cols,
+                       "l2": "inputs (994 MB of W) larger than the 126 MB L2; no flush"}}
+    lines = []
+    s_abs = torch.empty(G, dtype=torch.int16, device=dev)
+    c_abs = torch.empty((G, 16), dtype=torch.int32, device=dev)
+    ms = time_calls(lambda: cq.absmax_scales(Wd, out_scales=s_abs, out_codes=c_abs), args.steps, args.warmup,
+                    stream)
+    byt = G * (256 + 2 + 64)
+    lines.append(dict(base, metric="AbsMax policy groups/sec", op="absmax", value=G / ms * 1e3, unit="groups/s",
+                      ms_per_step=ms, higher_is_better=True, dtype="f64", gpu_launches=args.steps,
+                      roofline={"bound": "hbm", "achieved": byt / ms / 1e6, "peak": hbm, "unit": "GB/s",
+                                "frac": byt / ms / 1e6 / hbm, "traffic": None, "kernel": "absmax_kernel",
+                                "bytes_per_group": 322, "peak_note": hsrc}))
+
+    s_pool = torch.empty(G, dtype=torch.int16, device=dev)
+    c_pool = torch.empty((G, 16), dtype=torch.int32, device=dev)
+    ws = torch.empty(cq.workspace_bytes(G, 1), dtype=torch.uint8, device=dev)
+    kev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    kms = []
+
+    def pooled():
+        cq.select_scales_pooled(Wd, Dd, wl.cols, out_scales=s_pool, out_codes=c_pool, workspace=ws,
+                                main_events=kev)
+    for _ in range(args.warmup):
+        pooled()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        pooled()
+        kev[1].synchronize()
+        kms.append(kev[0].elapsed_time(kev[1]))
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / args.steps
+    f32, f64 = counted_flops(W.reshape(-1, 128), 1)
+    kernel_ms = statistics.mean(kms)
+    ach = (f32 + f64 * p32 / p64) / (kernel_ms / 1e3) / 1e12
+    lines.append(dict(base, metric="Pooled-WMSE policy groups/sec", op="pooled_wmse", value=G / ms * 1e3,
+                      unit="groups/s", ms_per_step=ms, higher_is_better=True, dtype="f64",
+                      gpu_launches=3 * args.steps,
+                      note="per-step host sync to read the main kernel's events; value from the outer events",
+                      roofline={"bound": "alu", "achieved": ach, "peak": p32, "unit": "TFLOP/s", "frac": ach / p32,
+                                "traffic": None, "kernel": "select_kernel<1>", "kernel_ms": kernel_ms,
+                                "fp32_flops": f32, "fp64_flops": f64, "peak_note": psrc}))
+
+    scales = cq.select_scales(Wd, Dd, wl.cols).scales
+    per_env = torch.empty((G, wl.E), dtype=torch.float64, device=dev)
+    obj = torch.empty(G, dtype=torch.float64, device=dev)
+    ms = time_calls(lambda: cq.group_objective(Wd, Dd, scales, wl.cols, per_env=per_env, out=obj), args.steps,
+                    args.warmup, stream)
+    bpg = 256 + 2 + 8 * wl.E + 8
+    byt = G * bpg
+    lines.append(dict(base, metric="objective of given scales groups/sec", op="objective", value=G / ms * 1e3,
+                      unit="groups/s", ms_per_step=ms, higher_is_better=True, dtype="f64",
+                      gpu_launches=2 * args.steps,
+                      roofline={"bound": "hbm", "achieved": byt / ms / 1e6, "peak": hbm, "unit": "GB/s",
+                                "frac": byt / ms / 1e6 / hbm, "traffic": None,
+                                "kernel": "objective_kernel + env_max_kernel", "bytes_per_group": bpg,
+                                "peak_note": hsrc}))
+
+    Wp, Dp, offsets = synth.make_proxy_inputs()
+    Wpd = torch.from_numpy(Wp.view(np.int16)).to(dev)
+    Dpd = torch.from_numpy(Dp).to(dev)
+    t = []
+    for k in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        res = cq.evaluate_policies(Wpd, Dpd, offsets)
+        if k >= args.warmup:
+            t.append(time.perf_counter() - t0)
+    ms = 1e3 * statistics.mean(t)
+    lines.append(dict(base, metric="reconstruction proxy, three policies, ms per evaluation", op="proxy",
+                      value=ms, unit="ms", ms_per_step=ms, higher_is_better=False, dtype="f64",
+                      gpu_launches=18 * args.steps,
+                      config={"workload": "proxy-4096-groups-150-modules-E4", "groups": int(Wp.shape[0]),
+                              "modules": len(offsets) - 1, "E": 4, "diagonals": "per-group [4, 4096, 128] fp32"},
+                      timing="host wall clock per call, including three device-to-host reads",
+                      proxy={p: v[0] for p, v in res.items()}))
+    for ln in lines:
+        print(json.dumps(ln), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -228,6 +349,8 @@ def main():
     ap.add_argument("--impl", default="cq", choices=["cq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--op", default="select", choices=["select", "policies"],
+                    help="select: the headline line; policies: one line per comparison-policy kernel")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -264,6 +387,11 @@ def main():
     out_c = torch.empty((G, 16), dtype=torch.int32, device=dev)
     ws = torch.empty(cq.workspace_bytes(G, wl.E), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
+    if args.op == "policies":
+        if world > 1:
+            ap.error("--op policies runs on one GPU")
+        bench_policies(args, wl, W, D, Wd, Dd, dev)
+        return
 
     def step(evs=None):
         return cq.select_scales(Wd, Dd, wl.cols, out_scales=out_s, out_codes=out_c, workspace=ws,

@@ -127,6 +127,52 @@ cq_status cq_select_scales_host(const uint16_t *W_host, int64_t G, const float *
                                 int64_t K, uint16_t *out_scales_host, uint32_t *out_codes_host,
                                 void *stream);
 
+/* ---- comparison policies and the reconstruction proxy ----------------------
+ * The project page's "Held-out reconstruction proxy" table (and the model
+ * card's section of the same name) compares CliffQuant's minimax scales with
+ * two policies, Pooled-WMSE and AbsMax, on the "module-macro worst-environment
+ * weighted MSE".  These entry points compute those policies and that proxy
+ * on the GPU.  All pointers are device pointers; all are asynchronous on
+ * `stream`; argument errors return before anything is enqueued. */
+
+/* AbsMax policy (the matched baseline checkpoint's scales): per group
+ * s = binary16 nearest (ties to even) to max_i |w_i| / 7 computed in fp64,
+ * raised to 0x0001 when that rounds to 0 (all-zero groups); codes are the
+ * quantiser's at s, packed like cq_select_scales.  A group with a non-finite
+ * weight gets scale 0x0001 and zero codes.
+ *  W [G][128] binary16 bits (16-byte aligned); out_scales [G]; out_codes [G][16]. */
+cq_status cq_absmax_scales(const uint16_t *W, int64_t G, uint16_t *out_scales, uint32_t *out_codes, void *stream);
+
+/* Pooled diagonals for the Pooled-WMSE policy: out[i] = fp32, rounded to
+ * nearest even, of (sum over e = 0..E-1 of D[e*n + i], summed in fp64 in that
+ * order) / E.  D is [E][n] fp32 (n = K for per-column, G*128 for per-group
+ * diagonals); out is [n].  The policy is cq_select_scales with E = 1 on out. */
+cq_status cq_pool_diagonals(const float *D, int E, int64_t n, float *out, void *stream);
+
+/* Objective of given scales (the proxy's per-group term): per_env[g*E + e] =
+ * sum_i d_{e,i} (w_i - s q_i(s))^2 in fp64, summed over i ascending without
+ * fused multiply-adds, and out_objective[g] = max_e of those; s = scales[g]
+ * (binary16 bits).  W and D as for cq_select_scales; per_env [G][E] and
+ * out_objective [G] are fp64 and 8-byte aligned.  The result is undefined for
+ * non-finite input. */
+cq_status cq_group_objective(const uint16_t *W, int64_t G, const float *D, int E, int64_t K,
+                             const uint16_t *scales, double *per_env, double *out_objective,
+                             void *stream);
+
+/* Module-macro worst-environment weighted MSE, from cq_group_objective's
+ * per_env output [G][E].  Module m holds groups offsets[m] .. offsets[m+1]-1
+ * (offsets: nmod+1 ascending int64 on the device, clamped to [0, G] so that no
+ * read leaves per_env); then
+ *   module_env[m*E + e] = scale * (sum of per_env[g*E + e] over its groups) / count,
+ *   module_worst[m]     = max_e module_env[m*E + e],
+ *   macro[0]            = mean over m of module_worst[m].
+ * With scale = 1/128 these are per-weight means.  Sums use a fixed order, so
+ * the results are deterministic; a module with no groups gives NaN.  All
+ * pointers are 8-byte-aligned device pointers. */
+cq_status cq_reconstruction_proxy(const double *per_env, int64_t G, int E, int64_t nmod,
+                                  const int64_t *offsets, double scale, double *module_env,
+                                  double *module_worst, double *macro, void *stream);
+
 /* Largest G that cq_select_scales_noalloc accepts. */
 #define CQ_NOALLOC_MAX_GROUPS (1 << 20)
 

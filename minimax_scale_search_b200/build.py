@@ -11,8 +11,8 @@ import sys
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
-SRC = os.path.join(PKG, "csrc", "cq_select.cu")
-HDR = os.path.join(ROOT, "include", "cq.h")
+SRCS = [os.path.join(PKG, "csrc", "cq_select.cu"), os.path.join(PKG, "csrc", "cq_policies.cu")]
+DEPS = SRCS + [os.path.join(PKG, "csrc", "cq_device.cuh"), os.path.join(ROOT, "include", "cq.h")]
 LIB = os.path.join(PKG, "libcq.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -25,12 +25,11 @@ def nvcc() -> str:
 
 
 def build(force: bool = False, ptxas_verbose: bool = False, out: str = LIB) -> str:
-    deps = [SRC, HDR]
-    if not force and os.path.exists(out) and all(os.path.getmtime(out) >= os.path.getmtime(d) for d in deps):
+    if not force and os.path.exists(out) and all(os.path.getmtime(out) >= os.path.getmtime(d) for d in DEPS):
         return out
     tmp = out + f".tmp{os.getpid()}"
     cmd = [nvcc(), "-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC", "-shared",
-           "-I", os.path.join(ROOT, "include"), "-o", tmp, SRC]
+           "-I", os.path.join(ROOT, "include"), "-o", tmp, *SRCS]
     if ptxas_verbose:
         cmd[1:1] = ["-Xptxas", "-v"]
     subprocess.check_call(cmd)

@@ -27,6 +27,7 @@ MAX_E = 8
 
 # Symbols the C header declares, in declaration order.
 EXPORTS = ("cq_workspace_bytes", "cq_select_scales", "cq_select_scales_ex", "cq_select_scales_host",
+           "cq_absmax_scales", "cq_pool_diagonals", "cq_group_objective", "cq_reconstruction_proxy",
            "cq_select_scales_noalloc", "cq_read_counters", "cq_status_string", "cq_version")
 
 
@@ -56,6 +57,14 @@ def _load():
                                       ctypes.c_size_t, vp, vp]
     L.cq_select_scales_host.restype = i32
     L.cq_select_scales_host.argtypes = [vp, i64, vp, i32, i64, vp, vp, vp]
+    L.cq_absmax_scales.restype = i32
+    L.cq_absmax_scales.argtypes = [vp, i64, vp, vp, vp]
+    L.cq_pool_diagonals.restype = i32
+    L.cq_pool_diagonals.argtypes = [vp, i32, i64, vp, vp]
+    L.cq_group_objective.restype = i32
+    L.cq_group_objective.argtypes = [vp, i64, vp, i32, i64, vp, vp, vp, vp]
+    L.cq_reconstruction_proxy.restype = i32
+    L.cq_reconstruction_proxy.argtypes = [vp, i64, i32, i64, vp, ctypes.c_double, vp, vp, vp, vp]
     L.cq_select_scales_noalloc.restype = i32
     L.cq_select_scales_noalloc.argtypes = [vp, i64, vp, i32, i64, vp, vp, vp]
     L.cq_read_counters.restype = i32
@@ -232,6 +241,120 @@ def select_scales_host(W, D, K: int | None = None, *, stream=None, out_scales=No
                                    _stream_handle(stream))
     _check(st, "cq_select_scales_host")
     return out_scales, out_codes
+
+
+def _check_w(W):
+    if not W.is_cuda or W.element_size() != 2 or not W.is_contiguous():
+        raise ValueError("W must be a contiguous CUDA tensor of 16-bit binary16 patterns")
+    if W.dim() != 2 or W.shape[-1] % GROUP:
+        raise ValueError("W must be 2-D with a multiple of 128 columns")
+
+
+def absmax_scales(W, *, stream=None, out_scales=None, out_codes=None):
+    """AbsMax policy: s = fp16(max|w| / 7) per group (at least the smallest
+    positive pattern) and the codes at s.  Returns (scales int16 [G], codes int32 [G, 16])."""
+    import torch
+    _check_w(W)
+    G = W.numel() // GROUP
+    if out_scales is None:
+        out_scales = torch.empty(G, dtype=torch.int16, device=W.device)
+    if out_codes is None:
+        out_codes = torch.empty((G, WORDS), dtype=torch.int32, device=W.device)
+    _check(lib.cq_absmax_scales(_ptr(W), G, _ptr(out_scales), _ptr(out_codes), _stream_handle(stream)),
+           "cq_absmax_scales")
+    return out_scales, out_codes
+
+
+def pool_diagonals(D, *, stream=None, out=None):
+    """Mean of the environments' diagonals (fp64 sum in environment order,
+    rounded once to fp32): [E, ...] -> [1, ...], the input of Pooled-WMSE."""
+    import torch
+    if not D.is_cuda or D.dtype != torch.float32 or not D.is_contiguous() or D.dim() < 2:
+        raise ValueError("D must be a contiguous CUDA float32 tensor [E, ...]")
+    E = D.shape[0]
+    n = D.numel() // E
+    if out is None:
+        out = torch.empty((1,) + tuple(D.shape[1:]), dtype=torch.float32, device=D.device)
+    _check(lib.cq_pool_diagonals(_ptr(D), E, n, _ptr(out), _stream_handle(stream)), "cq_pool_diagonals")
+    return out
+
+
+def select_scales_pooled(W, D, K: int | None = None, **kw) -> Result:
+    """Pooled-WMSE policy: the exact search with one environment whose
+    diagonal is the mean of D's environments."""
+    return select_scales(W, pool_diagonals(D, stream=kw.get("stream")), K, **kw)
+
+
+def group_objective(W, D, scales, K: int | None = None, *, stream=None, per_env=None, out=None):
+    """Objective of given scales: (max_e objective float64 [G], per-environment
+    objectives float64 [G, E]), each an fp64 sum over the group in index order."""
+    import torch
+    _check_w(W)
+    if not D.is_cuda or D.dtype != torch.float32 or not D.is_contiguous():
+        raise ValueError("D must be a contiguous CUDA float32 tensor")
+    G, E, K = _shapes(W, D, K)
+    if scales.numel() != G or scales.element_size() != 2 or not scales.is_contiguous():
+        raise ValueError("scales must hold G 16-bit patterns")
+    if per_env is None:
+        per_env = torch.empty((G, E), dtype=torch.float64, device=W.device)
+    if out is None:
+        out = torch.empty(G, dtype=torch.float64, device=W.device)
+    _check(lib.cq_group_objective(_ptr(W), G, _ptr(D), E, K, _ptr(scales), _ptr(per_env), _ptr(out),
+                                  _stream_handle(stream)), "cq_group_objective")
+    return out, per_env
+
+
+def reconstruction_proxy(per_env, offsets, scale: float = 1.0 / GROUP, *, stream=None):
+    """Module-macro worst-environment weighted MSE from per-environment group
+    objectives [G, E] and module offsets (int64, nmod + 1).  Returns
+    (module_env float64 [nmod, E], module_worst [nmod], macro [1]) on the device."""
+    import torch
+    if per_env.dtype != torch.float64 or per_env.dim() != 2 or not per_env.is_contiguous():
+        raise ValueError("per_env must be a contiguous float64 [G, E] tensor")
+    G, E = per_env.shape
+    off = np.asarray(offsets.cpu() if hasattr(offsets, "cpu") else offsets, dtype=np.int64).ravel()
+    if off.size < 1 or off[0] < 0 or off[-1] > G or np.any(np.diff(off) < 0):
+        raise ValueError("offsets must ascend from >= 0 to <= the number of groups")
+    offsets = torch.from_numpy(off).to(per_env.device)
+    nmod = off.size - 1
+    dev = per_env.device
+    module_env = torch.empty((max(nmod, 0), E), dtype=torch.float64, device=dev)
+    module_worst = torch.empty(max(nmod, 0), dtype=torch.float64, device=dev)
+    macro = torch.full((1,), float("nan"), dtype=torch.float64, device=dev)
+    _check(lib.cq_reconstruction_proxy(_ptr(per_env), G, E, nmod, _ptr(offsets), float(scale), _ptr(module_env),
+                                       _ptr(module_worst), _ptr(macro), _stream_handle(stream)),
+           "cq_reconstruction_proxy")
+    return module_env, module_worst, macro
+
+
+POLICIES = ("cliffquant", "pooled_wmse", "absmax")
+
+
+def policy_scales(policy: str, W, D, K: int | None = None, *, stream=None):
+    """(scales, codes) of one of POLICIES on the device."""
+    if policy == "cliffquant":
+        r = select_scales(W, D, K, stream=stream)
+        return r.scales, r.codes
+    if policy == "pooled_wmse":
+        r = select_scales_pooled(W, D, K, stream=stream)
+        return r.scales, r.codes
+    if policy == "absmax":
+        return absmax_scales(W, stream=stream)
+    raise ValueError(f"unknown policy {policy!r}; expected one of {POLICIES}")
+
+
+def evaluate_policies(W, D, offsets, K: int | None = None, *, policies=POLICIES, stream=None) -> dict:
+    """The reconstruction proxy for each policy: {policy: (macro, module_worst
+    numpy [nmod], scales)}; every step on the device, one host read per policy."""
+    out = {}
+    for pol in policies:
+        scales, _ = policy_scales(pol, W, D, K, stream=stream)
+        _, per_env = group_objective(W, D, scales, K, stream=stream)
+        _, worst, macro = reconstruction_proxy(per_env, offsets, stream=stream)
+        if stream is not None:
+            stream.synchronize()
+        out[pol] = (float(macro.cpu()[0]), worst.cpu().numpy(), scales)
+    return out
 
 
 def read_counters(workspace, stream=None) -> dict:

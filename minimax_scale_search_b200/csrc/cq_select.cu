@@ -48,12 +48,10 @@
 #include <mutex>
 
 #include "cq.h"
+#include "cq_device.cuh"
 
 namespace cq {
 
-constexpr int kGroup = 128;
-constexpr uint32_t kLast = 0x7BFFu;    // largest finite binary16 pattern (65504)
-constexpr uint32_t kBeyond = 0x7C00u;  // one past the grid
 constexpr int kWarps = 4;              // warps (groups in flight) per CTA of the main kernel
 constexpr uint32_t kInvalidKey = 0xFFFFFFFFu;
 constexpr int kMaxFinalists = 64;
@@ -61,7 +59,6 @@ constexpr int kDefaultFinalists = 32;
 constexpr int kMaxSurvivors = 128;  // runs passing the fp32 screen before the exhaustive fallback
 constexpr int kWalkMax = 16;        // longest delta walk between survivors before a direct sum
 constexpr uint32_t kUncertainBit = 0x8000u;
-constexpr unsigned kFull = 0xFFFFFFFFu;
 
 struct Params {
     const uint16_t *W;
@@ -82,23 +79,6 @@ struct Params {
     cudaEvent_t ev_end;
 };
 
-__device__ __forceinline__ float half_value(uint32_t bits)
-{
-    return __half2float(__ushort_as_half(static_cast<unsigned short>(bits)));
-}
-
-// Value of a positive binary16 pattern j in [1, 0x7C00] (0x7C00 gives 65536),
-// built from bits without a conversion instruction: for j >= 0x400 the fp32
-// pattern is (j << 13) + 0x38000000; for subnormal halves the same construction
-// with the exponent one higher gives 2^-14 + j 2^-24, and 2^-14 is subtracted
-// exactly.
-__device__ __forceinline__ float grid_value(uint32_t j)
-{
-    const bool sub = j < 0x400u;
-    const float v = __uint_as_float((j << 13) + (sub ? 0x38800000u : 0x38000000u));
-    return sub ? v - 0x1p-14f : v;
-}
-
 // Diagonals of group g: environment e's 128 values start at base + e * stride.
 struct DiagView {
     const float *base;
@@ -117,27 +97,6 @@ __device__ __forceinline__ const float *diag_ptr(const Params &p, int64_t g, int
     if (p.K > 0)
         return p.D + static_cast<int64_t>(e) * p.K + (g % p.gpr) * kGroup;
     return p.D + (static_cast<int64_t>(e) * p.G + g) * kGroup;
-}
-
-// |q| >= m for |w| = aw at scale s, before clipping: round-half-even(aw/s) >= m.
-// s * (m - 1/2) is exact in fp32 (11-bit s times a 5-bit odd/2 factor).
-__device__ __forceinline__ bool code_at_least(float aw, float s, int m)
-{
-    const float t = s * (static_cast<float>(m) - 0.5f);
-    return aw > t || (aw == t && (m & 1) == 0);
-}
-
-// min(round-half-even(aw / s), K), exact: an fp32 estimate corrected by the
-// exact threshold tests above (the estimate is within one of the answer).
-__device__ __forceinline__ int abs_code(float aw, float s, int K)
-{
-    const float x = fminf(__fdividef(aw, s), 15.0f);
-    int n = __float2int_rn(x);
-    if (n > 0 && !code_at_least(aw, s, n))
-        n -= 1;
-    else if (code_at_least(aw, s, n + 1))
-        n += 1;
-    return min(n, K);
 }
 
 // 1 / (k + 1/2), k = 0..7 (only an estimate's accuracy is needed).
@@ -161,15 +120,6 @@ __device__ __forceinline__ uint32_t transition_index(float aw, int k)
     if (j0 == kBeyond || !code_at_least(aw, grid_value(j0), k + 1))
         return j0;
     return j0 + 1;
-}
-
-template <typename T>
-__device__ __forceinline__ T warp_sum(T v)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        v += __shfl_xor_sync(kFull, v, o);
-    return v;
 }
 
 __device__ __forceinline__ void cx_asc(uint32_t &a, uint32_t &b)

@@ -29,6 +29,14 @@ Workloads (sizes follow the 0.8B model card's scale run of 3,883,008 groups):
               nonzero N(0, 0.02) weight at a uniform position
 5. large      32 matrices of 14336 x 4096, N(0, 0.015), 0.2% x12, E=4,
               lognormal(0, 1.5), one diagonal set per matrix
+
+Proxy inputs (``make_proxy_inputs``; project page, "Held-out reconstruction
+proxy": 4,096 groups sampled across 150 target matrices): the groups are split
+over the modules as evenly as possible, the first ``groups % modules`` modules
+taking one more.  Module m draws N(0, sigma_m) weights, sigma_m = 0.02 *
+2^U(-1, 1), with 0.5% of entries x8, and its own E lognormal(0, 1.5)
+diagonals over 4096 columns, each environment divided by its fp64 mean; each
+of its groups takes a uniformly drawn 128-column block of those diagonals.
 """
 from __future__ import annotations
 
@@ -44,6 +52,7 @@ ROW_BLOCK = 256
 _KIND_DIAG = 0
 _KIND_ROWS = 1
 _KIND_CLASS = 2
+_KIND_PROXY = 3
 
 
 @dataclass(frozen=True)
@@ -226,3 +235,36 @@ def sample_groups(idx: int, count: int, seed: int = 7, matrix: int = 0) -> np.nd
     count = min(count, wl.groups_per_matrix)
     rng = _rng(seed, 9, idx, matrix)
     return np.sort(rng.choice(wl.groups_per_matrix, size=count, replace=False))
+
+
+PROXY_GROUPS = 4096
+PROXY_MODULES = 150
+_PROXY_COLS = 4096
+
+
+def proxy_offsets(groups: int = PROXY_GROUPS, modules: int = PROXY_MODULES) -> np.ndarray:
+    """int64 [modules + 1]: module m holds groups offsets[m] .. offsets[m+1]-1."""
+    base, extra = divmod(groups, modules)
+    sizes = np.full(modules, base, dtype=np.int64)
+    sizes[:extra] += 1
+    return np.concatenate([[0], np.cumsum(sizes)]).astype(np.int64)
+
+
+def make_proxy_inputs(groups: int = PROXY_GROUPS, modules: int = PROXY_MODULES, E: int = 4,
+                      seed: int = 1006):
+    """(W uint16 [G, 128], per-group D fp32 [E, G, 128], offsets int64 [modules + 1])."""
+    offsets = proxy_offsets(groups, modules)
+    W = np.empty((groups, GROUP), dtype=np.uint16)
+    D = np.empty((E, groups, GROUP), dtype=np.float32)
+    for m in range(modules):
+        a, b = int(offsets[m]), int(offsets[m + 1])
+        rng = _rng(seed, _KIND_PROXY, m)
+        sigma = 0.02 * 2.0 ** rng.uniform(-1.0, 1.0)
+        w = _outliers(rng, rng.normal(0.0, sigma, (b - a, GROUP)), 0.005, 8.0)
+        W[a:b] = w.astype(np.float16).view(np.uint16)
+        d = rng.lognormal(0.0, 1.5, size=(E, _PROXY_COLS))
+        d = (d / d.mean(axis=1, keepdims=True)).astype(np.float32)
+        blocks = rng.integers(0, _PROXY_COLS // GROUP, b - a)
+        for k, c in enumerate(blocks):
+            D[:, a + k, :] = d[:, c * GROUP:(c + 1) * GROUP]
+    return W, D, offsets

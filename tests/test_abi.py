@@ -96,6 +96,46 @@ def test_plain_and_host_entry_points_validate(cq):
     assert cq.lib.cq_read_counters(vp(None), vp(FAKE), vp(None)) == cq.CQ_ERR_INVALID_ARG
 
 
+def test_policy_entry_points_validate(cq):
+    vp, L = ctypes.c_void_p, cq.lib
+    f = vp(FAKE)
+    # AbsMax: W [G][128] binary16, 16-byte aligned
+    assert L.cq_absmax_scales(f, -1, f, f, vp(None)) == cq.CQ_ERR_INVALID_ARG
+    assert L.cq_absmax_scales(f, 1 << 32, f, f, vp(None)) == cq.CQ_ERR_UNSUPPORTED
+    assert L.cq_absmax_scales(vp(None), 0, vp(None), vp(None), vp(None)) == cq.CQ_OK
+    assert L.cq_absmax_scales(vp(FAKE + 8), 4, f, f, vp(None)) == cq.CQ_ERR_INVALID_ARG
+    assert L.cq_absmax_scales(f, 4, f, vp(FAKE + 2), vp(None)) == cq.CQ_ERR_INVALID_ARG
+    assert L.cq_absmax_scales(f, 4, vp(None), f, vp(None)) == cq.CQ_ERR_INVALID_ARG
+    # pooling: 1 <= E <= 8
+    assert L.cq_pool_diagonals(f, 0, 10, f, vp(None)) == cq.CQ_ERR_INVALID_ARG
+    assert L.cq_pool_diagonals(f, 9, 10, f, vp(None)) == cq.CQ_ERR_UNSUPPORTED
+    assert L.cq_pool_diagonals(f, 4, -1, f, vp(None)) == cq.CQ_ERR_INVALID_ARG
+    assert L.cq_pool_diagonals(vp(None), 4, 0, vp(None), vp(None)) == cq.CQ_OK
+    assert L.cq_pool_diagonals(vp(None), 4, 10, f, vp(None)) == cq.CQ_ERR_INVALID_ARG
+    # objective of given scales
+    obj = lambda G=8, E=4, K=0, W=FAKE, D=FAKE, S=FAKE, P=FAKE, O=FAKE: L.cq_group_objective(  # noqa: E731
+        vp(W), G, vp(D), E, K, vp(S), vp(P), vp(O), vp(None))
+    assert obj(E=0) == cq.CQ_ERR_INVALID_ARG
+    assert obj(E=9) == cq.CQ_ERR_UNSUPPORTED
+    assert obj(G=-1) == cq.CQ_ERR_INVALID_ARG
+    assert obj(K=100) == cq.CQ_ERR_INVALID_ARG
+    assert obj(G=9, K=256) == cq.CQ_ERR_INVALID_ARG
+    assert obj(S=0) == cq.CQ_ERR_INVALID_ARG
+    assert obj(P=FAKE + 4) == cq.CQ_ERR_INVALID_ARG
+    assert obj(G=0, W=0, D=0, S=0, P=0, O=0) == cq.CQ_OK
+    # proxy reductions
+    prox = lambda G=8, E=4, nmod=3, scale=1.0, X=FAKE, off=FAKE: L.cq_reconstruction_proxy(  # noqa: E731
+        vp(X), G, E, nmod, vp(off), scale, f, f, f, vp(None))
+    assert prox(G=-1) == cq.CQ_ERR_INVALID_ARG
+    assert prox(E=0) == cq.CQ_ERR_INVALID_ARG
+    assert prox(E=9) == cq.CQ_ERR_UNSUPPORTED
+    assert prox(nmod=-1) == cq.CQ_ERR_INVALID_ARG
+    assert prox(scale=float("nan")) == cq.CQ_ERR_INVALID_ARG
+    assert prox(X=FAKE + 4) == cq.CQ_ERR_INVALID_ARG
+    assert prox(off=0) == cq.CQ_ERR_INVALID_ARG
+    assert prox(nmod=0, X=0, off=0) == cq.CQ_OK
+
+
 def test_no_cpu_fallback_in_binding():
     """The binding refuses to run without its CUDA library."""
     src = open(os.path.join(ROOT, "minimax_scale_search_b200", "cq.py")).read()
