@@ -140,7 +140,7 @@ cq_status cq_select_scales_host(const uint16_t *W_host, int64_t G, const float *
  * raised to 0x0001 when that rounds to 0 (all-zero groups); codes are the
  * quantiser's at s, packed like cq_select_scales.  A group with a non-finite
  * weight gets scale 0x0001 and zero codes.
- *  W [G][128] binary16 bits (16-byte aligned); out_scales [G]; out_codes [G][16]. */
+ *  W [G][128] binary16 bits and out_codes [G][16] 16-byte aligned; out_scales [G]. */
 cq_status cq_absmax_scales(const uint16_t *W, int64_t G, uint16_t *out_scales, uint32_t *out_codes, void *stream);
 
 /* Pooled diagonals for the Pooled-WMSE policy: out[i] = fp32, rounded to
@@ -152,9 +152,9 @@ cq_status cq_pool_diagonals(const float *D, int E, int64_t n, float *out, void *
 /* Objective of given scales (the proxy's per-group term): per_env[g*E + e] =
  * sum_i d_{e,i} (w_i - s q_i(s))^2 in fp64, summed over i ascending without
  * fused multiply-adds, and out_objective[g] = max_e of those; s = scales[g]
- * (binary16 bits).  W and D as for cq_select_scales; per_env [G][E] and
- * out_objective [G] are fp64 and 8-byte aligned.  The result is undefined for
- * non-finite input. */
+ * (binary16 bits).  W and D as for cq_select_scales (both 16-byte aligned);
+ * per_env [G][E] and out_objective [G] are fp64 and 8-byte aligned.  The
+ * result is undefined for non-finite input. */
 cq_status cq_group_objective(const uint16_t *W, int64_t G, const float *D, int E, int64_t K,
                              const uint16_t *scales, double *per_env, double *out_objective,
                              void *stream);

@@ -20,60 +20,116 @@
 namespace cq {
 namespace {
 
-constexpr int kPolicyWarps = 8;
-constexpr int kGroupsPerWarp = 4;  // loads in flight per warp
+constexpr int kStageWarps = 4;   // warps per CTA of the staged kernels
+constexpr int kRowPitch = 272;   // bytes per staged 256-byte row: the 16-byte pad puts the 16-byte reads
+                                 // of 8 consecutive rows (one shared-memory phase) on disjoint banks
+constexpr int kStageBytes = 32 * kRowPitch;
+
+// Stage 32 rows of 128 binary16 weights (row r at W + row_of(r) * 128, rows
+// r >= n skipped) into shared memory: 16 coalesced 16-byte loads per lane in
+// two batches of 8 (4 KB in flight per warp), streaming past L1.
+template <typename RowOf>
+__device__ __forceinline__ void stage_rows(uint8_t *sm, const uint16_t *__restrict__ W, int n, int lane,
+                                           RowOf row_of)
+{
+#pragma unroll
+    for (int half = 0; half < 2; half++) {
+        uint4 v[8];
+#pragma unroll
+        for (int k = 0; k < 8; k++) {
+            const int c = (8 * half + k) * 32 + lane, r = c >> 4;
+            v[k] = (r < n) ? __ldcs(reinterpret_cast<const uint4 *>(W + row_of(r) * kGroup) + (c & 15))
+                           : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; k++) {
+            const int c = (8 * half + k) * 32 + lane;
+            *reinterpret_cast<uint4 *>(sm + (c >> 4) * kRowPitch + (c & 15) * 16) = v[k];
+        }
+    }
+}
+
+// min(round-half-even(aw / s), cap) for aw >= 0, exact.  The estimate
+// aw * (1/s) is within one of the answer; adding 1.5 * 2^23 rounds it to the
+// nearest integer (ties even) in the low mantissa bits, and the exact
+// threshold tests s (n -+ 1/2) (11-bit s times a 5-bit factor) correct it.
+__device__ __forceinline__ int code_of(float aw, float s, float inv, int cap)
+{
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+    const float y = fminf(aw * inv, 15.0f) + kRound;
+    const float n = y - kRound;
+    const int ni = __float_as_int(y) - 0x4B400000;
+    const float lo = s * (n - 0.5f), hi = s * (n + 0.5f);
+    const bool odd = ni & 1;
+    const int below = (aw < lo || (aw == lo && odd)) ? 1 : 0;  // rne < n
+    const int above = (aw > hi || (aw == hi && odd)) ? 1 : 0;  // rne > n
+    return min(ni - below + above, cap);
+}
 
 // AbsMax: s = binary16 nearest (ties even) to max_i |w_i| / 7 computed in
 // fp64, raised to the smallest positive pattern when it rounds to 0; codes are
 // the quantiser's at s.  Non-finite weights give scale 0x0001 and zero codes,
-// as in the minimax kernel.  One warp per group, four groups per iteration.
-__global__ void __launch_bounds__(kPolicyWarps * 32) absmax_kernel(const uint16_t *__restrict__ W, int64_t G,
-                                                                   uint16_t *__restrict__ out_scales,
-                                                                   uint32_t *__restrict__ out_codes)
+// as in the minimax kernel.  One thread per group; each warp stages 32
+// consecutive groups and writes their codes back as contiguous 16-byte stores.
+__global__ void __launch_bounds__(kStageWarps * 32) absmax_kernel(const uint16_t *__restrict__ W, int64_t G,
+                                                                  uint16_t *__restrict__ out_scales,
+                                                                  uint32_t *__restrict__ out_codes)
 {
+    __shared__ __align__(16) uint8_t stage[kStageWarps][kStageBytes];
     const int lane = threadIdx.x & 31;
-    const int64_t warp = static_cast<int64_t>(blockIdx.x) * kPolicyWarps + (threadIdx.x >> 5);
-    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kPolicyWarps;
-    for (int64_t g0 = warp * kGroupsPerWarp; g0 < G; g0 += nwarps * kGroupsPerWarp) {
-        uint2 wv[kGroupsPerWarp];
+    uint8_t *sm = stage[threadIdx.x >> 5];
+    uint8_t *row = sm + lane * kRowPitch;
+    const int64_t chunks = (G + 31) / 32;
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * kStageWarps + (threadIdx.x >> 5); t < chunks;
+         t += static_cast<int64_t>(gridDim.x) * kStageWarps) {
+        const int64_t g0 = t * 32;
+        const int n = static_cast<int>(min(static_cast<int64_t>(32), G - g0));
+        __syncwarp();
+        stage_rows(sm, W, n, lane, [g0](int r) { return g0 + r; });
+        __syncwarp();
+        if (lane < n) {
+            uint32_t m2 = 0;
 #pragma unroll
-        for (int u = 0; u < kGroupsPerWarp; u++)
-            wv[u] = (g0 + u < G) ? reinterpret_cast<const uint2 *>(W + (g0 + u) * kGroup)[lane] : make_uint2(0, 0);
-#pragma unroll
-        for (int u = 0; u < kGroupsPerWarp; u++) {
-            const int64_t g = g0 + u;
-            if (g >= G)
-                break;
-            const uint32_t wb[4] = {wv[u].x & 0xFFFFu, wv[u].x >> 16, wv[u].y & 0xFFFFu, wv[u].y >> 16};
-            uint32_t mag = 0;
-#pragma unroll
-            for (int m = 0; m < 4; m++)
-                mag = max(mag, wb[m] & 0x7FFFu);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1)
-                mag = max(mag, __shfl_xor_sync(kFull, mag, o));
+            for (int j = 0; j < 16; j++) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(row + j * 16);
+                m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                                           __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu)));
+            }
+            const uint32_t mag = max(m2 & 0xFFFFu, m2 >> 16);
             uint32_t sbits = 1u;
-            if (mag < 0x7C00u) {
+            if (mag < kBeyond) {
                 const double amax = static_cast<double>(half_value(mag));
-                sbits = __half_as_ushort(__double2half(amax / 7.0));
-                sbits = min(max(sbits, 1u), kLast);
+                sbits = min(max(static_cast<uint32_t>(__half_as_ushort(__double2half(amax / 7.0))), 1u), kLast);
             }
             const float s = grid_value(sbits);
-            uint32_t h = 0;
+            const float inv = 1.0f / s;
+            // code word j (8 nibbles) overwrites bytes 4j..4j+3 of the row, which chunk j has already passed
+#pragma unroll 4
+            for (int j = 0; j < 16; j++) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(row + j * 16);
+                const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+                uint32_t word = 0x88888888u;
+                if (mag < kBeyond) {
+                    word = 0;
 #pragma unroll
-            for (int m = 0; m < 4; m++) {
-                int q = 0;
-                if (mag < 0x7C00u) {
-                    const int aq = abs_code(half_value(wb[m] & 0x7FFFu), s, (wb[m] & 0x8000u) ? 8 : 7);
-                    q = (wb[m] & 0x8000u) ? -aq : aq;
+                    for (int h = 0; h < 8; h++) {
+                        const uint32_t b = (wd[h >> 1] >> (16 * (h & 1))) & 0xFFFFu;
+                        const bool neg = b & 0x8000u;
+                        const int c = code_of(half_value(b & 0x7FFFu), s, inv, neg ? 8 : 7);
+                        word |= static_cast<uint32_t>(((neg ? -c : c) + 8) & 0xF) << (4 * h);
+                    }
                 }
-                h |= static_cast<uint32_t>((q + 8) & 0xF) << (4 * m);
+                *reinterpret_cast<uint32_t *>(row + 4 * j) = word;
             }
-            const uint32_t up = __shfl_down_sync(kFull, h, 1);
-            if ((lane & 1) == 0)
-                out_codes[g * 16 + (lane >> 1)] = h | (up << 16);
-            if (lane == 0)
-                out_scales[g] = static_cast<uint16_t>(sbits);
+            out_scales[g0 + lane] = static_cast<uint16_t>(sbits);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            const int c = k * 32 + lane, r = c >> 2;
+            if (r < n)
+                reinterpret_cast<uint4 *>(out_codes + (g0 + r) * 16)[c & 3] =
+                    *reinterpret_cast<const uint4 *>(sm + r * kRowPitch + (c & 3) * 16);
         }
     }
 }
@@ -91,44 +147,90 @@ __global__ void pool_kernel(const float *__restrict__ D, int E, int64_t n, float
     }
 }
 
-// Objective of given scales: out[g] = max_e sum_i d_{e,i} (w_i - s q_i)^2 in
-// fp64, summed over i ascending without contraction (the definition's own
-// order).  One thread per (group, environment) pair.
-__global__ void objective_kernel(const uint16_t *__restrict__ W, int64_t G, const float *__restrict__ D, int E,
-                                 int64_t K, const uint16_t *__restrict__ scales, double *__restrict__ out)
+// Objective of given scales: per_env[g][e] = sum_i d_{e,i} (w_i - s q_i)^2 in
+// fp64, the products and sums rounded in the definition's own order (i
+// ascending, r = w - s q exact, then r*r, then d*rr, then the running sum; no
+// contraction), and out[g] = max_e of those.  One thread per group.
+//
+// Per-column diagonals (K > 0): a CTA takes 128 rows of one column block, so
+// all its threads share that block's diagonals, which it stages once in fp64
+// and reads back as broadcasts.  Per-group diagonals (K == 0): a warp takes 32
+// consecutive groups and each thread streams its own.
+template <int E, bool kPerColumn>
+__global__ void __launch_bounds__(kStageWarps * 32) objective_kernel(const uint16_t *__restrict__ W, int64_t G,
+                                                                     const float *__restrict__ D, int64_t K,
+                                                                     const uint16_t *__restrict__ scales,
+                                                                     double *__restrict__ per_env,
+                                                                     double *__restrict__ out)
 {
-    const int64_t pairs = G * E;
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    const int64_t gpr = K > 0 ? K / kGroup : 1;
-    for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < pairs; t += stride) {
-        const int64_t g = t / E;
-        const int e = static_cast<int>(t - g * E);
-        const uint16_t *w = W + g * kGroup;
-        const float *d = (K > 0) ? D + e * K + (g % gpr) * kGroup : D + (static_cast<int64_t>(e) * G + g) * kGroup;
-        const uint32_t sb = scales[g];
-        const float s = grid_value(sb);
-        const double sd = s;
-        double acc = 0.0;
-        for (int i = 0; i < kGroup; i++) {
-            const uint32_t b = w[i];
-            const int aq = abs_code(half_value(b & 0x7FFFu), s, (b & 0x8000u) ? 8 : 7);
-            const double q = (b & 0x8000u) ? -static_cast<double>(aq) : static_cast<double>(aq);
-            const double r = static_cast<double>(half_value(b)) - sd * q;  // exact
-            acc = __dadd_rn(acc, __dmul_rn(static_cast<double>(d[i]), __dmul_rn(r, r)));
+    __shared__ __align__(16) uint8_t stage[kStageWarps][kStageBytes];
+    __shared__ double dstage[kPerColumn ? E : 1][kGroup];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    uint8_t *sm = stage[wid];
+    const uint8_t *row = sm + lane * kRowPitch;
+    const int64_t gpr = kPerColumn ? K / kGroup : 1;
+    const int64_t rows = G / gpr;
+    constexpr int kRowsPerItem = kPerColumn ? 32 * kStageWarps : 32;
+    const int64_t items = kPerColumn ? ((rows + kRowsPerItem - 1) / kRowsPerItem) * gpr : (G + 31) / 32;
+    const int64_t first = kPerColumn ? blockIdx.x : static_cast<int64_t>(blockIdx.x) * kStageWarps + wid;
+    const int64_t step = kPerColumn ? gridDim.x : static_cast<int64_t>(gridDim.x) * kStageWarps;
+    for (int64_t t = first; t < items; t += step) {
+        const int64_t cb = kPerColumn ? t % gpr : 0;
+        const int64_t r0 = kPerColumn ? (t / gpr) * kRowsPerItem + 32 * wid : t * 32;
+        const int n = static_cast<int>(max(min(static_cast<int64_t>(32), (kPerColumn ? rows : G) - r0),
+                                           static_cast<int64_t>(0)));
+        if (kPerColumn) {
+            __syncthreads();  // the previous item's diagonals are no longer read
+            for (int e = wid; e < E; e += kStageWarps) {
+                const float4 d4 = __ldg(reinterpret_cast<const float4 *>(D + e * K + cb * kGroup) + lane);
+                dstage[e][4 * lane] = d4.x;
+                dstage[e][4 * lane + 1] = d4.y;
+                dstage[e][4 * lane + 2] = d4.z;
+                dstage[e][4 * lane + 3] = d4.w;
+            }
         }
-        out[t] = acc;
-    }
-}
-
-__global__ void env_max_kernel(const double *__restrict__ per_env, int64_t G, int E, double *__restrict__ out)
-{
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < G; g += stride) {
-        double f = per_env[g * E];
-        for (int e = 1; e < E; e++) {
-            const double v = per_env[g * E + e];
-            if (v > f)
-                f = v;
+        __syncwarp();
+        stage_rows(sm, W, n, lane, [=](int r) { return (r0 + r) * gpr + cb; });
+        if (kPerColumn)
+            __syncthreads();
+        else
+            __syncwarp();
+        if (lane >= n)
+            continue;
+        const int64_t g = (r0 + lane) * gpr + cb;
+        const float s = grid_value(scales[g]);
+        const float inv = 1.0f / s;
+        const double nsd = -static_cast<double>(s);
+        double acc[E];
+#pragma unroll
+        for (int e = 0; e < E; e++)
+            acc[e] = 0.0;
+        const float *dg = kPerColumn ? nullptr : D + g * kGroup;
+#pragma unroll 1
+        for (int j = 0; j < 16; j++) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(row + j * 16);
+            const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int h = 0; h < 8; h++) {
+                const uint32_t bits = (wd[h >> 1] >> (16 * (h & 1))) & 0xFFFFu;
+                const bool neg = bits & 0x8000u;
+                const int c = code_of(half_value(bits & 0x7FFFu), s, inv, neg ? 8 : 7);
+                const double r = fma(nsd, static_cast<double>(neg ? -c : c), static_cast<double>(half_value(bits)));
+                const double rr = __dmul_rn(r, r);
+#pragma unroll
+                for (int e = 0; e < E; e++) {
+                    const double d = kPerColumn ? dstage[e][8 * j + h]
+                                                : static_cast<double>(__ldcs(dg + e * G * kGroup + 8 * j + h));
+                    acc[e] = __dadd_rn(acc[e], __dmul_rn(d, rr));
+                }
+            }
+        }
+        double f = acc[0];
+#pragma unroll
+        for (int e = 0; e < E; e++) {
+            per_env[g * E + e] = acc[e];
+            if (acc[e] > f)
+                f = acc[e];
         }
         out[g] = f;
     }
@@ -216,6 +318,36 @@ bool is_aligned(const void *p, size_t a)
     return (reinterpret_cast<uintptr_t>(p) % a) == 0;
 }
 
+// Grid of a grid-stride kernel over `chunks` warp-sized work items: as many
+// CTAs as fit on the device at once, fewer when there is less work.
+template <typename Kernel>
+unsigned resident_grid(Kernel kernel, int64_t chunks, int chunks_per_cta = kStageWarps)
+{
+    int per_sm = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kStageWarps * 32, 0) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    const int64_t cap = static_cast<int64_t>(sms_of_current()) * per_sm;
+    const int64_t need = (chunks + chunks_per_cta - 1) / chunks_per_cta;
+    return static_cast<unsigned>(need < cap ? need : cap);
+}
+
+template <int E>
+cudaError_t launch_objective(const uint16_t *W, int64_t G, const float *D, int64_t K, const uint16_t *scales,
+                             double *per_env, double *out, cudaStream_t st)
+{
+    if (K > 0) {
+        const int64_t rows_per_item = 32 * kStageWarps;
+        const int64_t items = ((G / (K / kGroup) + rows_per_item - 1) / rows_per_item) * (K / kGroup);
+        auto k = objective_kernel<E, true>;
+        k<<<resident_grid(k, items, 1), kStageWarps * 32, 0, st>>>(W, G, D, K, scales, per_env, out);
+    } else {
+        auto k = objective_kernel<E, false>;
+        k<<<resident_grid(k, (G + 31) / 32), kStageWarps * 32, 0, st>>>(W, G, D, K, scales, per_env, out);
+    }
+    return cudaGetLastError();
+}
+
 }  // namespace
 }  // namespace cq
 
@@ -231,16 +363,11 @@ cq_status cq_absmax_scales(const uint16_t *W, int64_t G, uint16_t *out_scales, u
         return CQ_ERR_UNSUPPORTED;
     if (G == 0)
         return CQ_OK;
-    if (!W || !out_scales || !out_codes || !is_aligned(W, 16) || !is_aligned(out_codes, 4) ||
+    if (!W || !out_scales || !out_codes || !is_aligned(W, 16) || !is_aligned(out_codes, 16) ||
         !is_aligned(out_scales, 2))
         return CQ_ERR_INVALID_ARG;
-    const int64_t warps = (G + kGroupsPerWarp - 1) / kGroupsPerWarp;
-    int64_t blocks = (warps + kPolicyWarps - 1) / kPolicyWarps;
-    const int64_t cap = static_cast<int64_t>(sms_of_current()) * 8;
-    if (blocks > cap)
-        blocks = cap;
-    absmax_kernel<<<static_cast<unsigned>(blocks), kPolicyWarps * 32, 0, static_cast<cudaStream_t>(stream)>>>(
-        W, G, out_scales, out_codes);
+    absmax_kernel<<<resident_grid(absmax_kernel, (G + 31) / 32), kStageWarps * 32, 0,
+                    static_cast<cudaStream_t>(stream)>>>(W, G, out_scales, out_codes);
     return cudaGetLastError() == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
 }
 
@@ -273,19 +400,23 @@ cq_status cq_group_objective(const uint16_t *W, int64_t G, const float *D, int E
         return CQ_ERR_INVALID_ARG;
     if (G == 0)
         return CQ_OK;
-    if (!W || !D || !scales || !per_env || !out_objective || !is_aligned(per_env, 8) ||
-        !is_aligned(out_objective, 8))
+    if (!W || !D || !scales || !per_env || !out_objective || !is_aligned(W, 16) || !is_aligned(D, 16) ||
+        !is_aligned(scales, 2) || !is_aligned(per_env, 8) || !is_aligned(out_objective, 8))
         return CQ_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int64_t cap = static_cast<int64_t>(sms_of_current()) * 16;
-    int64_t blocks = (G * E + 255) / 256;
-    objective_kernel<<<static_cast<unsigned>(blocks < cap ? blocks : cap), 256, 0, st>>>(W, G, D, E, K, scales,
-                                                                                          per_env);
-    if (cudaGetLastError() != cudaSuccess)
-        return CQ_ERR_CUDA;
-    blocks = (G + 255) / 256;
-    env_max_kernel<<<static_cast<unsigned>(blocks < cap ? blocks : cap), 256, 0, st>>>(per_env, G, E, out_objective);
-    return cudaGetLastError() == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
+    cudaError_t err = cudaErrorInvalidValue;
+    switch (E) {
+    case 1: err = launch_objective<1>(W, G, D, K, scales, per_env, out_objective, st); break;
+    case 2: err = launch_objective<2>(W, G, D, K, scales, per_env, out_objective, st); break;
+    case 3: err = launch_objective<3>(W, G, D, K, scales, per_env, out_objective, st); break;
+    case 4: err = launch_objective<4>(W, G, D, K, scales, per_env, out_objective, st); break;
+    case 5: err = launch_objective<5>(W, G, D, K, scales, per_env, out_objective, st); break;
+    case 6: err = launch_objective<6>(W, G, D, K, scales, per_env, out_objective, st); break;
+    case 7: err = launch_objective<7>(W, G, D, K, scales, per_env, out_objective, st); break;
+    case 8: err = launch_objective<8>(W, G, D, K, scales, per_env, out_objective, st); break;
+    default: break;
+    }
+    return err == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
 }
 
 cq_status cq_reconstruction_proxy(const double *per_env, int64_t G, int E, int64_t nmod, const int64_t *offsets,

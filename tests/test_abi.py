@@ -105,6 +105,7 @@ def test_policy_entry_points_validate(cq):
     assert L.cq_absmax_scales(vp(None), 0, vp(None), vp(None), vp(None)) == cq.CQ_OK
     assert L.cq_absmax_scales(vp(FAKE + 8), 4, f, f, vp(None)) == cq.CQ_ERR_INVALID_ARG
     assert L.cq_absmax_scales(f, 4, f, vp(FAKE + 2), vp(None)) == cq.CQ_ERR_INVALID_ARG
+    assert L.cq_absmax_scales(f, 4, f, vp(FAKE + 4), vp(None)) == cq.CQ_ERR_INVALID_ARG  # codes need 16 B
     assert L.cq_absmax_scales(f, 4, vp(None), f, vp(None)) == cq.CQ_ERR_INVALID_ARG
     # pooling: 1 <= E <= 8
     assert L.cq_pool_diagonals(f, 0, 10, f, vp(None)) == cq.CQ_ERR_INVALID_ARG
@@ -122,6 +123,8 @@ def test_policy_entry_points_validate(cq):
     assert obj(G=9, K=256) == cq.CQ_ERR_INVALID_ARG
     assert obj(S=0) == cq.CQ_ERR_INVALID_ARG
     assert obj(P=FAKE + 4) == cq.CQ_ERR_INVALID_ARG
+    assert obj(D=FAKE + 4) == cq.CQ_ERR_INVALID_ARG
+    assert obj(W=FAKE + 8) == cq.CQ_ERR_INVALID_ARG
     assert obj(G=0, W=0, D=0, S=0, P=0, O=0) == cq.CQ_OK
     # proxy reductions
     prox = lambda G=8, E=4, nmod=3, scale=1.0, X=FAKE, off=FAKE: L.cq_reconstruction_proxy(  # noqa: E731
