@@ -341,6 +341,52 @@ def bench_policies(args, wl, W, D, Wd, Dd, dev):
         print(json.dumps(ln), flush=True)
 
 
+def bench_gptq(args, wl, dev):
+    """One JSON line each for the GPTQ v1 export and dequantisation of the
+    sweep's layer shape (random codes and scales: the format steps do not
+    depend on their values)."""
+    import torch
+    from minimax_scale_search_b200 import cq, synth
+    stream = torch.cuda.current_stream()
+    R, K = wl.rows, wl.cols
+    G = R * K // 128
+    hbm, hsrc = hbm_peak()
+    scales, codes = synth.make_codes(G)
+    S = torch.from_numpy(scales.view(np.int16)).to(dev)
+    C = torch.from_numpy(codes.view(np.int32)).to(dev)
+    t = cq.gptq_export(S, C, R, K)
+    base = {"n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "data": "synthetic", "unit": "groups/s",
+            "higher_is_better": True, "dtype": "u32",
+            "config": {"workload": f"gptq-v1-{R}x{K}", "groups": G, "R": R, "K": K,
+                       "l2": "tensors (>= 248 MB each) larger than the 126 MB L2; no flush"}}
+    lines = []
+    ms = time_calls(lambda: cq.gptq_export(S, C, R, K), args.steps, args.warmup, stream)
+    bpg = 64 + 2 + 64 + 2 + 0.5  # codes and scales in, qweight, scales and qzeros out
+    lines.append(dict(base, metric="GPTQ v1 export groups/sec", op="gptq_export", value=G / ms * 1e3,
+                      ms_per_step=ms, gpu_launches=3 * args.steps,
+                      roofline={"bound": "hbm", "achieved": G * bpg / ms / 1e6, "peak": hbm, "unit": "GB/s",
+                                "frac": G * bpg / ms / 1e6 / hbm, "traffic": None,
+                                "kernel": "transpose_kernel<uint32_t> (+ scales transpose, fills)",
+                                "bytes_per_group": bpg, "peak_note": hsrc}))
+    for half in (True, False):
+        out = torch.empty((R, K), dtype=torch.float16 if half else torch.float32, device=dev)
+        fn = lambda: cq.lib.cq_gptq_dequantize(  # noqa: E731
+            cq._ptr(t.qweight), cq._ptr(t.qzeros), cq._ptr(t.scales), cq._ptr(t.g_idx), R, K, int(half),
+            cq._ptr(out), cq._stream_handle(stream))
+        ms = time_calls(fn, args.steps, args.warmup, stream)
+        bpg = 64 + 2 + 0.5 + 128 * (2 if half else 4)
+        lines.append(dict(base, metric=f"GPTQ v1 dequantisation to {'fp16' if half else 'fp32'} groups/sec",
+                          op="gptq_dequant_fp16" if half else "gptq_dequant_fp32", value=G / ms * 1e3,
+                          ms_per_step=ms, gpu_launches=args.steps, dtype="f16" if half else "f32",
+                          roofline={"bound": "hbm", "achieved": G * bpg / ms / 1e6, "peak": hbm, "unit": "GB/s",
+                                    "frac": G * bpg / ms / 1e6 / hbm, "traffic": None,
+                                    "kernel": f"dequant_kernel<{'true' if half else 'false'}>",
+                                    "bytes_per_group": bpg, "peak_note": hsrc}))
+        del out
+    for ln in lines:
+        print(json.dumps(ln), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -349,8 +395,8 @@ def main():
     ap.add_argument("--impl", default="cq", choices=["cq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--op", default="select", choices=["select", "policies"],
-                    help="select: the headline line; policies: one line per comparison-policy kernel")
+    ap.add_argument("--op", default="select", choices=["select", "policies", "gptq"],
+                    help="select: the headline line; policies / gptq: one line per kernel of those rows")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -376,6 +422,11 @@ def main():
     dev = torch.device("cuda", local)
 
     from minimax_scale_search_b200 import cq
+    if args.op == "gptq":
+        if world > 1:
+            ap.error("--op gptq runs on one GPU")
+        bench_gptq(args, wl, dev)
+        return
     W = synth.make_weights(WORKLOAD, matrix=rank_matrix(rank))
     D = synth.make_diagonals(WORKLOAD, matrix=rank_matrix(rank))
     Wg = W.reshape(-1, 128)

@@ -173,6 +173,33 @@ cq_status cq_reconstruction_proxy(const double *per_env, int64_t G, int E, int64
                                   const int64_t *offsets, double scale, double *module_env,
                                   double *module_worst, double *macro, void *stream);
 
+/* ---- GPTQ v1 tensors --------------------------------------------------------
+ * The project page and the model card ("Quantization configuration") release
+ * a GPTQ v1 checkpoint: 4-bit, group size 128, symmetric, act-order off.  The
+ * pages do not print the layout; these follow the public GPTQ v1 format for a
+ * linear layer with weight [R][K] (R outputs, K inputs, groups along K as in
+ * cq_select_scales with per-column diagonals):
+ *   qweight int32 [K/8][R]     inputs 8k..8k+7 of output r, input 8k+j in bits 4j..4j+3
+ *   qzeros  int32 [K/128][R/8] zero points of outputs 8c..8c+7, stored minus one (0x77777777)
+ *   scales  fp16  [K/128][R]   binary16 bits
+ *   g_idx   int32 [K]          i / 128
+ * Requires K % 128 == 0 and R % 8 == 0 (else CQ_ERR_INVALID_ARG).  All
+ * pointers are device pointers with their element's alignment. */
+
+/* Export: from the selection's scales [R*K/128] and packed codes [R*K/128][16]
+ * (group r*(K/128) + c is row r, columns 128c..128c+127) to the four tensors. */
+cq_status cq_gptq_export(const uint16_t *scales, const uint32_t *codes, int64_t R, int64_t K,
+                         int32_t *qweight, int32_t *qzeros, uint16_t *gptq_scales, int32_t *g_idx,
+                         void *stream);
+
+/* Dequantisation by the v1 rule w[r][i] = scales[g][r] * (u - (z + 1)), g = g_idx[i]
+ * (clamped to [0, K/128)), into out [R][K] (16-byte aligned): fp32 when
+ * out_fp16 == 0 (exact), binary16 rounded to nearest even when out_fp16 == 1.
+ * Reads only the four tensors: an unpacker independent of the export. */
+cq_status cq_gptq_dequantize(const int32_t *qweight, const int32_t *qzeros, const uint16_t *gptq_scales,
+                             const int32_t *g_idx, int64_t R, int64_t K, int out_fp16, void *out,
+                             void *stream);
+
 /* Largest G that cq_select_scales_noalloc accepts. */
 #define CQ_NOALLOC_MAX_GROUPS (1 << 20)
 

@@ -28,6 +28,7 @@ MAX_E = 8
 # Symbols the C header declares, in declaration order.
 EXPORTS = ("cq_workspace_bytes", "cq_select_scales", "cq_select_scales_ex", "cq_select_scales_host",
            "cq_absmax_scales", "cq_pool_diagonals", "cq_group_objective", "cq_reconstruction_proxy",
+           "cq_gptq_export", "cq_gptq_dequantize",
            "cq_select_scales_noalloc", "cq_read_counters", "cq_status_string", "cq_version")
 
 
@@ -65,6 +66,10 @@ def _load():
     L.cq_group_objective.argtypes = [vp, i64, vp, i32, i64, vp, vp, vp, vp]
     L.cq_reconstruction_proxy.restype = i32
     L.cq_reconstruction_proxy.argtypes = [vp, i64, i32, i64, vp, ctypes.c_double, vp, vp, vp, vp]
+    L.cq_gptq_export.restype = i32
+    L.cq_gptq_export.argtypes = [vp, vp, i64, i64, vp, vp, vp, vp, vp]
+    L.cq_gptq_dequantize.restype = i32
+    L.cq_gptq_dequantize.argtypes = [vp, vp, vp, vp, i64, i64, i32, vp, vp]
     L.cq_select_scales_noalloc.restype = i32
     L.cq_select_scales_noalloc.argtypes = [vp, i64, vp, i32, i64, vp, vp, vp]
     L.cq_read_counters.restype = i32
@@ -354,6 +359,46 @@ def evaluate_policies(W, D, offsets, K: int | None = None, *, policies=POLICIES,
         if stream is not None:
             stream.synchronize()
         out[pol] = (float(macro.cpu()[0]), worst.cpu().numpy(), scales)
+    return out
+
+
+@dataclass
+class GPTQTensors:
+    """GPTQ v1 tensors of one linear layer with weight [R, K] (R outputs, K inputs)."""
+    qweight: "object"  # torch.int32 [K/8, R]
+    qzeros: "object"   # torch.int32 [K/128, R/8]
+    scales: "object"   # torch.float16 [K/128, R]
+    g_idx: "object"    # torch.int32 [K]
+
+    def as_dict(self) -> dict:
+        return {"qweight": self.qweight, "qzeros": self.qzeros, "scales": self.scales, "g_idx": self.g_idx}
+
+
+def gptq_export(scales, codes, R: int, K: int, *, stream=None) -> GPTQTensors:
+    """GPTQ v1 tensors from the selection's scales [R*K/128] and codes [R*K/128, 16]
+    (groups along the rows of an [R, K] weight)."""
+    import torch
+    G = R * K // GROUP
+    if scales.numel() != G or codes.numel() != G * WORDS or not (scales.is_contiguous() and codes.is_contiguous()):
+        raise ValueError("scales and codes must hold R*K/128 contiguous groups")
+    dev = codes.device
+    t = GPTQTensors(torch.empty((K // 8, R), dtype=torch.int32, device=dev),
+                    torch.empty((K // GROUP, R // 8), dtype=torch.int32, device=dev),
+                    torch.empty((K // GROUP, R), dtype=torch.float16, device=dev),
+                    torch.empty(K, dtype=torch.int32, device=dev))
+    _check(lib.cq_gptq_export(_ptr(scales), _ptr(codes), R, K, _ptr(t.qweight), _ptr(t.qzeros), _ptr(t.scales),
+                              _ptr(t.g_idx), _stream_handle(stream)), "cq_gptq_export")
+    return t
+
+
+def gptq_dequantize(t: GPTQTensors, *, half: bool = False, stream=None):
+    """[R, K] weights by the v1 rule: float32 (exact) or float16 (rounded to nearest even)."""
+    import torch
+    K = t.qweight.shape[0] * 8
+    R = t.qweight.shape[1]
+    out = torch.empty((R, K), dtype=torch.float16 if half else torch.float32, device=t.qweight.device)
+    _check(lib.cq_gptq_dequantize(_ptr(t.qweight), _ptr(t.qzeros), _ptr(t.scales), _ptr(t.g_idx), R, K,
+                                  int(bool(half)), _ptr(out), _stream_handle(stream)), "cq_gptq_dequantize")
     return out
 
 

@@ -1,0 +1,219 @@
+// GPTQ v1 tensors from the selection's output, and their dequantisation.
+//
+// CliffQuant project page and the model card, "Quantization configuration":
+// the release is a GPTQ v1 checkpoint, 4-bit, group size 128, symmetric,
+// act-order off.  Layout (public GPTQ v1 format) for a linear layer with
+// weight [R, K], R output features and K input features:
+//   qweight int32 [K/8][R]     word (k, r): inputs 8k..8k+7 of output r, input 8k+j in bits 4j..4j+3
+//   qzeros  int32 [K/128][R/8] word (g, c): zero points of outputs 8c..8c+7, stored minus one
+//   scales  fp16  [K/128][R]
+//   g_idx   int32 [K]          i / 128
+// and w[r][i] = scales[g][r] * (u - (z + 1)) with g = g_idx[i].
+//
+// The selection's codes of group (r, c) are 16 words of 8 input-adjacent
+// nibbles (q + 8), low nibble first: word j of group (r, c) is exactly
+// qweight[16c + j][r].  So the export is a transpose of the [R][K/8] word
+// matrix, a transpose of the [R][K/128] scale matrix and two constant fills;
+// all are HBM-bound and run as 32 x 32 tiles through shared memory (reads and
+// writes both coalesced).
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "cq.h"
+
+namespace cq {
+namespace {
+
+constexpr int kTile = 32;
+constexpr int kTileRowsPerPass = 8;  // CTA of 32 x 8 threads, 4 elements per thread
+
+// dst[c][r] = src[r][c] for an [rows][cols] matrix, one 32 x 32 tile per CTA
+// iteration (grid-stride over tiles).
+template <typename T>
+__global__ void __launch_bounds__(kTile * kTileRowsPerPass) transpose_kernel(const T *__restrict__ src, int64_t rows,
+                                                                            int64_t cols, T *__restrict__ dst)
+{
+    __shared__ T tile[kTile][kTile + 1];
+    const int64_t tiles_c = (cols + kTile - 1) / kTile;
+    const int64_t tiles = ((rows + kTile - 1) / kTile) * tiles_c;
+    const int tx = threadIdx.x, ty = threadIdx.y;
+    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+        const int64_t r0 = (t / tiles_c) * kTile, c0 = (t % tiles_c) * kTile;
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < kTile; k += kTileRowsPerPass) {
+            const int64_t r = r0 + ty + k, c = c0 + tx;
+            if (r < rows && c < cols)
+                tile[ty + k][tx] = src[r * cols + c];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < kTile; k += kTileRowsPerPass) {
+            const int64_t c = c0 + ty + k, r = r0 + tx;
+            if (r < rows && c < cols)
+                dst[c * rows + r] = tile[tx][ty + k];
+        }
+    }
+}
+
+// qzeros = 0x77777777 (zero point 8, stored minus one) and g_idx[i] = i / 128.
+__global__ void fill_kernel(int32_t *__restrict__ qzeros, int64_t nz, int32_t *__restrict__ g_idx, int64_t K)
+{
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nz + K; i += stride) {
+        if (i < nz)
+            qzeros[i] = 0x77777777;
+        else
+            g_idx[i - nz] = static_cast<int32_t>((i - nz) / 128);
+    }
+}
+
+// Dequantisation, one 32 (words along k) x 32 (outputs) tile per CTA
+// iteration: the tile's qweight words are read coalesced along r, then each
+// lane writes the 8 values of one word, so a warp stores 256 consecutive
+// values of one output row.  Group indices outside [0, K/128) are clamped.
+template <bool kHalf>
+__global__ void __launch_bounds__(kTile * kTileRowsPerPass) dequant_kernel(const uint32_t *__restrict__ qweight,
+                                                                          const uint32_t *__restrict__ qzeros,
+                                                                          const uint16_t *__restrict__ scales,
+                                                                          const int32_t *__restrict__ g_idx,
+                                                                          int64_t R, int64_t K, void *__restrict__ out)
+{
+    __shared__ uint32_t tile[kTile][kTile + 1];
+    const int64_t K8 = K / 8, ngroups = K / 128;
+    const int64_t tiles_r = (R + kTile - 1) / kTile;
+    const int64_t tiles = ((K8 + kTile - 1) / kTile) * tiles_r;
+    const int tx = threadIdx.x, ty = threadIdx.y;
+    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+        const int64_t k0 = (t / tiles_r) * kTile, r0 = (t % tiles_r) * kTile;
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < kTile; k += kTileRowsPerPass) {
+            const int64_t kk = k0 + ty + k, r = r0 + tx;
+            if (kk < K8 && r < R)
+                tile[ty + k][tx] = qweight[kk * R + r];
+        }
+        __syncthreads();
+        const int64_t kk = k0 + tx;
+        if (kk >= K8)
+            continue;
+#pragma unroll
+        for (int k = 0; k < kTile; k += kTileRowsPerPass) {
+            const int64_t r = r0 + ty + k;
+            if (r >= R)
+                continue;
+            const uint32_t word = tile[tx][ty + k];
+            float v[8];
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                int64_t g = g_idx[8 * kk + j];
+                g = g < 0 ? 0 : (g >= ngroups ? ngroups - 1 : g);
+                const float s = __half2float(__ushort_as_half(scales[g * R + r]));
+                const int z = static_cast<int>((qzeros[g * (R / 8) + r / 8] >> (4 * (r % 8))) & 0xFu);
+                const int u = static_cast<int>((word >> (4 * j)) & 0xFu);
+                v[j] = s * static_cast<float>(u - (z + 1));  // exact: 11-bit scale times |n| <= 16
+            }
+            if (kHalf) {
+                uint32_t h[4];
+#pragma unroll
+                for (int j = 0; j < 4; j++)
+                    h[j] = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(v[2 * j]))) |
+                           (static_cast<uint32_t>(__half_as_ushort(__float2half_rn(v[2 * j + 1]))) << 16);
+                *reinterpret_cast<uint4 *>(static_cast<__half *>(out) + r * K + 8 * kk) =
+                    make_uint4(h[0], h[1], h[2], h[3]);
+            } else {
+                float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(out) + r * K + 8 * kk);
+                o[0] = make_float4(v[0], v[1], v[2], v[3]);
+                o[1] = make_float4(v[4], v[5], v[6], v[7]);
+            }
+        }
+    }
+}
+
+unsigned tile_grid(int64_t tiles)
+{
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t cap = static_cast<int64_t>(sms > 0 ? sms : 148) * 16;
+    return static_cast<unsigned>(tiles < cap ? tiles : cap);
+}
+
+bool aligned(const void *p, size_t a)
+{
+    return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+cq_status check_shape(int64_t R, int64_t K)
+{
+    if (R < 0 || K < 0 || K % 128 != 0 || R % 8 != 0)
+        return CQ_ERR_INVALID_ARG;
+    if (R >= (static_cast<int64_t>(1) << 31) || K >= (static_cast<int64_t>(1) << 31))
+        return CQ_ERR_UNSUPPORTED;
+    return CQ_OK;
+}
+
+}  // namespace
+}  // namespace cq
+
+using namespace cq;
+
+extern "C" {
+
+cq_status cq_gptq_export(const uint16_t *scales, const uint32_t *codes, int64_t R, int64_t K, int32_t *qweight,
+                         int32_t *qzeros, uint16_t *gptq_scales, int32_t *g_idx, void *stream)
+{
+    const cq_status st = check_shape(R, K);
+    if (st != CQ_OK)
+        return st;
+    if (R == 0 || K == 0)
+        return CQ_OK;
+    if (!scales || !codes || !qweight || !qzeros || !gptq_scales || !g_idx || !aligned(scales, 2) ||
+        !aligned(codes, 4) || !aligned(qweight, 4) || !aligned(qzeros, 4) || !aligned(gptq_scales, 2) ||
+        !aligned(g_idx, 4))
+        return CQ_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const dim3 block(kTile, kTileRowsPerPass);
+    const int64_t K8 = K / 8, ng = K / 128;
+    transpose_kernel<uint32_t><<<tile_grid(((R + 31) / 32) * ((K8 + 31) / 32)), block, 0, s>>>(
+        codes, R, K8, reinterpret_cast<uint32_t *>(qweight));
+    if (cudaGetLastError() != cudaSuccess)
+        return CQ_ERR_CUDA;
+    transpose_kernel<uint16_t><<<tile_grid(((R + 31) / 32) * ((ng + 31) / 32)), block, 0, s>>>(scales, R, ng,
+                                                                                               gptq_scales);
+    if (cudaGetLastError() != cudaSuccess)
+        return CQ_ERR_CUDA;
+    const int64_t nz = ng * (R / 8);
+    fill_kernel<<<tile_grid((nz + K + 255) / 256), 256, 0, s>>>(qzeros, nz, g_idx, K);
+    return cudaGetLastError() == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
+}
+
+cq_status cq_gptq_dequantize(const int32_t *qweight, const int32_t *qzeros, const uint16_t *gptq_scales,
+                             const int32_t *g_idx, int64_t R, int64_t K, int out_fp16, void *out, void *stream)
+{
+    const cq_status st = check_shape(R, K);
+    if (st != CQ_OK)
+        return st;
+    if (out_fp16 != 0 && out_fp16 != 1)
+        return CQ_ERR_INVALID_ARG;
+    if (R == 0 || K == 0)
+        return CQ_OK;
+    if (!qweight || !qzeros || !gptq_scales || !g_idx || !out || !aligned(qweight, 4) || !aligned(qzeros, 4) ||
+        !aligned(gptq_scales, 2) || !aligned(g_idx, 4) || !aligned(out, 16))
+        return CQ_ERR_INVALID_ARG;
+    const dim3 block(kTile, kTileRowsPerPass);
+    const unsigned grid = tile_grid(((R + 31) / 32) * ((K / 8 + 31) / 32));
+    const uint32_t *qw = reinterpret_cast<const uint32_t *>(qweight);
+    const uint32_t *qz = reinterpret_cast<const uint32_t *>(qzeros);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (out_fp16)
+        dequant_kernel<true><<<grid, block, 0, s>>>(qw, qz, gptq_scales, g_idx, R, K, out);
+    else
+        dequant_kernel<false><<<grid, block, 0, s>>>(qw, qz, gptq_scales, g_idx, R, K, out);
+    return cudaGetLastError() == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
+}
+
+}  // extern "C"

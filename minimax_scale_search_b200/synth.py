@@ -53,6 +53,8 @@ _KIND_DIAG = 0
 _KIND_ROWS = 1
 _KIND_CLASS = 2
 _KIND_PROXY = 3
+_KIND_CODES = 4
+_KIND_GPTQ = 5
 
 
 @dataclass(frozen=True)
@@ -268,3 +270,26 @@ def make_proxy_inputs(groups: int = PROXY_GROUPS, modules: int = PROXY_MODULES, 
         for k, c in enumerate(blocks):
             D[:, a + k, :] = d[:, c * GROUP:(c + 1) * GROUP]
     return W, D, offsets
+
+
+def make_codes(G: int, seed: int = 1007):
+    """Random selection outputs for format tests: (positive finite binary16 scale
+    bits uint16 [G], code words uint32 [G, 16]); every nibble is a valid code."""
+    rng = _rng(seed, _KIND_CODES, 0)
+    scales = rng.integers(1, 0x7C00, G, dtype=np.int64).astype(np.uint16)
+    codes = rng.integers(0, 1 << 32, (G, 16), dtype=np.uint64).astype(np.uint32)
+    return scales, codes
+
+
+def make_gptq_tensors(R: int, K: int, seed: int = 1008, act_order: bool = False):
+    """Random GPTQ v1 tensors of an [R, K] layer (qweight int32 [K/8, R], qzeros
+    int32 [K/128, R/8] with arbitrary zero nibbles, scales binary16 bits uint16
+    [K/128, R], g_idx int32 [K]: i // 128, or a random permutation of it)."""
+    rng = _rng(seed, _KIND_GPTQ, 0)
+    qweight = rng.integers(0, 1 << 32, (K // 8, R), dtype=np.uint64).astype(np.uint32).view(np.int32)
+    qzeros = rng.integers(0, 1 << 32, (K // GROUP, R // 8), dtype=np.uint64).astype(np.uint32).view(np.int32)
+    scales = rng.integers(1, 0x7C00, (K // GROUP, R), dtype=np.int64).astype(np.uint16)
+    g_idx = (np.arange(K) // GROUP).astype(np.int32)
+    if act_order:
+        g_idx = rng.permutation(g_idx).astype(np.int32)
+    return qweight, qzeros, scales, g_idx

@@ -139,6 +139,23 @@ def test_policy_entry_points_validate(cq):
     assert prox(nmod=0, X=0, off=0) == cq.CQ_OK
 
 
+def test_gptq_entry_points_validate(cq):
+    vp, L, f = ctypes.c_void_p, cq.lib, ctypes.c_void_p(FAKE)
+    exp = lambda R=8, K=128, S=FAKE, C=FAKE: L.cq_gptq_export(vp(S), vp(C), R, K, f, f, f, f, vp(None))  # noqa: E731
+    assert exp(R=4) == cq.CQ_ERR_INVALID_ARG      # R % 8
+    assert exp(K=100) == cq.CQ_ERR_INVALID_ARG    # K % 128
+    assert exp(R=-8) == cq.CQ_ERR_INVALID_ARG
+    assert exp(R=1 << 31) == cq.CQ_ERR_UNSUPPORTED
+    assert exp(S=0) == cq.CQ_ERR_INVALID_ARG
+    assert exp(C=FAKE + 2) == cq.CQ_ERR_INVALID_ARG
+    assert exp(R=0, S=0, C=0) == cq.CQ_OK
+    deq = lambda R=8, K=128, half=0, out=FAKE: L.cq_gptq_dequantize(f, f, f, f, R, K, half, vp(out), vp(None))  # noqa: E731
+    assert deq(half=2) == cq.CQ_ERR_INVALID_ARG
+    assert deq(out=FAKE + 8) == cq.CQ_ERR_INVALID_ARG  # out must be 16-byte aligned
+    assert deq(K=64) == cq.CQ_ERR_INVALID_ARG
+    assert deq(R=0, out=0) == cq.CQ_OK
+
+
 def test_no_cpu_fallback_in_binding():
     """The binding refuses to run without its CUDA library."""
     src = open(os.path.join(ROOT, "minimax_scale_search_b200", "cq.py")).read()

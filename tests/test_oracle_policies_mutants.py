@@ -1,14 +1,13 @@
 """The policy pins are sensitive: plant one plausible mistake at a time in a
 copy of oracle/policies.py (on the CPU), load the copy, and check that at
 least one pin in test_oracle_policies.py fails for every mutant."""
-import importlib.util
 import os
-import sys
 
 import pytest
 
 import oracle
 import test_oracle_policies as pins
+from mutate import apply, first_failure, load_mutant
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "policies.py")
 
@@ -29,38 +28,13 @@ MUTANTS = {
 }
 
 
-def _load_copy(text, tmp_path, tag):
-    path = tmp_path / f"policies_{tag}.py"
-    path.write_text(text)
-    name = f"oracle._policies_mutant_{tag}"
-    spec = importlib.util.spec_from_file_location(name, path)
-    mod = importlib.util.module_from_spec(spec)
-    sys.modules[name] = mod
-    try:
-        spec.loader.exec_module(mod)
-    finally:
-        sys.modules.pop(name, None)
-    return mod
-
-
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_policy_pins_catch_mutant(name, tmp_path):
-    src = open(SRC).read()
-    for old, new in MUTANTS[name]:
-        assert src.count(old) == 1, f"mutation anchor for {name} not unique: {old!r}"
-        src = src.replace(old, new)
-    mod = _load_copy(src, tmp_path, name)
-    caught = None
-    for check in pins.CHECKS:
-        try:
-            check(mod)
-        except Exception as exc:  # a failed assertion or an error both count as caught
-            caught = (check.__name__, exc)
-            break
-    assert caught is not None, f"no pin catches mutant {name}"
+    mod = load_mutant(apply(open(SRC).read(), MUTANTS[name], name), tmp_path, name)
+    assert first_failure(mod, pins.CHECKS) is not None, f"no pin catches mutant {name}"
 
 
 def test_unmutated_copy_passes(tmp_path):
-    mod = _load_copy(open(SRC).read(), tmp_path, "clean")
+    mod = load_mutant(open(SRC).read(), tmp_path, "clean")
     for check in pins.CHECKS:
         check(mod)
