@@ -193,7 +193,7 @@ cq_status cq_gptq_export(const uint16_t *scales, const uint32_t *codes, int64_t 
                          void *stream);
 
 /* Dequantisation by the v1 rule w[r][i] = scales[g][r] * (u - (z + 1)), g = g_idx[i]
- * (clamped to [0, K/128)), into out [R][K] (16-byte aligned): fp32 when
+ * (clamped to [0, K/128)), into out [R][K] (out and g_idx 16-byte aligned): fp32 when
  * out_fp16 == 0 (exact), binary16 rounded to nearest even when out_fp16 == 1.
  * Reads only the four tensors: an unpacker independent of the export. */
 cq_status cq_gptq_dequantize(const int32_t *qweight, const int32_t *qzeros, const uint16_t *gptq_scales,

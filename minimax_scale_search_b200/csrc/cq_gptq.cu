@@ -71,6 +71,11 @@ __global__ void fill_kernel(int32_t *__restrict__ qzeros, int64_t nz, int32_t *_
     }
 }
 
+__device__ __forceinline__ int64_t clamp_group(int g, int64_t ngroups)
+{
+    return g < 0 ? 0 : (g >= ngroups ? ngroups - 1 : g);
+}
+
 // Dequantisation, one 32 (words along k) x 32 (outputs) tile per CTA
 // iteration: the tile's qweight words are read coalesced along r, then each
 // lane writes the 8 values of one word, so a warp stores 256 consecutive
@@ -100,6 +105,14 @@ __global__ void __launch_bounds__(kTile * kTileRowsPerPass) dequant_kernel(const
         const int64_t kk = k0 + tx;
         if (kk >= K8)
             continue;
+        const int4 ga = reinterpret_cast<const int4 *>(g_idx)[2 * kk];
+        const int4 gb = reinterpret_cast<const int4 *>(g_idx)[2 * kk + 1];
+        const int gi[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+        bool uniform = true;
+#pragma unroll
+        for (int j = 1; j < 8; j++)
+            uniform = uniform && gi[j] == gi[0];
+        const int64_t g0 = clamp_group(gi[0], ngroups);
 #pragma unroll
         for (int k = 0; k < kTile; k += kTileRowsPerPass) {
             const int64_t r = r0 + ty + k;
@@ -107,14 +120,21 @@ __global__ void __launch_bounds__(kTile * kTileRowsPerPass) dequant_kernel(const
                 continue;
             const uint32_t word = tile[tx][ty + k];
             float v[8];
+            if (uniform) {  // one group for the word's 8 inputs (always so with act-order off)
+                const float s = __half2float(__ushort_as_half(scales[g0 * R + r]));
+                const int z1 = static_cast<int>((qzeros[g0 * (R / 8) + r / 8] >> (4 * (r % 8))) & 0xFu) + 1;
 #pragma unroll
-            for (int j = 0; j < 8; j++) {
-                int64_t g = g_idx[8 * kk + j];
-                g = g < 0 ? 0 : (g >= ngroups ? ngroups - 1 : g);
-                const float s = __half2float(__ushort_as_half(scales[g * R + r]));
-                const int z = static_cast<int>((qzeros[g * (R / 8) + r / 8] >> (4 * (r % 8))) & 0xFu);
-                const int u = static_cast<int>((word >> (4 * j)) & 0xFu);
-                v[j] = s * static_cast<float>(u - (z + 1));  // exact: 11-bit scale times |n| <= 16
+                for (int j = 0; j < 8; j++)
+                    v[j] = s * static_cast<float>(static_cast<int>((word >> (4 * j)) & 0xFu) - z1);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; j++) {
+                    const int64_t g = clamp_group(gi[j], ngroups);
+                    const float s = __half2float(__ushort_as_half(scales[g * R + r]));
+                    const int z = static_cast<int>((qzeros[g * (R / 8) + r / 8] >> (4 * (r % 8))) & 0xFu);
+                    const int u = static_cast<int>((word >> (4 * j)) & 0xFu);
+                    v[j] = s * static_cast<float>(u - (z + 1));  // exact: 11-bit scale times |n| <= 16
+                }
             }
             if (kHalf) {
                 uint32_t h[4];
@@ -202,7 +222,7 @@ cq_status cq_gptq_dequantize(const int32_t *qweight, const int32_t *qzeros, cons
     if (R == 0 || K == 0)
         return CQ_OK;
     if (!qweight || !qzeros || !gptq_scales || !g_idx || !out || !aligned(qweight, 4) || !aligned(qzeros, 4) ||
-        !aligned(gptq_scales, 2) || !aligned(g_idx, 4) || !aligned(out, 16))
+        !aligned(gptq_scales, 2) || !aligned(g_idx, 16) || !aligned(out, 16))
         return CQ_ERR_INVALID_ARG;
     const dim3 block(kTile, kTileRowsPerPass);
     const unsigned grid = tile_grid(((R + 31) / 32) * ((K / 8 + 31) / 32));

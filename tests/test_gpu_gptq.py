@@ -68,7 +68,10 @@ def test_dequantize_bit_exact(R, K, act_order):
     got32 = cq.gptq_dequantize(t).cpu().numpy()
     assert np.array_equal(got32.astype(np.float64), exp)
     got16 = cq.gptq_dequantize(t, half=True).cpu().numpy()
-    assert np.array_equal(got16.view(np.uint16), exp.astype(np.float16).view(np.uint16))
+    with np.errstate(over="ignore"):  # products above 65504 round to inf on both sides
+        exp16 = exp.astype(np.float16)
+    assert np.isinf(exp16).any() or R < 1024
+    assert np.array_equal(got16.view(np.uint16), exp16.view(np.uint16))
 
 
 def test_round_trip_to_s_times_q():
