@@ -387,6 +387,39 @@ def bench_gptq(args, wl, dev):
         print(json.dumps(ln), flush=True)
 
 
+DIAG_ENVS, DIAG_TOKENS = 4, 16384
+
+
+def bench_diag(args, wl, dev):
+    """Diagonal estimation from bf16 calibration inputs: 4 environments of
+    16,384 tokens over the sweep's 16,384 input columns (2.1 GB, drawn on the
+    device from a seeded generator)."""
+    import torch
+    from minimax_scale_search_b200 import cq
+    stream = torch.cuda.current_stream()
+    K, E, N = wl.cols, DIAG_ENVS, DIAG_TOKENS
+    g = torch.Generator(device=dev)
+    g.manual_seed(1010)
+    col = torch.exp(torch.randn(K, generator=g, device=dev))
+    X = (torch.randn((E * N, K), generator=g, device=dev) * col).to(torch.bfloat16)
+    off = np.arange(E + 1, dtype=np.int64) * N
+    means = torch.empty((E, K), dtype=torch.float64, device=dev)
+    D = torch.empty((E, K), dtype=torch.float32, device=dev)
+    hbm, hsrc = hbm_peak()
+    ms = time_calls(lambda: cq.estimate_diagonals(X, off, means=means, out=D), args.steps, args.warmup, stream)
+    byt = E * N * K * 2 + E * K * (8 + 8 + 4)
+    line = {"metric": "diagonal estimation tokens/sec", "op": "diag", "value": E * N / ms * 1e3, "unit": "tokens/s",
+            "ms_per_step": ms, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+            "dtype": "f64", "data": "synthetic", "gpu_launches": 2 * args.steps,
+            "config": {"workload": f"diag-{E}x{N}x{K}-bf16", "environments": E, "tokens_per_env": N, "K": K,
+                       "l2": "inputs (2.1 GB) larger than the 126 MB L2; no flush"},
+            "roofline": {"bound": "hbm", "achieved": byt / ms / 1e6, "peak": hbm, "unit": "GB/s",
+                         "frac": byt / ms / 1e6 / hbm, "traffic": None,
+                         "kernel": "column_squares_kernel<bf16> + normalise_kernel",
+                         "bytes_per_token": K * 2, "peak_note": hsrc}}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -395,7 +428,7 @@ def main():
     ap.add_argument("--impl", default="cq", choices=["cq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--op", default="select", choices=["select", "policies", "gptq"],
+    ap.add_argument("--op", default="select", choices=["select", "policies", "gptq", "diag"],
                     help="select: the headline line; policies / gptq: one line per kernel of those rows")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -422,10 +455,10 @@ def main():
     dev = torch.device("cuda", local)
 
     from minimax_scale_search_b200 import cq
-    if args.op == "gptq":
+    if args.op in ("gptq", "diag"):
         if world > 1:
-            ap.error("--op gptq runs on one GPU")
-        bench_gptq(args, wl, dev)
+            ap.error(f"--op {args.op} runs on one GPU")
+        (bench_gptq if args.op == "gptq" else bench_diag)(args, wl, dev)
         return
     W = synth.make_weights(WORKLOAD, matrix=rank_matrix(rank))
     D = synth.make_diagonals(WORKLOAD, matrix=rank_matrix(rank))

@@ -200,6 +200,24 @@ cq_status cq_gptq_dequantize(const int32_t *qweight, const int32_t *qzeros, cons
                              const int32_t *g_idx, int64_t R, int64_t K, int out_fp16, void *out,
                              void *stream);
 
+/* ---- sensitivity diagonals ----------------------------------------------------
+ * The project page ("What CliffQuant changes"; "The negative result that
+ * changed the method") takes separately normalised per-environment diagonals
+ * estimated as empirical activation-weighted sensitivity.  From calibration
+ * inputs X [rows][K] (row-major, 16-byte aligned, K % 8 == 0), environment e
+ * owning rows row_offsets[e] .. row_offsets[e+1]-1 (a HOST array of E+1
+ * ascending offsets, 1 <= E <= CQ_MAX_E):
+ *   means[e][k] = (sum over its rows of x^2) / N_e   fp64 [E][K], 8-byte aligned
+ *   D[e][k]     = fp32(means[e][k] / mean_j means[e][j])   fp32 [E][K]
+ * Squares are exact and summed in fp64 in a fixed order (deterministic).  An
+ * environment with no rows, or only zero activations, gives NaN.  D is the
+ * per-column diagonal layout cq_select_scales takes. */
+#define CQ_DTYPE_BF16 0
+#define CQ_DTYPE_FP16 1
+#define CQ_DTYPE_FP32 2
+cq_status cq_estimate_diagonals(const void *X, int dtype, int64_t K, const int64_t *row_offsets, int E,
+                                double *means, float *D, void *stream);
+
 /* Largest G that cq_select_scales_noalloc accepts. */
 #define CQ_NOALLOC_MAX_GROUPS (1 << 20)
 

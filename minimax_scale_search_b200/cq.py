@@ -28,7 +28,7 @@ MAX_E = 8
 # Symbols the C header declares, in declaration order.
 EXPORTS = ("cq_workspace_bytes", "cq_select_scales", "cq_select_scales_ex", "cq_select_scales_host",
            "cq_absmax_scales", "cq_pool_diagonals", "cq_group_objective", "cq_reconstruction_proxy",
-           "cq_gptq_export", "cq_gptq_dequantize",
+           "cq_gptq_export", "cq_gptq_dequantize", "cq_estimate_diagonals",
            "cq_select_scales_noalloc", "cq_read_counters", "cq_status_string", "cq_version")
 
 
@@ -70,6 +70,8 @@ def _load():
     L.cq_gptq_export.argtypes = [vp, vp, i64, i64, vp, vp, vp, vp, vp]
     L.cq_gptq_dequantize.restype = i32
     L.cq_gptq_dequantize.argtypes = [vp, vp, vp, vp, i64, i64, i32, vp, vp]
+    L.cq_estimate_diagonals.restype = i32
+    L.cq_estimate_diagonals.argtypes = [vp, i32, i64, vp, i32, vp, vp, vp]
     L.cq_select_scales_noalloc.restype = i32
     L.cq_select_scales_noalloc.argtypes = [vp, i64, vp, i32, i64, vp, vp, vp]
     L.cq_read_counters.restype = i32
@@ -400,6 +402,34 @@ def gptq_dequantize(t: GPTQTensors, *, half: bool = False, stream=None):
     _check(lib.cq_gptq_dequantize(_ptr(t.qweight), _ptr(t.qzeros), _ptr(t.scales), _ptr(t.g_idx), R, K,
                                   int(bool(half)), _ptr(out), _stream_handle(stream)), "cq_gptq_dequantize")
     return out
+
+
+DTYPE_BF16, DTYPE_FP16, DTYPE_FP32 = 0, 1, 2
+
+
+def estimate_diagonals(X, row_offsets, *, dtype=None, stream=None, means=None, out=None):
+    """Per-environment diagonals from calibration inputs X [rows, K] (CUDA
+    bfloat16, float16 or float32; environment e owns rows row_offsets[e] ..
+    row_offsets[e+1]-1).  Returns (means float64 [E, K], D float32 [E, K]);
+    D is the per-column diagonal input of select_scales."""
+    import torch
+    if not X.is_cuda or X.dim() != 2 or not X.is_contiguous():
+        raise ValueError("X must be a contiguous 2-D CUDA tensor")
+    if dtype is None:
+        dtype = {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_FP16, torch.float32: DTYPE_FP32}.get(X.dtype)
+        if dtype is None:
+            raise ValueError("X must be bfloat16, float16 or float32 (or pass dtype for 16-bit patterns)")
+    off = np.ascontiguousarray(np.asarray(row_offsets, dtype=np.int64).ravel())
+    E, K = off.size - 1, X.shape[1]
+    if E < 1 or off[-1] > X.shape[0]:
+        raise ValueError("row_offsets must hold E + 1 offsets within X's rows")
+    if means is None:
+        means = torch.empty((E, K), dtype=torch.float64, device=X.device)
+    if out is None:
+        out = torch.empty((E, K), dtype=torch.float32, device=X.device)
+    _check(lib.cq_estimate_diagonals(_ptr(X), int(dtype), K, _ptr(off), E, _ptr(means), _ptr(out),
+                                     _stream_handle(stream)), "cq_estimate_diagonals")
+    return means, out
 
 
 def read_counters(workspace, stream=None) -> dict:

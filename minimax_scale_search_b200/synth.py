@@ -55,6 +55,7 @@ _KIND_CLASS = 2
 _KIND_PROXY = 3
 _KIND_CODES = 4
 _KIND_GPTQ = 5
+_KIND_ACT = 6
 
 
 @dataclass(frozen=True)
@@ -293,3 +294,35 @@ def make_gptq_tensors(R: int, K: int, seed: int = 1008, act_order: bool = False)
     if act_order:
         g_idx = rng.permutation(g_idx).astype(np.int32)
     return qweight, qzeros, scales, g_idx
+
+
+def to_bf16_bits(x) -> np.ndarray:
+    """float32 -> bfloat16 bit patterns (uint16), round to nearest even (finite inputs)."""
+    b = np.asarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    return ((b + 0x7FFF + ((b >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def make_activations(tokens, K: int, dtype: int = 0, seed: int = 1009):
+    """Calibration inputs for diagonal estimation: (X [sum(tokens), K] as bf16 /
+    fp16 bit patterns (uint16, dtype 0 / 1) or float32 (dtype 2), row offsets
+    int64 [E + 1]).  Environment e draws N(0, 1) scaled per column by
+    lognormal(0, 1) shared across environments times an environment factor
+    lognormal(0, 0.5), with 0.5% of columns (outlier channels) x16."""
+    tokens = [int(n) for n in np.atleast_1d(tokens)]
+    shared = _rng(seed, _KIND_ACT, 0).lognormal(0.0, 1.0, K)
+    outl = _rng(seed, _KIND_ACT, 1).random(K) < 0.005
+    shared = np.where(outl, shared * 16.0, shared)
+    parts = []
+    for e, n in enumerate(tokens):
+        rng = _rng(seed, _KIND_ACT, 2 + e)
+        scale = shared * rng.lognormal(0.0, 0.5, K)
+        x = (rng.standard_normal((n, K)) * scale).astype(np.float32)
+        if dtype == 0:
+            parts.append(to_bf16_bits(x))
+        elif dtype == 1:
+            parts.append(x.astype(np.float16).view(np.uint16))
+        else:
+            parts.append(x)
+    offsets = np.concatenate([[0], np.cumsum(tokens)]).astype(np.int64)
+    empty = np.zeros((0, K), dtype=np.float32 if dtype == 2 else np.uint16)
+    return (np.concatenate(parts, axis=0) if parts else empty), offsets

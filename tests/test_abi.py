@@ -1,6 +1,8 @@
 """C-ABI checks that need no GPU: the library loads, exports every function
 include/cq.h declares, and rejects bad arguments before enqueuing anything."""
 import ctypes
+
+import numpy as np
 import os
 import re
 import subprocess
@@ -154,6 +156,24 @@ def test_gptq_entry_points_validate(cq):
     assert deq(out=FAKE + 8) == cq.CQ_ERR_INVALID_ARG  # out must be 16-byte aligned
     assert deq(K=64) == cq.CQ_ERR_INVALID_ARG
     assert deq(R=0, out=0) == cq.CQ_OK
+
+
+def test_diagonal_entry_point_validates(cq):
+    vp, L = ctypes.c_void_p, cq.lib
+    off = np.array([0, 10, 20], dtype=np.int64)
+    bad = np.array([0, 20, 10], dtype=np.int64)
+    f = vp(FAKE)
+    est = lambda dt=0, K=256, o=off, E=2, X=FAKE, M=FAKE: L.cq_estimate_diagonals(  # noqa: E731
+        vp(X), dt, K, vp(o.ctypes.data), E, vp(M), f, vp(None))
+    assert est(dt=3) == cq.CQ_ERR_INVALID_ARG
+    assert est(E=0) == cq.CQ_ERR_INVALID_ARG
+    assert est(E=9) == cq.CQ_ERR_UNSUPPORTED
+    assert est(K=12) == cq.CQ_ERR_INVALID_ARG            # K % 8
+    assert est(o=bad) == cq.CQ_ERR_INVALID_ARG           # offsets must ascend
+    assert est(X=FAKE + 8) == cq.CQ_ERR_INVALID_ARG      # X 16-byte aligned
+    assert est(M=FAKE + 4) == cq.CQ_ERR_INVALID_ARG
+    assert est(K=0) == cq.CQ_OK
+    assert L.cq_estimate_diagonals(f, 0, 256, vp(None), 2, f, f, vp(None)) == cq.CQ_ERR_INVALID_ARG
 
 
 def test_no_cpu_fallback_in_binding():
