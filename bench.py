@@ -43,16 +43,19 @@ def flop_run(E: int) -> int:
     return 4 * E + E + 12 * E * (E - 1) // 2 + (E * E + 4) * (5 * E - 1)
 
 
-def counted_flops(Wg: np.ndarray, E: int):
+def counted_flops(Wg: np.ndarray, E: int, qmin: int = -8, qmax: int = 7):
     """(fp32 flops, fp64 flops) of the method's candidate work for these groups:
-    per non-trivial group (T_g + 1) runs with T_g = 7 #(w>0) + 8 #(w<0), plus
-    fp64 rescoring of two finalists (2 * 128 * E * 5)."""
+    per non-trivial group (T_g + 1) runs with T_g = qmax #(w>0) + |qmin| #(w<0)
+    code transitions (7 and 8 for W4), plus fp64 rescoring of two finalists
+    (2 * n * E * 5)."""
+    n = Wg.shape[1]
     nz = (Wg & 0x7FFF) != 0
     neg = nz & ((Wg & 0x8000) != 0)
-    T = 7 * nz.sum(axis=1, dtype=np.int64) + neg.sum(axis=1, dtype=np.int64)
+    pos = nz & ~neg
+    T = qmax * pos.sum(axis=1, dtype=np.int64) + (-qmin) * neg.sum(axis=1, dtype=np.int64)
     live = nz.any(axis=1)
     f32 = int(((T + 1) * live).sum()) * flop_run(E)
-    f64 = int(live.sum()) * 2 * 128 * E * 5
+    f64 = int(live.sum()) * 2 * n * E * 5
     return f32, f64
 
 
@@ -420,6 +423,38 @@ def bench_diag(args, wl, dev):
     print(json.dumps(line), flush=True)
 
 
+SPEC_ROWS = 4096
+SPEC_CASES = ((-8, 7, 128), (-4, 3, 128), (-8, 7, 64), (-16, 15, 128))
+
+
+def bench_spec(args, wl, dev):
+    """The general-spec path on the first 4,096 rows of the sweep (524,288
+    groups of 128; 1,048,576 of 64), one JSON line per spec."""
+    import torch
+    from minimax_scale_search_b200 import cq, synth
+    stream = torch.cuda.current_stream()
+    W = synth.make_weights(WORKLOAD, 0, SPEC_ROWS)
+    D = synth.make_diagonals(WORKLOAD)
+    Wd = torch.from_numpy(W.view(np.int16)).to(dev)
+    Dd = torch.from_numpy(D).to(dev)
+    p32, p64, _, psrc = peaks()
+    for qmin, qmax, n in SPEC_CASES:
+        G = W.size // n
+        ms = time_calls(lambda: cq.select_scales_spec(Wd, Dd, wl.cols, qmin=qmin, qmax=qmax, group_size=n),
+                        args.steps, args.warmup, stream)
+        f32, f64 = counted_flops(W.reshape(-1, n), wl.E, qmin, qmax)
+        ach = (f32 + f64 * p32 / p64) / (ms / 1e3) / 1e12
+        line = {"metric": "general-spec minimax scale selection groups/sec", "op": "spec", "value": G / ms * 1e3,
+                "unit": "groups/s", "ms_per_step": ms, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+                "higher_is_better": True, "dtype": "f64", "data": "synthetic", "gpu_launches": args.steps,
+                "config": {"workload": f"sweep-rows0-{SPEC_ROWS}-q[{qmin},{qmax}]-n{n}", "groups": G, "E": wl.E,
+                           "K": wl.cols, "qmin": qmin, "qmax": qmax, "group_size": n},
+                "roofline": {"bound": "alu", "achieved": ach, "peak": p32, "unit": "TFLOP/s", "frac": ach / p32,
+                             "traffic": None, "kernel": "spec_kernel", "fp32_flops": f32, "fp64_flops": f64,
+                             "peak_note": psrc}}
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -428,7 +463,7 @@ def main():
     ap.add_argument("--impl", default="cq", choices=["cq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--op", default="select", choices=["select", "policies", "gptq", "diag"],
+    ap.add_argument("--op", default="select", choices=["select", "policies", "gptq", "diag", "spec"],
                     help="select: the headline line; policies / gptq: one line per kernel of those rows")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -455,10 +490,10 @@ def main():
     dev = torch.device("cuda", local)
 
     from minimax_scale_search_b200 import cq
-    if args.op in ("gptq", "diag"):
+    if args.op in ("gptq", "diag", "spec"):
         if world > 1:
             ap.error(f"--op {args.op} runs on one GPU")
-        (bench_gptq if args.op == "gptq" else bench_diag)(args, wl, dev)
+        {"gptq": bench_gptq, "diag": bench_diag, "spec": bench_spec}[args.op](args, wl, dev)
         return
     W = synth.make_weights(WORKLOAD, matrix=rank_matrix(rank))
     D = synth.make_diagonals(WORKLOAD, matrix=rank_matrix(rank))

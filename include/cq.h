@@ -218,6 +218,28 @@ cq_status cq_gptq_dequantize(const int32_t *qweight, const int32_t *qzeros, cons
 cq_status cq_estimate_diagonals(const void *X, int dtype, int64_t K, const int64_t *row_offsets, int E,
                                 double *means, float *D, void *stream);
 
+/* ---- general quantiser spec ---------------------------------------------------
+ * "Use the solver" on the project page passes QuantizerSpec(qmin, qmax); this
+ * entry point takes any qmin in [-128, -1], qmax in [1, 127] and group size n
+ * in [1, CQ_SPEC_MAX_GROUP], with the same objective, binary16 scale domain
+ * and tie rule as cq_select_scales.  W [G][n] binary16 bits; D per column
+ * [E][K] (K % n == 0, group g uses columns (g mod K/n)*n ..; G a whole number
+ * of rows) or per group [E][G][n] (K == 0).  Outputs: out_scales [G],
+ * out_codes int8 [G][n] (the codes q themselves), optional out_objective fp64
+ * [G] (8-byte aligned) and out_flags [G] (CQ_FLAG_TRIVIAL / CQ_FLAG_NONFINITE;
+ * such groups get scale 0x0001, zero codes and objective 0).  The kernel is a
+ * certified window plus an exact scan, slower than cq_select_scales, which
+ * serves (-8, 7, 128). */
+typedef struct cq_quantizer_spec {
+    int32_t qmin;
+    int32_t qmax;
+    int32_t group_size;
+} cq_quantizer_spec;
+#define CQ_SPEC_MAX_GROUP 1024
+cq_status cq_select_scales_spec(const uint16_t *W, int64_t G, const float *D, int E, int64_t K,
+                                const cq_quantizer_spec *spec, uint16_t *out_scales, int8_t *out_codes,
+                                double *out_objective, uint8_t *out_flags, void *stream);
+
 /* Largest G that cq_select_scales_noalloc accepts. */
 #define CQ_NOALLOC_MAX_GROUPS (1 << 20)
 

@@ -11,7 +11,8 @@ import sys
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
-SRCS = [os.path.join(PKG, "csrc", name) for name in ("cq_select.cu", "cq_policies.cu", "cq_gptq.cu", "cq_diag.cu")]
+SRCS = [os.path.join(PKG, "csrc", name) for name in ("cq_select.cu", "cq_policies.cu", "cq_gptq.cu", "cq_diag.cu",
+                                                           "cq_spec.cu")]
 DEPS = SRCS + [os.path.join(PKG, "csrc", "cq_device.cuh"), os.path.join(ROOT, "include", "cq.h")]
 LIB = os.path.join(PKG, "libcq.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -28,7 +28,7 @@ MAX_E = 8
 # Symbols the C header declares, in declaration order.
 EXPORTS = ("cq_workspace_bytes", "cq_select_scales", "cq_select_scales_ex", "cq_select_scales_host",
            "cq_absmax_scales", "cq_pool_diagonals", "cq_group_objective", "cq_reconstruction_proxy",
-           "cq_gptq_export", "cq_gptq_dequantize", "cq_estimate_diagonals",
+           "cq_gptq_export", "cq_gptq_dequantize", "cq_estimate_diagonals", "cq_select_scales_spec",
            "cq_select_scales_noalloc", "cq_read_counters", "cq_status_string", "cq_version")
 
 
@@ -36,6 +36,14 @@ class CQError(RuntimeError):
     def __init__(self, status: int, where: str = ""):
         self.status = status
         super().__init__(f"{where}: {status_string(status)}" if where else status_string(status))
+
+
+class QuantizerSpec(ctypes.Structure):
+    """Codes in [qmin, qmax], groups of group_size weights (the pages' QuantizerSpec)."""
+    _fields_ = [("qmin", ctypes.c_int32), ("qmax", ctypes.c_int32), ("group_size", ctypes.c_int32)]
+
+
+SPEC_MAX_GROUP = 1024
 
 
 class Opts(ctypes.Structure):
@@ -72,6 +80,8 @@ def _load():
     L.cq_gptq_dequantize.argtypes = [vp, vp, vp, vp, i64, i64, i32, vp, vp]
     L.cq_estimate_diagonals.restype = i32
     L.cq_estimate_diagonals.argtypes = [vp, i32, i64, vp, i32, vp, vp, vp]
+    L.cq_select_scales_spec.restype = i32
+    L.cq_select_scales_spec.argtypes = [vp, i64, vp, i32, i64, ctypes.POINTER(QuantizerSpec), vp, vp, vp, vp, vp]
     L.cq_select_scales_noalloc.restype = i32
     L.cq_select_scales_noalloc.argtypes = [vp, i64, vp, i32, i64, vp, vp, vp]
     L.cq_read_counters.restype = i32
@@ -402,6 +412,42 @@ def gptq_dequantize(t: GPTQTensors, *, half: bool = False, stream=None):
     _check(lib.cq_gptq_dequantize(_ptr(t.qweight), _ptr(t.qzeros), _ptr(t.scales), _ptr(t.g_idx), R, K,
                                   int(bool(half)), _ptr(out), _stream_handle(stream)), "cq_gptq_dequantize")
     return out
+
+
+def select_scales_spec(W, D, K: int | None = None, *, qmin: int = -8, qmax: int = 7, group_size: int = 128,
+                       stream=None, want_objective: bool = False, want_flags: bool = False) -> Result:
+    """Exact minimax scales for a general spec (codes in [qmin, qmax], groups of
+    group_size weights).  W: CUDA 16-bit binary16 patterns whose last dimension
+    is a multiple of group_size; D: float32 per column [E, K] or per group
+    [E, G, group_size].  Returns scales int16 [G] and codes int8 [G, group_size]
+    (the q values).  (-8, 7, 128) is served faster by select_scales."""
+    import torch
+    n = int(group_size)
+    if not (W.is_cuda and D.is_cuda and W.is_contiguous() and D.is_contiguous()):
+        raise ValueError("W and D must be contiguous CUDA tensors")
+    if W.element_size() != 2 or D.dtype != torch.float32:
+        raise ValueError("W must hold binary16 patterns and D float32")
+    if n < 1 or W.shape[-1] % n:
+        raise ValueError("the last dimension of W must be a multiple of group_size")
+    G = W.numel() // n
+    if D.dim() == 2:
+        E, Kd = D.shape
+        if K is not None and K != Kd:
+            raise ValueError("K does not match D")
+        K = Kd
+    elif D.dim() == 3 and D.shape[1:] == (G, n):
+        E, K = D.shape[0], 0
+    else:
+        raise ValueError("D must be [E, K] or [E, G, group_size]")
+    dev = W.device
+    scales = torch.empty(G, dtype=torch.int16, device=dev)
+    codes = torch.empty((G, n), dtype=torch.int8, device=dev)
+    obj = torch.empty(G, dtype=torch.float64, device=dev) if want_objective else None
+    flags = torch.empty(G, dtype=torch.uint8, device=dev) if want_flags else None
+    spec = QuantizerSpec(int(qmin), int(qmax), n)
+    _check(lib.cq_select_scales_spec(_ptr(W), G, _ptr(D), E, K, ctypes.byref(spec), _ptr(scales), _ptr(codes),
+                                     _ptr(obj), _ptr(flags), _stream_handle(stream)), "cq_select_scales_spec")
+    return Result(scales, codes, obj, flags)
 
 
 DTYPE_BF16, DTYPE_FP16, DTYPE_FP32 = 0, 1, 2

@@ -1,0 +1,377 @@
+// Exact minimax scale selection for a general quantiser spec: codes in
+// [qmin, qmax] (qmin <= -1 <= 1 <= qmax) and groups of n <= 1024 weights.
+//
+// CliffQuant project page, "What CliffQuant changes" (the objective, the
+// quantiser and the binary16 scale domain with the lower pattern winning a tie)
+// and "Use the solver" (QuantizerSpec(qmin, qmax)).  The warp-per-group kernel
+// in cq_select.cu is specialised to (-8, 7) and 128 weights; this path serves
+// every other spec with the same result definition.
+//
+// One CTA per group (grid-stride over groups):
+//  1. stage w (exact fp32 and fp64) and the group's diagonals (fp64);
+//  2. U = the smallest objective, computed exactly as the definition does,
+//     at the AbsMax-type scales fp16(max|w|/qmax), fp16(max|w|/|qmin|), their
+//     grid neighbours and the first scale at which every code is 0;
+//  3. a certified window [J0, J1]: below a scale, the clipped weights' error
+//     sum_e-max of sum d (|w| - c s)^2 only grows as s falls; above one, the
+//     error of the weights that round to 0, sum d w^2, only grows as s rises.
+//     Both are fp64 lower bounds of the exact objective, taken with a 2^-40
+//     margin that covers the rounding of either side (n <= 4096), so a scale
+//     they exclude has an objective above U and cannot be the minimum or tie it;
+//  4. every scale of the window, one thread per scale, evaluated in the
+//     definition's own order (i ascending, r = w - s q exact, r*r, d*rr and the
+//     running sum rounded separately, environments maxed in order), so each
+//     value equals the oracle's bit for bit; above the first all-zero scale j_z
+//     every scale has the same value, so only j_z is evaluated there;
+//  5. the (objective, pattern) minimum and its codes.
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cfloat>
+#include <cstdint>
+
+#include "cq.h"
+#include "cq_device.cuh"
+
+namespace cq {
+namespace {
+
+constexpr int kSpecThreads = 256;
+constexpr int kSpecWarps = kSpecThreads / 32;
+constexpr int kCandidates = 7;
+
+struct SpecParams {
+    const uint16_t *W;
+    int64_t G;
+    const float *D;
+    int E;
+    int64_t K;
+    int qmin, qmax, n;
+    uint16_t *out_scales;
+    int8_t *out_codes;
+    double *out_obj;
+    uint8_t *out_flags;
+};
+
+// min(round-half-even(aw / s), cap) for aw >= 0, exact (cap <= 128): an
+// estimate from 1/s, rounded by adding 1.5 * 2^23, corrected by the exact
+// thresholds s (m -+ 1/2) (an 11-bit scale times a factor of at most 9 bits).
+__device__ __forceinline__ int spec_code(float aw, float s, float inv, int cap)
+{
+    constexpr float kRound = 12582912.0f;
+    const float y = fminf(aw * inv, static_cast<float>(cap + 1)) + kRound;
+    const float m = y - kRound;
+    const int mi = __float_as_int(y) - 0x4B400000;
+    const float lo = s * (m - 0.5f), hi = s * (m + 0.5f);
+    const bool odd = mi & 1;
+    const int below = (aw < lo || (aw == lo && odd)) ? 1 : 0;
+    const int above = (aw > hi || (aw == hi && odd)) ? 1 : 0;
+    return min(mi - below + above, cap);
+}
+
+struct Smem {
+    float *wf;   // [n] exact weights
+    double *wd;  // [n]
+    double *dd;  // [E][n]
+};
+
+// Objective at grid index j, in the definition's order; one thread.
+__device__ double objective_at(const Smem &sm, int n, int E, int qmin, int qmax, uint32_t j)
+{
+    const float s = grid_value(j);
+    const float inv = 1.0f / s;
+    const double nsd = -static_cast<double>(s);
+    double acc[CQ_MAX_E];
+#pragma unroll
+    for (int e = 0; e < CQ_MAX_E; e++)
+        acc[e] = 0.0;
+    for (int i = 0; i < n; i++) {
+        const float w = sm.wf[i];
+        const bool neg = w < 0.0f;
+        const int c = spec_code(fabsf(w), s, inv, neg ? -qmin : qmax);
+        const double r = fma(nsd, static_cast<double>(neg ? -c : c), sm.wd[i]);
+        const double rr = __dmul_rn(r, r);
+#pragma unroll
+        for (int e = 0; e < CQ_MAX_E; e++)
+            if (e < E)
+                acc[e] = __dadd_rn(acc[e], __dmul_rn(sm.dd[e * n + i], rr));
+    }
+    double f = acc[0];
+#pragma unroll
+    for (int e = 1; e < CQ_MAX_E; e++)
+        if (e < E && acc[e] > f)
+            f = acc[e];
+    return f;
+}
+
+// Block-wide (min objective, lowest pattern); every thread gets the result.
+__device__ void block_best(double &f, uint32_t &j, double *red_f, uint32_t *red_j)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const double of = __shfl_xor_sync(kFull, f, o);
+        const uint32_t oj = __shfl_xor_sync(kFull, j, o);
+        if (of < f || (of == f && oj < j)) {
+            f = of;
+            j = oj;
+        }
+    }
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    __syncthreads();
+    if (lane == 0) {
+        red_f[wid] = f;
+        red_j[wid] = j;
+    }
+    __syncthreads();
+    f = red_f[0];
+    j = red_j[0];
+    for (int w = 1; w < kSpecWarps; w++)
+        if (red_f[w] < f || (red_f[w] == f && red_j[w] < j)) {
+            f = red_f[w];
+            j = red_j[w];
+        }
+}
+
+// Block-wide max over environments of a per-environment sum of per-weight
+// terms (any order: a bound, used with a margin).  kind 0: clipped weights'
+// error at s; kind 1: error of the weights that quantise to 0 at s.
+__device__ double bound_at(const Smem &sm, int n, int E, int qmin, int qmax, uint32_t j, int kind, double *red)
+{
+    const float s = grid_value(j);
+    const double sd = s;
+    double acc[CQ_MAX_E];
+#pragma unroll
+    for (int e = 0; e < CQ_MAX_E; e++)
+        acc[e] = 0.0;
+    for (int i = threadIdx.x; i < n; i += kSpecThreads) {
+        const float w = sm.wf[i];
+        const float aw = fabsf(w);
+        double t = 0.0;
+        if (kind == 0) {
+            const int cap = w < 0.0f ? -qmin : qmax;
+            if (code_at_least(aw, s, cap + 1)) {
+                const double x = static_cast<double>(aw) - cap * sd;
+                t = x * x;
+            }
+        } else if (!code_at_least(aw, s, 1)) {
+            t = sm.wd[i] * sm.wd[i];
+        }
+#pragma unroll
+        for (int e = 0; e < CQ_MAX_E; e++)
+            if (e < E)
+                acc[e] += sm.dd[e * n + i] * t;
+    }
+    double best = 0.0;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+    for (int e = 0; e < CQ_MAX_E; e++) {
+        if (e >= E)
+            break;
+        double v = warp_sum(acc[e]);
+        __syncthreads();
+        if (lane == 0)
+            red[wid] = v;
+        __syncthreads();
+        v = 0.0;
+        for (int w = 0; w < kSpecWarps; w++)
+            v += red[w];
+        best = fmax(best, v);
+    }
+    return best;
+}
+
+__global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
+{
+    extern __shared__ __align__(16) unsigned char dyn[];
+    __shared__ double red_f[kSpecWarps];
+    __shared__ uint32_t red_j[kSpecWarps];
+    __shared__ int flag_bad;
+    __shared__ float amax_s;
+    const int n = p.n, E = p.E;
+    Smem sm;
+    sm.dd = reinterpret_cast<double *>(dyn);
+    sm.wd = sm.dd + static_cast<size_t>(E) * n;
+    sm.wf = reinterpret_cast<float *>(sm.wd + n);
+    const int64_t gpr = p.K > 0 ? p.K / n : 1;
+    constexpr double kKeep = 1.0 - 0x1p-40;
+    for (int64_t g = blockIdx.x; g < p.G; g += gridDim.x) {
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            flag_bad = 0;
+            amax_s = 0.0f;
+        }
+        __syncthreads();
+        // 1. stage
+        float am = 0.0f;
+        int bad = 0;
+        for (int i = threadIdx.x; i < n; i += kSpecThreads) {
+            const uint32_t b = p.W[g * n + i];
+            bad |= (b & 0x7FFFu) >= kBeyond;
+            const float w = half_value(b);
+            sm.wf[i] = w;
+            sm.wd[i] = w;
+            am = fmaxf(am, fabsf(w));
+            for (int e = 0; e < E; e++) {
+                const float d = p.K > 0 ? p.D[e * p.K + (g % gpr) * n + i] : p.D[(e * p.G + g) * n + i];
+                bad |= !(d >= 0.0f && d <= FLT_MAX);
+                sm.dd[e * n + i] = d;
+            }
+        }
+        if (bad)
+            atomicOr(&flag_bad, 1);
+        am = fmaxf(am, __shfl_xor_sync(kFull, am, 16));
+        am = fmaxf(am, __shfl_xor_sync(kFull, am, 8));
+        am = fmaxf(am, __shfl_xor_sync(kFull, am, 4));
+        am = fmaxf(am, __shfl_xor_sync(kFull, am, 2));
+        am = fmaxf(am, __shfl_xor_sync(kFull, am, 1));
+        if ((threadIdx.x & 31) == 0 && am > 0.0f)
+            atomicMax(reinterpret_cast<int *>(&amax_s), __float_as_int(am));  // non-negative floats order as ints
+        __syncthreads();
+        const float amax = amax_s;
+        if (flag_bad || amax == 0.0f) {
+            for (int i = threadIdx.x; i < n; i += kSpecThreads)
+                p.out_codes[g * n + i] = 0;
+            if (threadIdx.x == 0) {
+                p.out_scales[g] = 0x0001;
+                if (p.out_obj)
+                    p.out_obj[g] = 0.0;
+                if (p.out_flags)
+                    p.out_flags[g] = flag_bad ? CQ_FLAG_NONFINITE : CQ_FLAG_TRIVIAL;
+            }
+            continue;
+        }
+        // 2. upper bound from exact objectives at a few scales
+        uint32_t jz = kLast + 1;  // first scale where every code is 0 (s >= 2 max|w|)
+        {
+            const float two = 2.0f * amax;  // exact
+            if (two <= 65504.0f)
+                jz = max(static_cast<uint32_t>(__half_as_ushort(__float2half_ru(two))), 1u);
+        }
+        double f = INFINITY;
+        uint32_t jb = 0xFFFFFFFFu;
+        if (threadIdx.x < kCandidates) {
+            const int t = threadIdx.x;
+            uint32_t j;
+            if (t == 6) {
+                j = jz;
+            } else {
+                const double base = static_cast<double>(amax) / (t < 3 ? p.qmax : -p.qmin);
+                const int off = (t % 3) - 1;
+                const int jc = static_cast<int>(__half_as_ushort(__double2half(base))) + off;
+                j = static_cast<uint32_t>(min(max(jc, 1), static_cast<int>(kLast)));
+            }
+            if (j <= kLast) {
+                f = objective_at(sm, n, E, p.qmin, p.qmax, j);
+                jb = j;
+            }
+        }
+        block_best(f, jb, red_f, red_j);
+        const double U = f;
+        // 3. certified window [J0, J1]
+        uint32_t lo = 1, hi = jb;  // smallest index whose clipping bound does not exclude it
+        if (bound_at(sm, n, E, p.qmin, p.qmax, 1, 0, red_f) * kKeep > U) {
+            while (hi - lo > 1) {  // invariant: lo excluded, hi not
+                const uint32_t mid = (lo + hi) / 2;
+                if (bound_at(sm, n, E, p.qmin, p.qmax, mid, 0, red_f) * kKeep > U)
+                    lo = mid;
+                else
+                    hi = mid;
+            }
+            lo = hi;
+        }
+        const uint32_t J0 = lo;
+        lo = jb;
+        hi = kLast;
+        if (bound_at(sm, n, E, p.qmin, p.qmax, kLast, 1, red_f) * kKeep > U) {
+            while (hi - lo > 1) {  // invariant: lo not excluded, hi excluded
+                const uint32_t mid = (lo + hi) / 2;
+                if (bound_at(sm, n, E, p.qmin, p.qmax, mid, 1, red_f) * kKeep > U)
+                    hi = mid;
+                else
+                    lo = mid;
+            }
+            hi = lo;
+        }
+        const uint32_t J1 = min(hi, jz);
+        // 4. scan the window
+        double bf = INFINITY;
+        uint32_t bj = 0xFFFFFFFFu;
+        for (uint32_t j = J0 + threadIdx.x; j <= J1; j += kSpecThreads) {
+            const double v = objective_at(sm, n, E, p.qmin, p.qmax, j);
+            if (v < bf) {  // ascending j per thread: strict < keeps the lowest pattern
+                bf = v;
+                bj = j;
+            }
+        }
+        if (bf > U || (bf == U && bj > jb)) {  // the bound's own scale may lie outside the scanned range
+            bf = U;
+            bj = jb;
+        }
+        block_best(bf, bj, red_f, red_j);
+        // 5. outputs
+        const float s = grid_value(bj);
+        const float inv = 1.0f / s;
+        for (int i = threadIdx.x; i < n; i += kSpecThreads) {
+            const float w = sm.wf[i];
+            const bool neg = w < 0.0f;
+            const int c = spec_code(fabsf(w), s, inv, neg ? -p.qmin : p.qmax);
+            p.out_codes[g * n + i] = static_cast<int8_t>(neg ? -c : c);
+        }
+        if (threadIdx.x == 0) {
+            p.out_scales[g] = static_cast<uint16_t>(bj);
+            if (p.out_obj)
+                p.out_obj[g] = bf;
+            if (p.out_flags)
+                p.out_flags[g] = 0;
+        }
+    }
+}
+
+}  // namespace
+}  // namespace cq
+
+using namespace cq;
+
+extern "C" {
+
+cq_status cq_select_scales_spec(const uint16_t *W, int64_t G, const float *D, int E, int64_t K,
+                                const cq_quantizer_spec *spec, uint16_t *out_scales, int8_t *out_codes,
+                                double *out_objective, uint8_t *out_flags, void *stream)
+{
+    if (!spec || G < 0 || K < 0 || E < 1)
+        return CQ_ERR_INVALID_ARG;
+    const int n = spec->group_size;
+    if (spec->qmin > -1 || spec->qmax < 1 || n < 1)
+        return CQ_ERR_INVALID_ARG;
+    if (spec->qmin < -128 || spec->qmax > 127 || n > CQ_SPEC_MAX_GROUP || E > CQ_MAX_E ||
+        G >= (static_cast<int64_t>(1) << 31))
+        return CQ_ERR_UNSUPPORTED;
+    if (K > 0 && (K % n != 0 || G % (K / n) != 0))
+        return CQ_ERR_INVALID_ARG;
+    if (G == 0)
+        return CQ_OK;
+    if (!W || !D || !out_scales || !out_codes)
+        return CQ_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(W) & 1) || (reinterpret_cast<uintptr_t>(D) & 3) ||
+        (reinterpret_cast<uintptr_t>(out_scales) & 1) || (reinterpret_cast<uintptr_t>(out_objective) & 7))
+        return CQ_ERR_INVALID_ARG;
+    SpecParams p{W, G, D, E, K, spec->qmin, spec->qmax, n, out_scales, out_codes, out_objective, out_flags};
+    const size_t smem = static_cast<size_t>(E) * n * sizeof(double) + n * sizeof(double) + n * sizeof(float);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(spec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+            cudaSuccess)
+        return CQ_ERR_CUDA;
+    int per_sm = 1, dev = 0, sms = 148;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, spec_kernel, kSpecThreads, smem) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t cap = static_cast<int64_t>(sms) * per_sm;
+    const unsigned grid = static_cast<unsigned>(G < cap ? G : cap);
+    spec_kernel<<<grid, kSpecThreads, smem, static_cast<cudaStream_t>(stream)>>>(p);
+    return cudaGetLastError() == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -176,6 +176,27 @@ def test_diagonal_entry_point_validates(cq):
     assert L.cq_estimate_diagonals(f, 0, 256, vp(None), 2, f, f, vp(None)) == cq.CQ_ERR_INVALID_ARG
 
 
+def test_spec_entry_point_validates(cq):
+    vp, L, f = ctypes.c_void_p, cq.lib, ctypes.c_void_p(FAKE)
+
+    def call(qmin=-4, qmax=3, n=64, G=8, E=2, K=0, W=FAKE, obj=0):
+        spec = cq.QuantizerSpec(qmin, qmax, n)
+        return L.cq_select_scales_spec(vp(W), G, f, E, K, ctypes.byref(spec), f, f, vp(obj), vp(None), vp(None))
+    assert call(qmin=0) == cq.CQ_ERR_INVALID_ARG
+    assert call(qmax=0) == cq.CQ_ERR_INVALID_ARG
+    assert call(n=0) == cq.CQ_ERR_INVALID_ARG
+    assert call(qmin=-129) == cq.CQ_ERR_UNSUPPORTED
+    assert call(qmax=128) == cq.CQ_ERR_UNSUPPORTED
+    assert call(n=2048) == cq.CQ_ERR_UNSUPPORTED
+    assert call(E=9) == cq.CQ_ERR_UNSUPPORTED
+    assert call(K=100) == cq.CQ_ERR_INVALID_ARG     # K % n
+    assert call(G=3, K=128) == cq.CQ_ERR_INVALID_ARG  # G not whole rows of K/n groups
+    assert call(W=FAKE + 1) == cq.CQ_ERR_INVALID_ARG
+    assert call(obj=FAKE + 4) == cq.CQ_ERR_INVALID_ARG
+    assert call(G=0, W=0) == cq.CQ_OK
+    assert L.cq_select_scales_spec(f, 8, f, 2, 0, None, f, f, vp(None), vp(None), vp(None)) == cq.CQ_ERR_INVALID_ARG
+
+
 def test_no_cpu_fallback_in_binding():
     """The binding refuses to run without its CUDA library."""
     src = open(os.path.join(ROOT, "minimax_scale_search_b200", "cq.py")).read()

@@ -8,6 +8,7 @@ import pytest
 
 import oracle
 import test_oracle_pins as pins
+import test_oracle_spec as spec_pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "cq_oracle.c")
 
@@ -25,6 +26,10 @@ MUTANTS = {
     "pack_offset": ("(q[8 * j + t] + 8)", "(q[8 * j + t] + 7)"),
     "domain_skips_first": ("b = CQO_FIRST_SCALE;", "b = CQO_FIRST_SCALE + 1;"),
     "codes_not_clipped_high": ("if (r > (double)qmax)\n            r = (double)qmax;", ""),
+    "qmin_fixed_at_minus_8": ("if (r < (double)qmin)\n            r = (double)qmin;",
+                              "if (r < -8.0)\n            r = -8.0;"),
+    "qmax_fixed_at_7": ("if (r > (double)qmax)\n            r = (double)qmax;",
+                        "if (r > 7.0)\n            r = 7.0;"),
 }
 
 
@@ -42,6 +47,8 @@ def _checks():
         yield lambda c=c: pins.test_oracle_matches_exact_bruteforce(c)
     yield lambda: pins.test_env_duplicate_permute_pow2_invariance(g128)
     yield lambda: pins.test_bounds_absmax_single_env_and_added_env(g128)
+    for spec in spec_pins.SPECS:
+        yield lambda spec=spec: spec_pins.test_spec_matches_exact_bruteforce(spec)
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
