@@ -8,8 +8,9 @@
 // with an exact tie going to the lower bit pattern, and emit the codes packed
 // as (q+8) nibbles, 8 per uint32, low nibble first.
 //
-// Design (one warp per group, persistent grid, no tensor cores: the work is
-// comparisons and short fp64 dot products, not a dense contraction):
+// Design (one warp per group, persistent grid of one CTA per SM whose 16-20
+// warps start each group together; no tensor cores: the work is comparisons
+// and short fp64 dot products, not a dense contraction):
 //
 //  1. Load: 8-byte weight loads and 16-byte diagonal loads per lane; the
 //     group's w and d are staged in shared memory for indexed access.
@@ -52,7 +53,14 @@
 
 namespace cq {
 
-constexpr int kWarps = 4;              // warps (groups in flight) per CTA of the main kernel
+// Warps (groups in flight) per CTA of the main kernel.  One CTA fills an SM and
+// its warps start every group together, so the warps that share a scheduler
+// tend to run the same phase and share its instructions in cache (the kernel's
+// code is ~110 KB; with independent CTAs per SM, instruction fetch was the top
+// stall).  20 warps of <= 96 registers fit the register file for E <= 4;
+// larger E needs more shared memory per warp and up to 128 registers: 16.
+template <int E>
+constexpr int kWarpsPerCta = E <= 4 ? 20 : 16;
 constexpr uint32_t kInvalidKey = 0xFFFFFFFFu;
 constexpr int kMaxFinalists = 64;
 constexpr int kDefaultFinalists = 32;
@@ -1146,19 +1154,24 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
 }
 
 template <int E>
-__global__ void __launch_bounds__(kWarps * 32, (E <= 4 ? 5 : 4)) select_kernel(Params p)
+__global__ void __launch_bounds__(kWarpsPerCta<E> * 32, 1) select_kernel(Params p)
 {
+    constexpr int kWarps = kWarpsPerCta<E>;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int lane = threadIdx.x & 31;
     const int wib = threadIdx.x >> 5;
     WarpSmem<E> &sm = reinterpret_cast<WarpSmem<E> *>(smem_raw)[wib];
     Tally tl;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * kWarps;
-    for (int64_t g = static_cast<int64_t>(blockIdx.x) * kWarps + wib; g < p.G; g += stride) {
-        if (lane < 2 && g + stride < p.G)
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(p.W + (g + stride) * kGroup + 64 * lane));
-        process_group<E>(p, sm, g, lane, tl);
-        __syncwarp();
+    // the trip count is the same for every warp of the CTA, so the barrier is uniform
+    for (int64_t b0 = static_cast<int64_t>(blockIdx.x) * kWarps; b0 < p.G; b0 += stride) {
+        const int64_t g = b0 + wib;
+        if (g < p.G) {
+            if (lane < 2 && g + stride < p.G)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(p.W + (g + stride) * kGroup + 64 * lane));
+            process_group<E>(p, sm, g, lane, tl);
+        }
+        __syncthreads();  // the warps start the next group together
     }
     if (lane == 0) {
         const uint32_t v[7] = {tl.fallback, tl.near_tie, tl.nonfinite, tl.trivial, tl.finalists, tl.uncertain,
@@ -1365,6 +1378,7 @@ cudaError_t launch(const Params &p, cudaStream_t st)
     if (err != cudaSuccess)
         return err;
     const int sms = sm_count(dev);
+    constexpr int kWarps = kWarpsPerCta<E>;
     const size_t smem = sizeof(WarpSmem<E>) * kWarps;
     err = cudaFuncSetAttribute(select_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
