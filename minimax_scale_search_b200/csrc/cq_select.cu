@@ -596,10 +596,20 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
 #pragma unroll
             for (int e = 0; e < E; e++)
                 acc[c][e] = 0.0f;
-#pragma unroll 1
+        const float4 w4 = *reinterpret_cast<const float4 *>(&sm.w[4 * lane]);
+        const float wq[4] = {w4.x, w4.y, w4.z, w4.w};
+        float dq[E][4];
+#pragma unroll
+        for (int e = 0; e < E; e++) {
+            const float4 t = *reinterpret_cast<const float4 *>(&sm.d[e][4 * lane]);
+            dq[e][0] = t.x;
+            dq[e][1] = t.y;
+            dq[e][2] = t.z;
+            dq[e][3] = t.w;
+        }
+#pragma unroll
         for (int m = 0; m < 4; m++) {
-            const int r = 32 * m + lane;
-            const float wv = sm.w[r];
+            const float wv = wq[m];
             const float aw = fabsf(wv);
             const int K = wv < 0.0f ? 8 : 7;
 #pragma unroll
@@ -612,7 +622,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
                 const float rr = res * res;
 #pragma unroll
                 for (int e = 0; e < E; e++)
-                    acc[c][e] = fmaf(sm.d[e][r], rr, acc[c][e]);
+                    acc[c][e] = fmaf(dq[e][m], rr, acc[c][e]);
             }
         }
         U = INFINITY;
@@ -637,32 +647,33 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     {
         // prefix sums over ranks of d w^2 (fp32), ph[e][c] = sum over ranks < c
         float *ph = reinterpret_cast<float *>(sm.bufB);  // [E][kGroup + 1]
-        float carry[E];
+        // lane L sums ranks 4L .. 4L+3 locally, then one warp scan per environment
+        // (w^2 is exact; each entry passes through at most 10 fp32 roundings)
+        const float4 w4 = *reinterpret_cast<const float4 *>(&sm.w[4 * lane]);
+        const float q0 = w4.x * w4.x, q1 = w4.y * w4.y, q2 = w4.z * w4.z, q3 = w4.w * w4.w;
 #pragma unroll
-        for (int e = 0; e < E; e++)
-            carry[e] = 0.0f;
-        if (lane == 0) {
+        for (int e = 0; e < E; e++) {
+            const float4 d4 = *reinterpret_cast<const float4 *>(&sm.d[e][4 * lane]);
+            const float a0 = d4.x * q0;
+            const float a1 = fmaf(d4.y, q1, a0);
+            const float a2 = fmaf(d4.z, q2, a1);
+            const float a3 = fmaf(d4.w, q3, a2);
+            float v = a3;
 #pragma unroll
-            for (int e = 0; e < E; e++)
-                ph[e * (kGroup + 1)] = 0.0f;
-        }
-#pragma unroll 1
-        for (int m = 0; m < 4; m++) {
-            const int r = 32 * m + lane;
-            const float wv = sm.w[r];
-            const float w2 = wv * wv;
-#pragma unroll
-            for (int e = 0; e < E; e++) {
-                float v = sm.d[e][r] * w2;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float u = __shfl_up_sync(kFull, v, o);
-                    if (lane >= o)
-                        v += u;
-                }
-                ph[e * (kGroup + 1) + r + 1] = carry[e] + v;
-                carry[e] += __shfl_sync(kFull, v, 31);
+            for (int o = 1; o < 32; o <<= 1) {
+                const float u = __shfl_up_sync(kFull, v, o);
+                if (lane >= o)
+                    v += u;
             }
+            const float before = __shfl_up_sync(kFull, v, 1);  // sum over lanes < L
+            const float base = lane == 0 ? 0.0f : before;
+            float *row = ph + e * (kGroup + 1) + 4 * lane;
+            if (lane == 0)
+                row[0] = 0.0f;
+            row[1] = base + a0;
+            row[2] = base + a1;
+            row[3] = base + a2;
+            row[4] = base + a3;
         }
         // lower end: clip bound of the top 8 weights at scale ja0 - 128 * lane
         const uint32_t jl = ja0 > 128u * lane ? ja0 - 128u * lane : 1u;
