@@ -130,6 +130,50 @@ __device__ __forceinline__ uint32_t transition_index(float aw, int k)
     return j0 + 1;
 }
 
+template <int N>
+struct Pow2Up {
+    static constexpr int value = 2 * Pow2Up<(N + 1) / 2>::value;
+};
+template <>
+struct Pow2Up<1> {
+    static constexpr int value = 1;
+};
+
+// Totals of n values summed across the warp, every lane receiving all of them.
+// A reduce-scatter halves the values a lane carries at each of the first
+// log2(N) butterfly steps (N = n rounded up to a power of two), the remaining
+// steps add the one value left, and each total is then read from a lane that
+// holds it.  The lanes pair up at offsets 16, 8, 4, 2, 1 exactly as in a plain
+// butterfly, so every total has the same bits as warp_sum's, with 2N + 5 - log2 N
+// shuffles instead of 5n.
+template <int n, typename T>
+__device__ __forceinline__ void warp_sum_all(T (&v)[n], int lane)
+{
+    constexpr int N = Pow2Up<n>::value;
+    static_assert(N <= 32, "at most 32 values");
+    T x[N];
+#pragma unroll
+    for (int i = 0; i < N; i++)
+        x[i] = i < n ? v[i] : T(0);
+    int o = 16;
+#pragma unroll
+    for (int h = N / 2; h >= 1; h /= 2, o >>= 1) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < h; i++) {
+            const T send = up ? x[i] : x[i + h];
+            const T keep = up ? x[i + h] : x[i];
+            x[i] = keep + __shfl_xor_sync(kFull, send, o);
+        }
+    }
+#pragma unroll
+    for (; o > 0; o >>= 1)
+        x[0] += __shfl_xor_sync(kFull, x[0], o);
+#pragma unroll
+    for (int j = 0; j < n; j++)
+        v[j] = __shfl_sync(kFull, x[0], j * (32 / N));
+}
+
 __device__ __forceinline__ void cx_asc(uint32_t &a, uint32_t &b)
 {
     const uint32_t lo = min(a, b);
@@ -488,10 +532,17 @@ __device__ __forceinline__ void direct_coefficients(const WarpSmem<E> &sm, float
             C[e] = fma(dd, cq, C[e]);
         }
     }
+    double t[2 * E];
 #pragma unroll
     for (int e = 0; e < E; e++) {
-        B[e] = warp_sum(B[e]);
-        C[e] = warp_sum(C[e]);
+        t[e] = B[e];
+        t[E + e] = C[e];
+    }
+    warp_sum_all(t, lane);
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        B[e] = t[e];
+        C[e] = t[E + e];
     }
 }
 
@@ -1128,10 +1179,11 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
             for (int e = 0; e < E; e++)
                 acc[e] = __dadd_rn(acc[e], __dmul_rn(static_cast<double>(sm.d[e][r]), rr));
         }
+        warp_sum_all(acc, lane);
         double v = -INFINITY;
 #pragma unroll
         for (int e = 0; e < E; e++)
-            v = fmax(v, warp_sum(acc[e]));
+            v = fmax(v, acc[e]);
         if (v < best || (v == best && j < bj)) {
             second = best;
             best = v;
