@@ -86,7 +86,9 @@ __device__ double objective_at(const Smem &sm, int n, int E, int qmin, int qmax,
 #pragma unroll
     for (int e = 0; e < CQ_MAX_E; e++)
         acc[e] = 0.0;
-    for (int i = 0; i < n; i++) {
+    // the codes of 4 consecutive weights are computed independently; each
+    // environment's running sum still takes the weights in ascending order
+    auto term = [&](int i) {
         const float w = sm.wf[i];
         const bool neg = w < 0.0f;
         const int c = spec_code(fabsf(w), s, inv, neg ? -qmin : qmax);
@@ -96,7 +98,15 @@ __device__ double objective_at(const Smem &sm, int n, int E, int qmin, int qmax,
         for (int e = 0; e < CQ_MAX_E; e++)
             if (e < E)
                 acc[e] = __dadd_rn(acc[e], __dmul_rn(sm.dd[e * n + i], rr));
+    };
+    int i = 0;
+    for (; i + 4 <= n; i += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; u++)
+            term(i + u);
     }
+    for (; i < n; i++)
+        term(i);
     double f = acc[0];
 #pragma unroll
     for (int e = 1; e < CQ_MAX_E; e++)
@@ -133,10 +143,45 @@ __device__ void block_best(double &f, uint32_t &j, double *red_f, uint32_t *red_
         }
 }
 
+// Block-wide sums of E per-thread values, every thread getting the totals.
+// The scratch alternates between two halves; each thread keeps the parity in
+// a register (every thread makes the same calls).  One barrier per call keeps
+// a call's writes from overtaking the previous call's reads: a thread writes a
+// half again only after the next call's barrier, which every thread reaches
+// after its reads.
+struct BlockScratch {
+    double (*v)[kSpecWarps][CQ_MAX_E];  // two halves in shared memory
+    int half;                           // this thread's parity
+};
+
+__device__ void block_sum_env(double (&acc)[CQ_MAX_E], int E, BlockScratch &bs)
+{
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    double(*buf)[CQ_MAX_E] = bs.v[bs.half];
+    bs.half ^= 1;
+#pragma unroll
+    for (int e = 0; e < CQ_MAX_E; e++)
+        if (e < E) {
+            const double v = warp_sum(acc[e]);
+            if (lane == 0)
+                buf[wid][e] = v;
+        }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < CQ_MAX_E; e++)
+        if (e < E) {
+            double v = 0.0;
+            for (int w = 0; w < kSpecWarps; w++)
+                v += buf[w][e];
+            acc[e] = v;
+        }
+}
+
 // Block-wide max over environments of a per-environment sum of per-weight
 // terms (any order: a bound, used with a margin).  kind 0: clipped weights'
 // error at s; kind 1: error of the weights that quantise to 0 at s.
-__device__ double bound_at(const Smem &sm, int n, int E, int qmin, int qmax, uint32_t j, int kind, double *red)
+__device__ double bound_at(const Smem &sm, int n, int E, int qmin, int qmax, uint32_t j, int kind,
+                           BlockScratch &bs)
 {
     const float s = grid_value(j);
     const double sd = s;
@@ -162,23 +207,46 @@ __device__ double bound_at(const Smem &sm, int n, int E, int qmin, int qmax, uin
             if (e < E)
                 acc[e] += sm.dd[e * n + i] * t;
     }
+    block_sum_env(acc, E, bs);
     double best = 0.0;
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
 #pragma unroll
-    for (int e = 0; e < CQ_MAX_E; e++) {
-        if (e >= E)
-            break;
-        double v = warp_sum(acc[e]);
-        __syncthreads();
-        if (lane == 0)
-            red[wid] = v;
-        __syncthreads();
-        v = 0.0;
-        for (int w = 0; w < kSpecWarps; w++)
-            v += red[w];
-        best = fmax(best, v);
-    }
+    for (int e = 0; e < CQ_MAX_E; e++)
+        if (e < E)
+            best = fmax(best, acc[e]);
     return best;
+}
+
+// An upper bound of the objective at grid index j that the whole block sums in
+// any order: the exact value's fp64 sums err by at most n 2^-53 relative either
+// way, so the block sum times (1 + 2^-40) is at least the definition's own
+// value for n <= 4096.
+__device__ double upper_at(const Smem &sm, int n, int E, int qmin, int qmax, uint32_t j, BlockScratch &bs)
+{
+    const float s = grid_value(j);
+    const float inv = 1.0f / s;
+    const double nsd = -static_cast<double>(s);
+    double acc[CQ_MAX_E];
+#pragma unroll
+    for (int e = 0; e < CQ_MAX_E; e++)
+        acc[e] = 0.0;
+    for (int i = threadIdx.x; i < n; i += kSpecThreads) {
+        const float w = sm.wf[i];
+        const bool neg = w < 0.0f;
+        const int c = spec_code(fabsf(w), s, inv, neg ? -qmin : qmax);
+        const double r = fma(nsd, static_cast<double>(neg ? -c : c), sm.wd[i]);
+        const double rr = r * r;
+#pragma unroll
+        for (int e = 0; e < CQ_MAX_E; e++)
+            if (e < E)
+                acc[e] = fma(sm.dd[e * n + i], rr, acc[e]);
+    }
+    block_sum_env(acc, E, bs);
+    double f = 0.0;
+#pragma unroll
+    for (int e = 0; e < CQ_MAX_E; e++)
+        if (e < E)
+            f = fmax(f, acc[e]);
+    return f * (1.0 + 0x1p-40);
 }
 
 __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
@@ -186,6 +254,8 @@ __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
     extern __shared__ __align__(16) unsigned char dyn[];
     __shared__ double red_f[kSpecWarps];
     __shared__ uint32_t red_j[kSpecWarps];
+    __shared__ double scratch[2][kSpecWarps][CQ_MAX_E];
+    BlockScratch bs{scratch, 0};
     __shared__ int flag_bad;
     __shared__ float amax_s;
     const int n = p.n, E = p.E;
@@ -248,12 +318,14 @@ __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
             if (two <= 65504.0f)
                 jz = max(static_cast<uint32_t>(__half_as_ushort(__float2half_ru(two))), 1u);
         }
-        double f = INFINITY;
-        uint32_t jb = 0xFFFFFFFFu;
-        if (threadIdx.x < kCandidates) {
-            const int t = threadIdx.x;
+        // Every thread evaluates the same candidates, so U and jb are uniform.
+        // jb lies in the window found below (its bounds are below U there) and
+        // below j_z, so the scan evaluates it exactly.
+        double U = INFINITY;
+        uint32_t jb = 1;
+        for (int t = 0; t < kCandidates; t++) {
             uint32_t j;
-            if (t == 6) {
+            if (t == kCandidates - 1) {
                 j = jz;
             } else {
                 const double base = static_cast<double>(amax) / (t < 3 ? p.qmax : -p.qmin);
@@ -261,19 +333,20 @@ __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
                 const int jc = static_cast<int>(__half_as_ushort(__double2half(base))) + off;
                 j = static_cast<uint32_t>(min(max(jc, 1), static_cast<int>(kLast)));
             }
-            if (j <= kLast) {
-                f = objective_at(sm, n, E, p.qmin, p.qmax, j);
+            if (j > kLast)
+                continue;
+            const double u = upper_at(sm, n, E, p.qmin, p.qmax, j, bs);
+            if (u < U) {
+                U = u;
                 jb = j;
             }
         }
-        block_best(f, jb, red_f, red_j);
-        const double U = f;
         // 3. certified window [J0, J1]
         uint32_t lo = 1, hi = jb;  // smallest index whose clipping bound does not exclude it
-        if (bound_at(sm, n, E, p.qmin, p.qmax, 1, 0, red_f) * kKeep > U) {
+        if (bound_at(sm, n, E, p.qmin, p.qmax, 1, 0, bs) * kKeep > U) {
             while (hi - lo > 1) {  // invariant: lo excluded, hi not
                 const uint32_t mid = (lo + hi) / 2;
-                if (bound_at(sm, n, E, p.qmin, p.qmax, mid, 0, red_f) * kKeep > U)
+                if (bound_at(sm, n, E, p.qmin, p.qmax, mid, 0, bs) * kKeep > U)
                     lo = mid;
                 else
                     hi = mid;
@@ -283,10 +356,10 @@ __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
         const uint32_t J0 = lo;
         lo = jb;
         hi = kLast;
-        if (bound_at(sm, n, E, p.qmin, p.qmax, kLast, 1, red_f) * kKeep > U) {
+        if (bound_at(sm, n, E, p.qmin, p.qmax, kLast, 1, bs) * kKeep > U) {
             while (hi - lo > 1) {  // invariant: lo not excluded, hi excluded
                 const uint32_t mid = (lo + hi) / 2;
-                if (bound_at(sm, n, E, p.qmin, p.qmax, mid, 1, red_f) * kKeep > U)
+                if (bound_at(sm, n, E, p.qmin, p.qmax, mid, 1, bs) * kKeep > U)
                     hi = mid;
                 else
                     lo = mid;
@@ -303,10 +376,6 @@ __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
                 bf = v;
                 bj = j;
             }
-        }
-        if (bf > U || (bf == U && bj > jb)) {  // the bound's own scale may lie outside the scanned range
-            bf = U;
-            bj = jb;
         }
         block_best(bf, bj, red_f, red_j);
         // 5. outputs
