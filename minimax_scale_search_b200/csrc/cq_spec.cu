@@ -40,6 +40,9 @@ namespace {
 constexpr int kSpecThreads = 256;
 constexpr int kSpecWarps = kSpecThreads / 32;
 constexpr int kCandidates = 7;
+constexpr uint32_t kChunk = 32;                               // scales per interval bound
+constexpr int kMaxChunks = (static_cast<int>(kLast) + 31) / 32;  // 992
+constexpr float kKeepChunk = 1.0f - 0x1p-12f;                  // covers the fp32 rounding of a bound
 
 struct SpecParams {
     const uint16_t *W;
@@ -249,12 +252,55 @@ __device__ double upper_at(const Smem &sm, int n, int E, int qmin, int qmax, uin
     return f * (1.0 + 0x1p-40);
 }
 
+// A lower bound of the objective at every scale in [s_lo, s_hi]: at any such s
+// the residual of weight i is at least its distance to the union of the
+// intervals [k s_lo, k s_hi], k = 0..cap, which is zero if |w| lies in one of
+// them and otherwise min(|w| - k1 s_hi, k2 s_lo - |w|) with k1 the largest k
+// whose interval ends at or below |w| (at most cap) and k2 = k1 + 1 (at most
+// cap).  An fp32 floor off by one only lowers the computed distance.  Each
+// term passes through 3 fp32 roundings and the running sum through n - 1, so
+// for n <= 1024 the computed bound errs by less than 2^-14 relative; a chunk is
+// skipped only when the bound times 1 - 2^-12 exceeds U, which leaves the exact
+// bound, and so the definition's fp64 objective at every scale of the chunk,
+// above U.
+__device__ float chunk_bound(const Smem &sm, int n, int E, int qmin, int qmax, float s_lo, float s_hi)
+{
+    const float inv_hi = 1.0f / s_hi;
+    float acc[CQ_MAX_E];
+#pragma unroll
+    for (int e = 0; e < CQ_MAX_E; e++)
+        acc[e] = 0.0f;
+    for (int i = 0; i < n; i++) {
+        const float w = sm.wf[i];
+        const float aw = fabsf(w);
+        const float cap = static_cast<float>(w < 0.0f ? -qmin : qmax);
+        const float k1 = fminf(floorf(aw * inv_hi), cap);
+        const float e1 = fmaxf(fmaf(-k1, s_hi, aw), 0.0f);
+        const float e2 = k1 < cap ? fmaxf(fmaf(k1 + 1.0f, s_lo, -aw), 0.0f) : INFINITY;
+        const float dist = fminf(e1, e2);
+        const float d2 = dist * dist;
+#pragma unroll
+        for (int e = 0; e < CQ_MAX_E; e++)
+            if (e < E)
+                acc[e] = fmaf(static_cast<float>(sm.dd[e * n + i]), d2, acc[e]);
+    }
+    float best = 0.0f;
+#pragma unroll
+    for (int e = 0; e < CQ_MAX_E; e++)
+        if (e < E)
+            best = fmaxf(best, acc[e]);
+    return best;
+}
+
 __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
 {
     extern __shared__ __align__(16) unsigned char dyn[];
     __shared__ double red_f[kSpecWarps];
     __shared__ uint32_t red_j[kSpecWarps];
     __shared__ double scratch[2][kSpecWarps][CQ_MAX_E];
+    __shared__ bool keep[kMaxChunks];
+    __shared__ uint16_t kept[kMaxChunks];
+    __shared__ int nkept;
     BlockScratch bs{scratch, 0};
     __shared__ int flag_bad;
     __shared__ float amax_s;
@@ -367,10 +413,36 @@ __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
             hi = lo;
         }
         const uint32_t J1 = min(hi, jz);
-        // 4. scan the window
+        // 4. chunks of kChunk scales whose interval bound exceeds U are skipped
+        const int nch = static_cast<int>((J1 - J0) / kChunk + 1);
+        for (int ch = threadIdx.x; ch < nch; ch += kSpecThreads) {
+            const uint32_t a = J0 + static_cast<uint32_t>(ch) * kChunk;
+            const uint32_t b = min(a + kChunk - 1, J1);
+            keep[ch] = chunk_bound(sm, n, E, p.qmin, p.qmax, grid_value(a), grid_value(b)) * kKeepChunk <= U;
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) {  // compact the kept chunks, ascending
+            int m = 0;
+            for (int c0 = 0; c0 < nch; c0 += 32) {
+                const int ch = c0 + static_cast<int>(threadIdx.x);
+                const bool k = ch < nch && keep[ch];
+                const unsigned bal = __ballot_sync(kFull, k);
+                if (k)
+                    kept[m + __popc(bal & ((1u << threadIdx.x) - 1u))] = static_cast<uint16_t>(ch);
+                m += __popc(bal);
+            }
+            if (threadIdx.x == 0)
+                nkept = m;
+        }
+        __syncthreads();
+        // 5. scan the kept scales
         double bf = INFINITY;
         uint32_t bj = 0xFFFFFFFFu;
-        for (uint32_t j = J0 + threadIdx.x; j <= J1; j += kSpecThreads) {
+        const int nscan = nkept * kChunk;
+        for (int u = threadIdx.x; u < nscan; u += kSpecThreads) {
+            const uint32_t j = J0 + static_cast<uint32_t>(kept[u / kChunk]) * kChunk + (u % kChunk);
+            if (j > J1)
+                break;  // only the last kept chunk can be short, and u grows with j
             const double v = objective_at(sm, n, E, p.qmin, p.qmax, j);
             if (v < bf) {  // ascending j per thread: strict < keeps the lowest pattern
                 bf = v;
@@ -378,7 +450,7 @@ __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
             }
         }
         block_best(bf, bj, red_f, red_j);
-        // 5. outputs
+        // 6. outputs
         const float s = grid_value(bj);
         const float inv = 1.0f / s;
         for (int i = threadIdx.x; i < n; i += kSpecThreads) {
