@@ -80,7 +80,8 @@ struct Smem {
 };
 
 // Objective at grid index j, in the definition's order; one thread.
-__device__ double objective_at(const Smem &sm, int n, int E, int qmin, int qmax, uint32_t j)
+template <int E>
+__device__ double objective_at(const Smem &sm, int n, int qmin, int qmax, uint32_t j)
 {
     const float s = grid_value(j);
     const float inv = 1.0f / s;
@@ -157,7 +158,8 @@ struct BlockScratch {
     int half;                           // this thread's parity
 };
 
-__device__ void block_sum_env(double (&acc)[CQ_MAX_E], int E, BlockScratch &bs)
+template <int E>
+__device__ void block_sum_env(double (&acc)[CQ_MAX_E], BlockScratch &bs)
 {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     double(*buf)[CQ_MAX_E] = bs.v[bs.half];
@@ -183,8 +185,8 @@ __device__ void block_sum_env(double (&acc)[CQ_MAX_E], int E, BlockScratch &bs)
 // Block-wide max over environments of a per-environment sum of per-weight
 // terms (any order: a bound, used with a margin).  kind 0: clipped weights'
 // error at s; kind 1: error of the weights that quantise to 0 at s.
-__device__ double bound_at(const Smem &sm, int n, int E, int qmin, int qmax, uint32_t j, int kind,
-                           BlockScratch &bs)
+template <int E>
+__device__ double bound_at(const Smem &sm, int n, int qmin, int qmax, uint32_t j, int kind, BlockScratch &bs)
 {
     const float s = grid_value(j);
     const double sd = s;
@@ -210,7 +212,7 @@ __device__ double bound_at(const Smem &sm, int n, int E, int qmin, int qmax, uin
             if (e < E)
                 acc[e] += sm.dd[e * n + i] * t;
     }
-    block_sum_env(acc, E, bs);
+    block_sum_env<E>(acc, bs);
     double best = 0.0;
 #pragma unroll
     for (int e = 0; e < CQ_MAX_E; e++)
@@ -223,7 +225,8 @@ __device__ double bound_at(const Smem &sm, int n, int E, int qmin, int qmax, uin
 // any order: the exact value's fp64 sums err by at most n 2^-53 relative either
 // way, so the block sum times (1 + 2^-40) is at least the definition's own
 // value for n <= 4096.
-__device__ double upper_at(const Smem &sm, int n, int E, int qmin, int qmax, uint32_t j, BlockScratch &bs)
+template <int E>
+__device__ double upper_at(const Smem &sm, int n, int qmin, int qmax, uint32_t j, BlockScratch &bs)
 {
     const float s = grid_value(j);
     const float inv = 1.0f / s;
@@ -243,7 +246,7 @@ __device__ double upper_at(const Smem &sm, int n, int E, int qmin, int qmax, uin
             if (e < E)
                 acc[e] = fma(sm.dd[e * n + i], rr, acc[e]);
     }
-    block_sum_env(acc, E, bs);
+    block_sum_env<E>(acc, bs);
     double f = 0.0;
 #pragma unroll
     for (int e = 0; e < CQ_MAX_E; e++)
@@ -263,7 +266,8 @@ __device__ double upper_at(const Smem &sm, int n, int E, int qmin, int qmax, uin
 // skipped only when the bound times 1 - 2^-12 exceeds U, which leaves the exact
 // bound, and so the definition's fp64 objective at every scale of the chunk,
 // above U.
-__device__ float chunk_bound(const Smem &sm, int n, int E, int qmin, int qmax, float s_lo, float s_hi)
+template <int E>
+__device__ float chunk_bound(const Smem &sm, int n, int qmin, int qmax, float s_lo, float s_hi)
 {
     const float inv_hi = 1.0f / s_hi;
     float acc[CQ_MAX_E];
@@ -292,6 +296,7 @@ __device__ float chunk_bound(const Smem &sm, int n, int E, int qmin, int qmax, f
     return best;
 }
 
+template <int E>
 __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
 {
     extern __shared__ __align__(16) unsigned char dyn[];
@@ -304,7 +309,7 @@ __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
     BlockScratch bs{scratch, 0};
     __shared__ int flag_bad;
     __shared__ float amax_s;
-    const int n = p.n, E = p.E;
+    const int n = p.n;
     Smem sm;
     sm.dd = reinterpret_cast<double *>(dyn);
     sm.wd = sm.dd + static_cast<size_t>(E) * n;
@@ -381,7 +386,7 @@ __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
             }
             if (j > kLast)
                 continue;
-            const double u = upper_at(sm, n, E, p.qmin, p.qmax, j, bs);
+            const double u = upper_at<E>(sm, n, p.qmin, p.qmax, j, bs);
             if (u < U) {
                 U = u;
                 jb = j;
@@ -389,10 +394,10 @@ __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
         }
         // 3. certified window [J0, J1]
         uint32_t lo = 1, hi = jb;  // smallest index whose clipping bound does not exclude it
-        if (bound_at(sm, n, E, p.qmin, p.qmax, 1, 0, bs) * kKeep > U) {
+        if (bound_at<E>(sm, n, p.qmin, p.qmax, 1, 0, bs) * kKeep > U) {
             while (hi - lo > 1) {  // invariant: lo excluded, hi not
                 const uint32_t mid = (lo + hi) / 2;
-                if (bound_at(sm, n, E, p.qmin, p.qmax, mid, 0, bs) * kKeep > U)
+                if (bound_at<E>(sm, n, p.qmin, p.qmax, mid, 0, bs) * kKeep > U)
                     lo = mid;
                 else
                     hi = mid;
@@ -402,10 +407,10 @@ __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
         const uint32_t J0 = lo;
         lo = jb;
         hi = kLast;
-        if (bound_at(sm, n, E, p.qmin, p.qmax, kLast, 1, bs) * kKeep > U) {
+        if (bound_at<E>(sm, n, p.qmin, p.qmax, kLast, 1, bs) * kKeep > U) {
             while (hi - lo > 1) {  // invariant: lo not excluded, hi excluded
                 const uint32_t mid = (lo + hi) / 2;
-                if (bound_at(sm, n, E, p.qmin, p.qmax, mid, 1, bs) * kKeep > U)
+                if (bound_at<E>(sm, n, p.qmin, p.qmax, mid, 1, bs) * kKeep > U)
                     hi = mid;
                 else
                     lo = mid;
@@ -418,7 +423,7 @@ __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
         for (int ch = threadIdx.x; ch < nch; ch += kSpecThreads) {
             const uint32_t a = J0 + static_cast<uint32_t>(ch) * kChunk;
             const uint32_t b = min(a + kChunk - 1, J1);
-            keep[ch] = chunk_bound(sm, n, E, p.qmin, p.qmax, grid_value(a), grid_value(b)) * kKeepChunk <= U;
+            keep[ch] = chunk_bound<E>(sm, n, p.qmin, p.qmax, grid_value(a), grid_value(b)) * kKeepChunk <= U;
         }
         __syncthreads();
         if (threadIdx.x < 32) {  // compact the kept chunks, ascending
@@ -443,7 +448,7 @@ __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
             const uint32_t j = J0 + static_cast<uint32_t>(kept[u / kChunk]) * kChunk + (u % kChunk);
             if (j > J1)
                 break;  // only the last kept chunk can be short, and u grows with j
-            const double v = objective_at(sm, n, E, p.qmin, p.qmax, j);
+            const double v = objective_at<E>(sm, n, p.qmin, p.qmax, j);
             if (v < bf) {  // ascending j per thread: strict < keeps the lowest pattern
                 bf = v;
                 bj = j;
@@ -467,6 +472,28 @@ __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
                 p.out_flags[g] = 0;
         }
     }
+}
+
+template <int E>
+cudaError_t launch_spec(const SpecParams &p, cudaStream_t st)
+{
+    const int n = p.n;
+    const size_t smem = static_cast<size_t>(E) * n * sizeof(double) + n * sizeof(double) + n * sizeof(float);
+    cudaError_t err = cudaSuccess;
+    if (smem > 48 * 1024 &&
+        (err = cudaFuncSetAttribute(spec_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(smem))) != cudaSuccess)
+        return err;
+    int per_sm = 1, dev = 0, sms = 148;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, spec_kernel<E>, kSpecThreads, smem) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t cap = static_cast<int64_t>(sms) * per_sm;
+    const unsigned grid = static_cast<unsigned>(p.G < cap ? p.G : cap);
+    spec_kernel<E><<<grid, kSpecThreads, smem, st>>>(p);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -498,21 +525,19 @@ cq_status cq_select_scales_spec(const uint16_t *W, int64_t G, const float *D, in
         (reinterpret_cast<uintptr_t>(out_scales) & 1) || (reinterpret_cast<uintptr_t>(out_objective) & 7))
         return CQ_ERR_INVALID_ARG;
     SpecParams p{W, G, D, E, K, spec->qmin, spec->qmax, n, out_scales, out_codes, out_objective, out_flags};
-    const size_t smem = static_cast<size_t>(E) * n * sizeof(double) + n * sizeof(double) + n * sizeof(float);
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(spec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-            cudaSuccess)
-        return CQ_ERR_CUDA;
-    int per_sm = 1, dev = 0, sms = 148;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, spec_kernel, kSpecThreads, smem) != cudaSuccess ||
-        per_sm < 1)
-        per_sm = 1;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int64_t cap = static_cast<int64_t>(sms) * per_sm;
-    const unsigned grid = static_cast<unsigned>(G < cap ? G : cap);
-    spec_kernel<<<grid, kSpecThreads, smem, static_cast<cudaStream_t>(stream)>>>(p);
-    return cudaGetLastError() == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
+    cudaError_t err = cudaErrorInvalidValue;
+    switch (E) {
+    case 1: err = launch_spec<1>(p, static_cast<cudaStream_t>(stream)); break;
+    case 2: err = launch_spec<2>(p, static_cast<cudaStream_t>(stream)); break;
+    case 3: err = launch_spec<3>(p, static_cast<cudaStream_t>(stream)); break;
+    case 4: err = launch_spec<4>(p, static_cast<cudaStream_t>(stream)); break;
+    case 5: err = launch_spec<5>(p, static_cast<cudaStream_t>(stream)); break;
+    case 6: err = launch_spec<6>(p, static_cast<cudaStream_t>(stream)); break;
+    case 7: err = launch_spec<7>(p, static_cast<cudaStream_t>(stream)); break;
+    case 8: err = launch_spec<8>(p, static_cast<cudaStream_t>(stream)); break;
+    default: break;
+    }
+    return err == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
 }
 
 }  // extern "C"
