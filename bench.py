@@ -95,6 +95,26 @@ def recorded_traffic(groups: int):
     return float(kv["dram_bytes"]) / float(kv["groups"]) * groups
 
 
+def recorded_kernel_traffic(kernel: str, units: int):
+    """DRAM bytes of one launch of a secondary kernel over `units` units, from the
+    committed ncu record (profiles/secondary_kernels_traffic.txt) scaled by
+    units; None when the kernel's source changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "secondary_kernels_traffic.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    for ln in lines:
+        kv = dict(tok.split("=", 1) for tok in ln.split() if "=" in tok)
+        if kv.get("kernel") != kernel:
+            continue
+        src = os.path.join(ROOT, "minimax_scale_search_b200", "csrc", kv["src"])
+        if hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != kv.get("sha"):
+            return None
+        return float(kv["dram_bytes"]) / float(kv["units"]) * units
+    return None
+
+
 class ClockSampler:
     """nvidia-smi samples (200 ms) of SM clock and throttle reasons."""
 
@@ -273,7 +293,8 @@ def bench_policies(args, wl, W, D, Wd, Dd, dev):
     lines.append(dict(base, metric="AbsMax policy groups/sec", op="absmax", value=G / ms * 1e3, unit="groups/s",
                       ms_per_step=ms, higher_is_better=True, dtype="f64", gpu_launches=args.steps,
                       roofline={"bound": "hbm", "achieved": byt / ms / 1e6, "peak": hbm, "unit": "GB/s",
-                                "frac": byt / ms / 1e6 / hbm, "traffic": None, "kernel": "absmax_kernel",
+                                "frac": byt / ms / 1e6 / hbm, "traffic": recorded_kernel_traffic("absmax_kernel", G),
+                                "kernel": "absmax_kernel",
                                 "bytes_per_group": 322, "peak_note": hsrc}))
 
     s_pool = torch.empty(G, dtype=torch.int16, device=dev)
@@ -319,8 +340,9 @@ def bench_policies(args, wl, W, D, Wd, Dd, dev):
                       unit="groups/s", ms_per_step=ms, higher_is_better=True, dtype="f64",
                       gpu_launches=2 * args.steps,
                       roofline={"bound": "hbm", "achieved": byt / ms / 1e6, "peak": hbm, "unit": "GB/s",
-                                "frac": byt / ms / 1e6 / hbm, "traffic": None,
-                                "kernel": "objective_kernel + env_max_kernel", "bytes_per_group": bpg,
+                                "frac": byt / ms / 1e6 / hbm,
+                                "traffic": recorded_kernel_traffic("objective_kernel<4,", G),
+                                "kernel": "objective_kernel<4, per-column>", "bytes_per_group": bpg,
                                 "peak_note": hsrc}))
 
     Wp, Dp, offsets = synth.make_proxy_inputs()
@@ -368,7 +390,8 @@ def bench_gptq(args, wl, dev):
     lines.append(dict(base, metric="GPTQ v1 export groups/sec", op="gptq_export", value=G / ms * 1e3,
                       ms_per_step=ms, gpu_launches=3 * args.steps,
                       roofline={"bound": "hbm", "achieved": G * bpg / ms / 1e6, "peak": hbm, "unit": "GB/s",
-                                "frac": G * bpg / ms / 1e6 / hbm, "traffic": None,
+                                "frac": G * bpg / ms / 1e6 / hbm,
+                                "traffic": recorded_kernel_traffic("transpose_kernel<uint32_t>", G),
                                 "kernel": "transpose_kernel<uint32_t> (+ scales transpose, fills)",
                                 "bytes_per_group": bpg, "peak_note": hsrc}))
     for half in (True, False):
@@ -382,7 +405,9 @@ def bench_gptq(args, wl, dev):
                           op="gptq_dequant_fp16" if half else "gptq_dequant_fp32", value=G / ms * 1e3,
                           ms_per_step=ms, gpu_launches=args.steps, dtype="f16" if half else "f32",
                           roofline={"bound": "hbm", "achieved": G * bpg / ms / 1e6, "peak": hbm, "unit": "GB/s",
-                                    "frac": G * bpg / ms / 1e6 / hbm, "traffic": None,
+                                    "frac": G * bpg / ms / 1e6 / hbm,
+                                    "traffic": recorded_kernel_traffic(
+                                        f"dequant_kernel<{'fp16' if half else 'fp32'}>", G),
                                     "kernel": f"dequant_kernel<{'true' if half else 'false'}>",
                                     "bytes_per_group": bpg, "peak_note": hsrc}))
         del out
@@ -417,7 +442,8 @@ def bench_diag(args, wl, dev):
             "config": {"workload": f"diag-{E}x{N}x{K}-bf16", "environments": E, "tokens_per_env": N, "K": K,
                        "l2": "inputs (2.1 GB) larger than the 126 MB L2; no flush"},
             "roofline": {"bound": "hbm", "achieved": byt / ms / 1e6, "peak": hbm, "unit": "GB/s",
-                         "frac": byt / ms / 1e6 / hbm, "traffic": None,
+                         "frac": byt / ms / 1e6 / hbm,
+                         "traffic": recorded_kernel_traffic("column_squares_kernel<bf16>", E * N),
                          "kernel": "column_squares_kernel<bf16> + normalise_kernel",
                          "bytes_per_token": K * 2, "peak_note": hsrc}}
     print(json.dumps(line), flush=True)

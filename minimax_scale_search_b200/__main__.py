@@ -1,11 +1,15 @@
-"""Command-line runner: select scales for one synthetic workload on the GPU.
+"""Command-line runner for synthetic workloads on the GPU.
 
     python -m minimax_scale_search_b200 --workload 2 [--rows R] [--repeat N]
-        [--matrix M] [--check N] [--force-exhaustive]
+        [--matrix M] [--force-exhaustive]
+    python -m minimax_scale_search_b200 --ops
 
-Prints one JSON line with the device time per call (CUDA events), groups/s and
-the kernel counters.  --check N compares N sampled groups with the exhaustive
-CPU oracle (test infrastructure; needs the oracle's C library).
+The first form selects scales for one synthetic workload and prints one JSON
+line with the device time per call (CUDA events), groups/s and the kernel
+counters.  --ops runs each of the other kernels once (AbsMax, objective of
+given scales, GPTQ export and dequantisation, diagonal estimation, the
+three-policy reconstruction proxy) on inputs larger than L2 and prints their
+device times.
 """
 from __future__ import annotations
 
@@ -16,15 +20,56 @@ import time
 import numpy as np
 
 
+def timed(fn):
+    import torch
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    out = fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return out, round(e0.elapsed_time(e1), 3)
+
+
+def run_ops():
+    """Each secondary kernel once: the first 4,096 sweep rows (524,288 groups,
+    134 MB of W), 4 x 8,192 bf16 activation rows of 16,384 columns (1.07 GB),
+    and the 4,096-group proxy input."""
+    import torch
+
+    from minimax_scale_search_b200 import cq, synth
+    W = synth.make_weights(3, 0, 4096)
+    D = synth.make_diagonals(3)
+    Wd = torch.from_numpy(W.view(np.int16)).cuda()
+    Dd = torch.from_numpy(D).cuda()
+    ms = {}
+    (s_abs, c_abs), ms["absmax"] = timed(lambda: cq.absmax_scales(Wd))
+    _, ms["objective"] = timed(lambda: cq.group_objective(Wd, Dd, s_abs, 16384))
+    t, ms["gptq_export"] = timed(lambda: cq.gptq_export(s_abs, c_abs, 4096, 16384))
+    _, ms["gptq_dequant_fp16"] = timed(lambda: cq.gptq_dequantize(t, half=True))
+    _, ms["gptq_dequant_fp32"] = timed(lambda: cq.gptq_dequantize(t))
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    X = torch.randn((4 * 8192, 16384), generator=g, device="cuda").to(torch.bfloat16)
+    _, ms["diagonals"] = timed(lambda: cq.estimate_diagonals(X, np.arange(5, dtype=np.int64) * 8192))
+    Wp, Dp, off = synth.make_proxy_inputs()
+    res, ms["proxy_three_policies"] = timed(lambda: cq.evaluate_policies(
+        torch.from_numpy(Wp.view(np.int16)).cuda(), torch.from_numpy(Dp).cuda(), off))
+    print(json.dumps({"groups": int(W.size // 128), "ms": ms, "proxy": {k: v[0] for k, v in res.items()}}),
+          flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(prog="python -m minimax_scale_search_b200")
     ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--rows", type=int, default=0, help="only the first R rows of the matrix")
     ap.add_argument("--matrix", type=int, default=0)
     ap.add_argument("--repeat", type=int, default=3)
-    ap.add_argument("--check", type=int, default=0)
     ap.add_argument("--force-exhaustive", action="store_true")
+    ap.add_argument("--ops", action="store_true", help="run each of the other kernels once")
     a = ap.parse_args()
+    if a.ops:
+        run_ops()
+        return
 
     import torch
 
@@ -43,28 +88,10 @@ def main():
     times = []
     res = None
     for _ in range(a.repeat):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        res = cq.select_scales(Wd, Dd, wl.cols, workspace=ws, force_exhaustive=a.force_exhaustive,
-                               want_objective=a.check > 0)
-        e1.record()
-        torch.cuda.synchronize()
-        times.append(e0.elapsed_time(e1))
+        res, t = timed(lambda: cq.select_scales(Wd, Dd, wl.cols, workspace=ws, force_exhaustive=a.force_exhaustive))
+        times.append(t)
     out = {"workload": wl.name, "rows": rows, "groups": G, "E": wl.E, "gen_s": round(gen_s, 2),
-           "ms": [round(t, 3) for t in times], "groups_per_s": G / (min(times) / 1e3),
-           "counters": res.counters()}
-    if a.check:
-        import oracle
-        scales, codes = cq.to_numpy_bits(res)
-        sel = synth.sample_groups(a.workload, min(a.check, G), seed=3)
-        sel = sel[sel < G]
-        Wg = W.reshape(-1, 128)
-        o = oracle.solve(Wg, D, K=wl.cols, sel=sel)
-        strict = (o["best_obj"] == 0) | (np.abs(o["runner_obj"] - o["best_obj"]) >
-                                         1e-12 * np.maximum(np.abs(o["best_obj"]), np.abs(o["runner_obj"])))
-        same = scales[sel] == o["best_bits"]
-        out["check"] = {"groups": int(len(sel)), "strict": int(strict.sum()),
-                        "strict_mismatch": int((strict & ~same).sum())}
+           "ms": times, "groups_per_s": G / (min(times) / 1e3), "counters": res.counters()}
     print(json.dumps(out), flush=True)
 
 
