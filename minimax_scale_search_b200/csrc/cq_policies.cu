@@ -51,14 +51,20 @@ __device__ __forceinline__ void stage_rows(uint8_t *sm, const uint16_t *__restri
 
 // min(round-half-even(aw / s), cap) for aw >= 0, exact.  The estimate
 // aw * (1/s) is within one of the answer; adding 1.5 * 2^23 rounds it to the
-// nearest integer (ties even) in the low mantissa bits, and the exact
-// threshold tests s (n -+ 1/2) (11-bit s times a 5-bit factor) correct it.
+// nearest integer (ties even) in the low mantissa bits.  Near a half-integer
+// the exact threshold tests s (n -+ 1/2) (11-bit s times a 5-bit factor)
+// decide instead.
 __device__ __forceinline__ int code_of(float aw, float s, float inv, int cap)
 {
     constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-    const float y = fminf(aw * inv, 15.0f) + kRound;
+    const float x = fminf(aw * inv, 15.0f);
+    const float y = x + kRound;
     const float n = y - kRound;
     const int ni = __float_as_int(y) - 0x4B400000;
+    // x is within 15 * 2^-23 of aw / s, so away from a half-integer its own
+    // rounding is the exact one (x - n is exact)
+    if (fabsf(fabsf(x - n) - 0.5f) > 0x1p-12f)
+        return min(ni, cap);
     const float lo = s * (n - 0.5f), hi = s * (n + 0.5f);
     const bool odd = ni & 1;
     const int below = (aw < lo || (aw == lo && odd)) ? 1 : 0;  // rne < n

@@ -58,14 +58,20 @@ struct SpecParams {
 };
 
 // min(round-half-even(aw / s), cap) for aw >= 0, exact (cap <= 128): an
-// estimate from 1/s, rounded by adding 1.5 * 2^23, corrected by the exact
-// thresholds s (m -+ 1/2) (an 11-bit scale times a factor of at most 9 bits).
+// estimate from 1/s, rounded by adding 1.5 * 2^23; near a half-integer the
+// exact thresholds s (m -+ 1/2) (an 11-bit scale times a factor of at most 9
+// bits) decide instead.
 __device__ __forceinline__ int spec_code(float aw, float s, float inv, int cap)
 {
     constexpr float kRound = 12582912.0f;
-    const float y = fminf(aw * inv, static_cast<float>(cap + 1)) + kRound;
+    const float x = fminf(aw * inv, static_cast<float>(cap + 1));
+    const float y = x + kRound;
     const float m = y - kRound;
     const int mi = __float_as_int(y) - 0x4B400000;
+    // x is within 129 * 2^-23 < 2^-15 of aw / s, so away from a half-integer
+    // its own rounding is the exact one (x - m is exact)
+    if (fabsf(fabsf(x - m) - 0.5f) > 0x1p-12f)
+        return min(mi, cap);
     const float lo = s * (m - 0.5f), hi = s * (m + 0.5f);
     const bool odd = mi & 1;
     const int below = (aw < lo || (aw == lo && odd)) ? 1 : 0;
