@@ -2,11 +2,13 @@
 
     python -m minimax_scale_search_b200 --workload 2 [--rows R] [--repeat N]
         [--matrix M] [--force-exhaustive]
+    python -m minimax_scale_search_b200 --workload 3 --rows 1024 --qmin -4 --qmax 3 [--group-size 128]
     python -m minimax_scale_search_b200 --ops
 
 The first form selects scales for one synthetic workload and prints one JSON
 line with the device time per call (CUDA events), groups/s and the kernel
-counters.  --ops runs each of the other kernels once (AbsMax, objective of
+counters; with --qmin/--qmax/--group-size it runs the general-spec path
+instead.  --ops runs each of the other kernels once (AbsMax, objective of
 given scales, GPTQ export and dequantisation, diagonal estimation, the
 three-policy reconstruction proxy) on inputs larger than L2 and prints their
 device times.
@@ -66,6 +68,9 @@ def main():
     ap.add_argument("--repeat", type=int, default=3)
     ap.add_argument("--force-exhaustive", action="store_true")
     ap.add_argument("--ops", action="store_true", help="run each of the other kernels once")
+    ap.add_argument("--qmin", type=int, default=None, help="general spec: smallest code")
+    ap.add_argument("--qmax", type=int, default=None, help="general spec: largest code")
+    ap.add_argument("--group-size", type=int, default=128, help="general spec: weights per group")
     a = ap.parse_args()
     if a.ops:
         run_ops()
@@ -83,6 +88,18 @@ def main():
     gen_s = time.perf_counter() - t0
     Wd = torch.from_numpy(W.view(np.int16)).cuda()
     Dd = torch.from_numpy(D).cuda()
+    if a.qmin is not None or a.qmax is not None:
+        qmin = -8 if a.qmin is None else a.qmin
+        qmax = 7 if a.qmax is None else a.qmax
+        n = a.group_size
+        times = []
+        for _ in range(a.repeat):
+            _, t = timed(lambda: cq.select_scales_spec(Wd, Dd, wl.cols, qmin=qmin, qmax=qmax, group_size=n))
+            times.append(t)
+        G = W.size // n
+        print(json.dumps({"workload": wl.name, "rows": rows, "groups": G, "E": wl.E, "qmin": qmin, "qmax": qmax,
+                          "group_size": n, "ms": times, "groups_per_s": G / (min(times) / 1e3)}), flush=True)
+        return
     G = W.size // 128
     ws = torch.empty(cq.workspace_bytes(G, wl.E), dtype=torch.uint8, device="cuda")
     times = []
