@@ -7,10 +7,11 @@
 // in cq_select.cu is specialised to (-8, 7) and 128 weights; this path serves
 // every other spec with the same result definition.
 //
-// One CTA per group (grid-stride over groups):
+// One warp per group (a grid of one-warp CTAs, grid-stride over groups; many
+// groups in flight per SM hide the latency of each group's serial steps):
 //  1. stage w (exact fp32 and fp64) and the group's diagonals (fp64);
-//  2. U = the smallest objective, computed exactly as the definition does,
-//     at the AbsMax-type scales fp16(max|w|/qmax), fp16(max|w|/|qmin|), their
+//  2. U: an upper bound of the smallest objective, from warp-parallel sums at
+//     the AbsMax-type scales fp16(max|w|/qmax), fp16(max|w|/|qmin|), their
 //     grid neighbours and the first scale at which every code is 0;
 //  3. a certified window [J0, J1]: below a scale, the clipped weights' error
 //     sum_e-max of sum d (|w| - c s)^2 only grows as s falls; above one, the
@@ -18,12 +19,14 @@
 //     Both are fp64 lower bounds of the exact objective, taken with a 2^-40
 //     margin that covers the rounding of either side (n <= 4096), so a scale
 //     they exclude has an objective above U and cannot be the minimum or tie it;
-//  4. every scale of the window, one thread per scale, evaluated in the
+//  4. the window in chunks of 32 scales, each with an interval lower bound
+//     (one lane per chunk); chunks whose bound exceeds U are skipped;
+//  5. every scale of the kept chunks, one lane per scale, evaluated in the
 //     definition's own order (i ascending, r = w - s q exact, r*r, d*rr and the
 //     running sum rounded separately, environments maxed in order), so each
 //     value equals the oracle's bit for bit; above the first all-zero scale j_z
 //     every scale has the same value, so only j_z is evaluated there;
-//  5. the (objective, pattern) minimum and its codes.
+//  6. the (objective, pattern) minimum and its codes.
 
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -37,12 +40,10 @@
 namespace cq {
 namespace {
 
-constexpr int kSpecThreads = 256;
-constexpr int kSpecWarps = kSpecThreads / 32;
 constexpr int kCandidates = 7;
-constexpr uint32_t kChunk = 32;                               // scales per interval bound
-constexpr int kMaxChunks = (static_cast<int>(kLast) + 31) / 32;  // 992
-constexpr float kKeepChunk = 1.0f - 0x1p-12f;                  // covers the fp32 rounding of a bound
+constexpr uint32_t kChunk = 32;                                     // scales per interval bound (one per lane)
+constexpr int kMaxChunkWords = ((static_cast<int>(kLast) + 31) / 32 + 31) / 32;  // 31 words of chunk flags
+constexpr float kKeepChunk = 1.0f - 0x1p-12f;                        // covers the fp32 rounding of a bound
 
 struct SpecParams {
     const uint16_t *W;
@@ -125,8 +126,8 @@ __device__ double objective_at(const Smem &sm, int n, int qmin, int qmax, uint32
     return f;
 }
 
-// Block-wide (min objective, lowest pattern); every thread gets the result.
-__device__ void block_best(double &f, uint32_t &j, double *red_f, uint32_t *red_j)
+// Warp-wide (min objective, lowest pattern); every lane gets the result.
+__device__ __forceinline__ void warp_best(double &f, uint32_t &j)
 {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -137,70 +138,22 @@ __device__ void block_best(double &f, uint32_t &j, double *red_f, uint32_t *red_
             j = oj;
         }
     }
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    __syncthreads();
-    if (lane == 0) {
-        red_f[wid] = f;
-        red_j[wid] = j;
-    }
-    __syncthreads();
-    f = red_f[0];
-    j = red_j[0];
-    for (int w = 1; w < kSpecWarps; w++)
-        if (red_f[w] < f || (red_f[w] == f && red_j[w] < j)) {
-            f = red_f[w];
-            j = red_j[w];
-        }
 }
 
-// Block-wide sums of E per-thread values, every thread getting the totals.
-// The scratch alternates between two halves; each thread keeps the parity in
-// a register (every thread makes the same calls).  One barrier per call keeps
-// a call's writes from overtaking the previous call's reads: a thread writes a
-// half again only after the next call's barrier, which every thread reaches
-// after its reads.
-struct BlockScratch {
-    double (*v)[kSpecWarps][CQ_MAX_E];  // two halves in shared memory
-    int half;                           // this thread's parity
-};
-
+// Max over environments of a per-environment sum of per-weight terms, the
+// lanes taking weights lane, lane + 32, ... (any order: a bound, used with a
+// margin).  kind 0: clipped weights' error at s; kind 1: error of the weights
+// that quantise to 0 at s.  Every lane gets the result.
 template <int E>
-__device__ void block_sum_env(double (&acc)[CQ_MAX_E], BlockScratch &bs)
-{
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    double(*buf)[CQ_MAX_E] = bs.v[bs.half];
-    bs.half ^= 1;
-#pragma unroll
-    for (int e = 0; e < CQ_MAX_E; e++)
-        if (e < E) {
-            const double v = warp_sum(acc[e]);
-            if (lane == 0)
-                buf[wid][e] = v;
-        }
-    __syncthreads();
-#pragma unroll
-    for (int e = 0; e < CQ_MAX_E; e++)
-        if (e < E) {
-            double v = 0.0;
-            for (int w = 0; w < kSpecWarps; w++)
-                v += buf[w][e];
-            acc[e] = v;
-        }
-}
-
-// Block-wide max over environments of a per-environment sum of per-weight
-// terms (any order: a bound, used with a margin).  kind 0: clipped weights'
-// error at s; kind 1: error of the weights that quantise to 0 at s.
-template <int E>
-__device__ double bound_at(const Smem &sm, int n, int qmin, int qmax, uint32_t j, int kind, BlockScratch &bs)
+__device__ double bound_at(const Smem &sm, int n, int qmin, int qmax, uint32_t j, int kind)
 {
     const float s = grid_value(j);
     const double sd = s;
-    double acc[CQ_MAX_E];
+    double acc[E];
 #pragma unroll
-    for (int e = 0; e < CQ_MAX_E; e++)
+    for (int e = 0; e < E; e++)
         acc[e] = 0.0;
-    for (int i = threadIdx.x; i < n; i += kSpecThreads) {
+    for (int i = threadIdx.x & 31; i < n; i += 32) {
         const float w = sm.wf[i];
         const float aw = fabsf(w);
         double t = 0.0;
@@ -214,50 +167,44 @@ __device__ double bound_at(const Smem &sm, int n, int qmin, int qmax, uint32_t j
             t = sm.wd[i] * sm.wd[i];
         }
 #pragma unroll
-        for (int e = 0; e < CQ_MAX_E; e++)
-            if (e < E)
-                acc[e] += sm.dd[e * n + i] * t;
+        for (int e = 0; e < E; e++)
+            acc[e] += sm.dd[e * n + i] * t;
     }
-    block_sum_env<E>(acc, bs);
     double best = 0.0;
 #pragma unroll
-    for (int e = 0; e < CQ_MAX_E; e++)
-        if (e < E)
-            best = fmax(best, acc[e]);
+    for (int e = 0; e < E; e++)
+        best = fmax(best, warp_sum(acc[e]));
     return best;
 }
 
-// An upper bound of the objective at grid index j that the whole block sums in
-// any order: the exact value's fp64 sums err by at most n 2^-53 relative either
-// way, so the block sum times (1 + 2^-40) is at least the definition's own
-// value for n <= 4096.
+// An upper bound of the objective at grid index j that the warp sums in any
+// order: the exact value's fp64 sums err by at most n 2^-53 relative either
+// way, so the warp sum times (1 + 2^-40) is at least the definition's own
+// value for n <= 4096.  Every lane gets the result.
 template <int E>
-__device__ double upper_at(const Smem &sm, int n, int qmin, int qmax, uint32_t j, BlockScratch &bs)
+__device__ double upper_at(const Smem &sm, int n, int qmin, int qmax, uint32_t j)
 {
     const float s = grid_value(j);
     const float inv = 1.0f / s;
     const double nsd = -static_cast<double>(s);
-    double acc[CQ_MAX_E];
+    double acc[E];
 #pragma unroll
-    for (int e = 0; e < CQ_MAX_E; e++)
+    for (int e = 0; e < E; e++)
         acc[e] = 0.0;
-    for (int i = threadIdx.x; i < n; i += kSpecThreads) {
+    for (int i = threadIdx.x & 31; i < n; i += 32) {
         const float w = sm.wf[i];
         const bool neg = w < 0.0f;
         const int c = spec_code(fabsf(w), s, inv, neg ? -qmin : qmax);
         const double r = fma(nsd, static_cast<double>(neg ? -c : c), sm.wd[i]);
         const double rr = r * r;
 #pragma unroll
-        for (int e = 0; e < CQ_MAX_E; e++)
-            if (e < E)
-                acc[e] = fma(sm.dd[e * n + i], rr, acc[e]);
+        for (int e = 0; e < E; e++)
+            acc[e] = fma(sm.dd[e * n + i], rr, acc[e]);
     }
-    block_sum_env<E>(acc, bs);
     double f = 0.0;
 #pragma unroll
-    for (int e = 0; e < CQ_MAX_E; e++)
-        if (e < E)
-            f = fmax(f, acc[e]);
+    for (int e = 0; e < E; e++)
+        f = fmax(f, warp_sum(acc[e]));
     return f * (1.0 + 0x1p-40);
 }
 
@@ -303,19 +250,12 @@ __device__ float chunk_bound(const Smem &sm, int n, int qmin, int qmax, float s_
 }
 
 template <int E>
-__global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
+__global__ void __launch_bounds__(32) spec_kernel(SpecParams p)
 {
     extern __shared__ __align__(16) unsigned char dyn[];
-    __shared__ double red_f[kSpecWarps];
-    __shared__ uint32_t red_j[kSpecWarps];
-    __shared__ double scratch[2][kSpecWarps][CQ_MAX_E];
-    __shared__ bool keep[kMaxChunks];
-    __shared__ uint16_t kept[kMaxChunks];
-    __shared__ int nkept;
-    BlockScratch bs{scratch, 0};
-    __shared__ int flag_bad;
-    __shared__ float amax_s;
+    __shared__ uint32_t keepw[kMaxChunkWords];
     const int n = p.n;
+    const int lane = threadIdx.x & 31;
     Smem sm;
     sm.dd = reinterpret_cast<double *>(dyn);
     sm.wd = sm.dd + static_cast<size_t>(E) * n;
@@ -323,61 +263,51 @@ __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
     const int64_t gpr = p.K > 0 ? p.K / n : 1;
     constexpr double kKeep = 1.0 - 0x1p-40;
     for (int64_t g = blockIdx.x; g < p.G; g += gridDim.x) {
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            flag_bad = 0;
-            amax_s = 0.0f;
-        }
-        __syncthreads();
+        __syncwarp();
         // 1. stage
         float am = 0.0f;
-        int bad = 0;
-        for (int i = threadIdx.x; i < n; i += kSpecThreads) {
+        bool bad = false;
+        for (int i = lane; i < n; i += 32) {
             const uint32_t b = p.W[g * n + i];
             bad |= (b & 0x7FFFu) >= kBeyond;
             const float w = half_value(b);
             sm.wf[i] = w;
             sm.wd[i] = w;
             am = fmaxf(am, fabsf(w));
+#pragma unroll
             for (int e = 0; e < E; e++) {
                 const float d = p.K > 0 ? p.D[e * p.K + (g % gpr) * n + i] : p.D[(e * p.G + g) * n + i];
                 bad |= !(d >= 0.0f && d <= FLT_MAX);
                 sm.dd[e * n + i] = d;
             }
         }
-        if (bad)
-            atomicOr(&flag_bad, 1);
-        am = fmaxf(am, __shfl_xor_sync(kFull, am, 16));
-        am = fmaxf(am, __shfl_xor_sync(kFull, am, 8));
-        am = fmaxf(am, __shfl_xor_sync(kFull, am, 4));
-        am = fmaxf(am, __shfl_xor_sync(kFull, am, 2));
-        am = fmaxf(am, __shfl_xor_sync(kFull, am, 1));
-        if ((threadIdx.x & 31) == 0 && am > 0.0f)
-            atomicMax(reinterpret_cast<int *>(&amax_s), __float_as_int(am));  // non-negative floats order as ints
-        __syncthreads();
-        const float amax = amax_s;
-        if (flag_bad || amax == 0.0f) {
-            for (int i = threadIdx.x; i < n; i += kSpecThreads)
+        bad = __any_sync(kFull, bad);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            am = fmaxf(am, __shfl_xor_sync(kFull, am, o));
+        const float amax = am;
+        __syncwarp();
+        if (bad || amax == 0.0f) {
+            for (int i = lane; i < n; i += 32)
                 p.out_codes[g * n + i] = 0;
-            if (threadIdx.x == 0) {
+            if (lane == 0) {
                 p.out_scales[g] = 0x0001;
                 if (p.out_obj)
                     p.out_obj[g] = 0.0;
                 if (p.out_flags)
-                    p.out_flags[g] = flag_bad ? CQ_FLAG_NONFINITE : CQ_FLAG_TRIVIAL;
+                    p.out_flags[g] = bad ? CQ_FLAG_NONFINITE : CQ_FLAG_TRIVIAL;
             }
             continue;
         }
-        // 2. upper bound from exact objectives at a few scales
+        // 2. upper bound U.  Every lane evaluates the same candidates, so U and
+        // jb are uniform; jb lies in the window found below (its bounds are
+        // below U there) and not above j_z, so the scan evaluates it exactly.
         uint32_t jz = kLast + 1;  // first scale where every code is 0 (s >= 2 max|w|)
         {
             const float two = 2.0f * amax;  // exact
             if (two <= 65504.0f)
                 jz = max(static_cast<uint32_t>(__half_as_ushort(__float2half_ru(two))), 1u);
         }
-        // Every thread evaluates the same candidates, so U and jb are uniform.
-        // jb lies in the window found below (its bounds are below U there) and
-        // below j_z, so the scan evaluates it exactly.
         double U = INFINITY;
         uint32_t jb = 1;
         for (int t = 0; t < kCandidates; t++) {
@@ -392,7 +322,7 @@ __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
             }
             if (j > kLast)
                 continue;
-            const double u = upper_at<E>(sm, n, p.qmin, p.qmax, j, bs);
+            const double u = upper_at<E>(sm, n, p.qmin, p.qmax, j);
             if (u < U) {
                 U = u;
                 jb = j;
@@ -400,10 +330,10 @@ __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
         }
         // 3. certified window [J0, J1]
         uint32_t lo = 1, hi = jb;  // smallest index whose clipping bound does not exclude it
-        if (bound_at<E>(sm, n, p.qmin, p.qmax, 1, 0, bs) * kKeep > U) {
+        if (bound_at<E>(sm, n, p.qmin, p.qmax, 1, 0) * kKeep > U) {
             while (hi - lo > 1) {  // invariant: lo excluded, hi not
                 const uint32_t mid = (lo + hi) / 2;
-                if (bound_at<E>(sm, n, p.qmin, p.qmax, mid, 0, bs) * kKeep > U)
+                if (bound_at<E>(sm, n, p.qmin, p.qmax, mid, 0) * kKeep > U)
                     lo = mid;
                 else
                     hi = mid;
@@ -413,10 +343,10 @@ __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
         const uint32_t J0 = lo;
         lo = jb;
         hi = kLast;
-        if (bound_at<E>(sm, n, p.qmin, p.qmax, kLast, 1, bs) * kKeep > U) {
+        if (bound_at<E>(sm, n, p.qmin, p.qmax, kLast, 1) * kKeep > U) {
             while (hi - lo > 1) {  // invariant: lo not excluded, hi excluded
                 const uint32_t mid = (lo + hi) / 2;
-                if (bound_at<E>(sm, n, p.qmin, p.qmax, mid, 1, bs) * kKeep > U)
+                if (bound_at<E>(sm, n, p.qmin, p.qmax, mid, 1) * kKeep > U)
                     hi = mid;
                 else
                     lo = mid;
@@ -424,53 +354,52 @@ __global__ void __launch_bounds__(kSpecThreads) spec_kernel(SpecParams p)
             hi = lo;
         }
         const uint32_t J1 = min(hi, jz);
-        // 4. chunks of kChunk scales whose interval bound exceeds U are skipped
+        // 4. chunks of 32 scales whose interval bound exceeds U are skipped; lane
+        // L bounds chunks L, L + 32, ...; bit c of the flag words marks chunk c kept
         const int nch = static_cast<int>((J1 - J0) / kChunk + 1);
-        for (int ch = threadIdx.x; ch < nch; ch += kSpecThreads) {
-            const uint32_t a = J0 + static_cast<uint32_t>(ch) * kChunk;
-            const uint32_t b = min(a + kChunk - 1, J1);
-            keep[ch] = chunk_bound<E>(sm, n, p.qmin, p.qmax, grid_value(a), grid_value(b)) * kKeepChunk <= U;
-        }
-        __syncthreads();
-        if (threadIdx.x < 32) {  // compact the kept chunks, ascending
-            int m = 0;
-            for (int c0 = 0; c0 < nch; c0 += 32) {
-                const int ch = c0 + static_cast<int>(threadIdx.x);
-                const bool k = ch < nch && keep[ch];
-                const unsigned bal = __ballot_sync(kFull, k);
-                if (k)
-                    kept[m + __popc(bal & ((1u << threadIdx.x) - 1u))] = static_cast<uint16_t>(ch);
-                m += __popc(bal);
+        for (int c0 = 0; c0 < nch; c0 += 32) {
+            const int ch = c0 + lane;
+            bool k = false;
+            if (ch < nch) {
+                const uint32_t a = J0 + static_cast<uint32_t>(ch) * kChunk;
+                const uint32_t b = min(a + kChunk - 1, J1);
+                k = chunk_bound<E>(sm, n, p.qmin, p.qmax, grid_value(a), grid_value(b)) * kKeepChunk <= U;
             }
-            if (threadIdx.x == 0)
-                nkept = m;
+            const unsigned bal = __ballot_sync(kFull, k);
+            if (lane == 0)
+                keepw[c0 >> 5] = bal;
         }
-        __syncthreads();
-        // 5. scan the kept scales
+        __syncwarp();
+        // 5. scan the kept chunks in ascending order, one scale per lane, so each
+        // lane meets its scales in ascending order and strict < keeps the lowest
         double bf = INFINITY;
         uint32_t bj = 0xFFFFFFFFu;
-        const int nscan = nkept * kChunk;
-        for (int u = threadIdx.x; u < nscan; u += kSpecThreads) {
-            const uint32_t j = J0 + static_cast<uint32_t>(kept[u / kChunk]) * kChunk + (u % kChunk);
-            if (j > J1)
-                break;  // only the last kept chunk can be short, and u grows with j
-            const double v = objective_at<E>(sm, n, p.qmin, p.qmax, j);
-            if (v < bf) {  // ascending j per thread: strict < keeps the lowest pattern
-                bf = v;
-                bj = j;
+        for (int wi = 0; wi < (nch + 31) / 32; wi++) {
+            uint32_t bits = keepw[wi];
+            while (bits) {
+                const int ch = 32 * wi + __ffs(bits) - 1;
+                bits &= bits - 1;
+                const uint32_t j = J0 + static_cast<uint32_t>(ch) * kChunk + static_cast<uint32_t>(lane);
+                if (j <= J1) {
+                    const double v = objective_at<E>(sm, n, p.qmin, p.qmax, j);
+                    if (v < bf) {
+                        bf = v;
+                        bj = j;
+                    }
+                }
             }
         }
-        block_best(bf, bj, red_f, red_j);
+        warp_best(bf, bj);
         // 6. outputs
         const float s = grid_value(bj);
         const float inv = 1.0f / s;
-        for (int i = threadIdx.x; i < n; i += kSpecThreads) {
+        for (int i = lane; i < n; i += 32) {
             const float w = sm.wf[i];
             const bool neg = w < 0.0f;
             const int c = spec_code(fabsf(w), s, inv, neg ? -p.qmin : p.qmax);
             p.out_codes[g * n + i] = static_cast<int8_t>(neg ? -c : c);
         }
-        if (threadIdx.x == 0) {
+        if (lane == 0) {
             p.out_scales[g] = static_cast<uint16_t>(bj);
             if (p.out_obj)
                 p.out_obj[g] = bf;
@@ -491,14 +420,14 @@ cudaError_t launch_spec(const SpecParams &p, cudaStream_t st)
                                     static_cast<int>(smem))) != cudaSuccess)
         return err;
     int per_sm = 1, dev = 0, sms = 148;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, spec_kernel<E>, kSpecThreads, smem) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, spec_kernel<E>, 32, smem) != cudaSuccess ||
         per_sm < 1)
         per_sm = 1;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t cap = static_cast<int64_t>(sms) * per_sm;
     const unsigned grid = static_cast<unsigned>(p.G < cap ? p.G : cap);
-    spec_kernel<E><<<grid, kSpecThreads, smem, st>>>(p);
+    spec_kernel<E><<<grid, 32, smem, st>>>(p);
     return cudaGetLastError();
 }
 
