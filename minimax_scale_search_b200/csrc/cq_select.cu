@@ -1633,12 +1633,12 @@ cq_status cq_select_scales_host(const uint16_t *W_host, int64_t G, const float *
     if (chunk > G)
         chunk = G;
     const int64_t nchunks = (G + chunk - 1) / chunk;
-    const int nslots = nchunks > 1 ? 2 : 1;
+    const int nslots = nchunks > 2 ? 3 : static_cast<int>(nchunks);  // three device slots in flight
 
-    cudaStream_t ss[2] = {nullptr, nullptr};
+    cudaStream_t ss[3] = {nullptr, nullptr, nullptr};
     cudaEvent_t ev_start = nullptr, ev_d = nullptr;
-    void *dW[2] = {nullptr, nullptr}, *dD[2] = {nullptr, nullptr}, *dS[2] = {nullptr, nullptr},
-         *dC[2] = {nullptr, nullptr}, *dWs[2] = {nullptr, nullptr};
+    void *dW[3] = {nullptr, nullptr, nullptr}, *dD[3] = {nullptr, nullptr, nullptr}, *dS[3] = {nullptr, nullptr, nullptr},
+         *dC[3] = {nullptr, nullptr, nullptr}, *dWs[3] = {nullptr, nullptr, nullptr};
     void *dDcol = nullptr;
     cudaError_t err = cudaSuccess;
     const size_t wsb = workspace_bytes(chunk);
@@ -1670,8 +1670,8 @@ cq_status cq_select_scales_host(const uint16_t *W_host, int64_t G, const float *
         CQ_TRY(pool_alloc(&dDcol, dcol_bytes, ss[0]));
         CQ_TRY(cudaMemcpyAsync(dDcol, D_host, dcol_bytes, cudaMemcpyHostToDevice, ss[0]));
         CQ_TRY(cudaEventRecord(ev_d, ss[0]));
-        if (nslots > 1)
-            CQ_TRY(cudaStreamWaitEvent(ss[1], ev_d, 0));
+        for (int k = 1; k < nslots; k++)
+            CQ_TRY(cudaStreamWaitEvent(ss[k], ev_d, 0));
     }
     for (int64_t c = 0; c < nchunks; c++) {
         const int k = static_cast<int>(c % nslots);
