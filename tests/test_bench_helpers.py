@@ -1,0 +1,47 @@
+"""The benchmark's accounting helpers, on hand-computed cases (CPU).
+
+The roofline fraction the benchmark reports rests on these: the counted FLOP
+convention (per non-trivial group, (T + 1) runs of FLOP_run(E) fp32 flops with
+T = qmax #(w > 0) + |qmin| #(w < 0), plus 2 n E 5 fp64 rescoring flops), the
+peaks from unit counts and the clock, and the whole-job rate."""
+import os
+import sys
+
+import numpy as np
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+import bench  # noqa: E402
+
+
+def f16bits(x):
+    return np.asarray(x, dtype=np.float64).astype(np.float16).view(np.uint16)
+
+
+def test_flop_run_values():
+    # 4E + E + 12 E(E-1)/2 + (E^2 + 4)(5E - 1)
+    assert bench.flop_run(1) == 4 + 1 + 0 + 5 * 4
+    assert bench.flop_run(4) == 472
+    assert bench.flop_run(8) == 3028
+
+
+def test_counted_flops_hand_example():
+    W = np.zeros((3, 128), dtype=np.uint16)
+    W[0, 5] = f16bits([0.5])[0]          # one positive weight: T = 7
+    W[0, 9] = f16bits([-0.25])[0]        # one negative weight: T += 8
+    W[1, :] = f16bits(np.full(128, 0.1))  # 128 positive: T = 896
+    W[2, 7] = 0x8000                      # -0 only: a trivial group, not counted
+    f32, f64 = bench.counted_flops(W, 4)
+    assert f32 == (15 + 1) * 472 + (896 + 1) * 472
+    assert f64 == 2 * 2 * 128 * 4 * 5
+    # a general spec counts its own transitions and group size
+    f32s, f64s = bench.counted_flops(W[:2, :64], 4, qmin=-4, qmax=3)
+    assert f32s == (3 + 4 + 1) * 472 + (3 * 64 + 1) * 472
+    assert f64s == 2 * 2 * 64 * 4 * 5
+
+
+def test_peaks_and_job_rate():
+    p32, p64, mhz, _ = bench.peaks()
+    assert abs(p32 - 148 * 128 * 2 * mhz * 1e6 / 1e12) < 1e-9
+    assert abs(p64 - p32 / 2) < 1e-9
+    # whole-job rate: all ranks' units over the slowest rank's time
+    assert bench.job_rate(8, 1000, 0.5) == 16000.0
