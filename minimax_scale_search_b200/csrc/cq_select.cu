@@ -1627,18 +1627,23 @@ cq_status cq_select_scales_host(const uint16_t *W_host, int64_t G, const float *
         return st;
     cudaStream_t user = static_cast<cudaStream_t>(stream);
     const int64_t gpr = K > 0 ? K / kGroup : 1;
-    int64_t chunk = (static_cast<int64_t>(1) << 19) / gpr * gpr;
+    // Chunks of 2^16 groups through six slots, one stream each.  A slot's
+    // short fallback kernel queues behind the persistent main kernels of the
+    // other slots, which holds back that slot's copy-out and its next copy-in;
+    // with three slots that left the SMs idle between rounds of chunks, with
+    // four or more the copies stay ahead of the kernels.
+    constexpr int kSlots = 6;
+    int64_t chunk = (static_cast<int64_t>(1) << 16) / gpr * gpr;
     if (chunk < gpr)
         chunk = gpr;
     if (chunk > G)
         chunk = G;
     const int64_t nchunks = (G + chunk - 1) / chunk;
-    const int nslots = nchunks > 2 ? 3 : static_cast<int>(nchunks);  // three device slots in flight
+    const int nslots = nchunks > kSlots ? kSlots : static_cast<int>(nchunks);
 
-    cudaStream_t ss[3] = {nullptr, nullptr, nullptr};
+    cudaStream_t ss[kSlots] = {};
     cudaEvent_t ev_start = nullptr, ev_d = nullptr;
-    void *dW[3] = {nullptr, nullptr, nullptr}, *dD[3] = {nullptr, nullptr, nullptr}, *dS[3] = {nullptr, nullptr, nullptr},
-         *dC[3] = {nullptr, nullptr, nullptr}, *dWs[3] = {nullptr, nullptr, nullptr};
+    void *dW[kSlots] = {}, *dD[kSlots] = {}, *dS[kSlots] = {}, *dC[kSlots] = {}, *dWs[kSlots] = {};
     void *dDcol = nullptr;
     cudaError_t err = cudaSuccess;
     const size_t wsb = workspace_bytes(chunk);

@@ -212,8 +212,8 @@ def test_entry_points_agree_and_empty_input():
 
 
 def test_host_entry_point_chunks_large_input():
-    """More groups than one host-path chunk (2^19), so the copy/compute pipeline
-    runs over several chunks and both buffer slots."""
+    """Many more groups than one host-path chunk (2^16), so the copy/compute
+    pipeline runs over 20 chunks and reuses each of its six slots."""
     from minimax_scale_search_b200 import cq
     rows = 10240  # 1.31M groups over 16384-wide rows
     W = synth.make_weights(3, 0, rows)
@@ -221,3 +221,26 @@ def test_host_entry_point_chunks_large_input():
     hs, hc = cq.select_scales_host(W, D)
     ex = P.run_gpu(W, D)
     assert np.array_equal(hs, ex["scales"]) and np.array_equal(hc, ex["codes"])
+
+
+def test_host_entry_point_ragged_chunks():
+    """Chunks rounded down to whole rows (3 groups per row: 65,535-group
+    chunks) with a ragged last chunk, and the per-group diagonal layout over
+    several chunks, against the device entry point."""
+    import torch
+    from minimax_scale_search_b200 import cq
+    rng = np.random.default_rng(77)
+    rows, K, E = 50_001, 384, 3
+    W = np.clip(rng.normal(0, 0.02, (rows, K)), -1, 1).astype(np.float16).view(np.uint16)
+    D = rng.lognormal(0, 1.0, (E, K)).astype(np.float32)
+    hs, hc = cq.select_scales_host(W, D)
+    ex = P.run_gpu(W, D, K)
+    assert np.array_equal(hs, ex["scales"]) and np.array_equal(hc, ex["codes"])
+    G = 140_000  # two full 2^16 chunks and a ragged 8,928-group one
+    Wg = np.ascontiguousarray(W.reshape(-1, 128)[:G])
+    Dg = rng.lognormal(0, 1.0, (E, G, 128)).astype(np.float32)
+    hs2, hc2 = cq.select_scales_host(Wg, Dg)
+    r = cq.select_scales(torch.from_numpy(Wg.view(np.int16)).cuda(), torch.from_numpy(Dg).cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(hs2, r.scales.cpu().numpy().view(np.uint16))
+    assert np.array_equal(hc2, r.codes.cpu().numpy().view(np.uint32))
