@@ -553,7 +553,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     const DiagView dv_g = diag_view(p, g);
     const uint2 wv = *reinterpret_cast<const uint2 *>(p.W + g * kGroup + 4 * lane);
     const uint32_t wb[4] = {wv.x & 0xFFFFu, wv.x >> 16, wv.y & 0xFFFFu, wv.y >> 16};
-    bool bad = false, nonzero = false;
+    bool bad = false, nonzero = false, odd = false;
     double A[E];
 #pragma unroll
     for (int m = 0; m < 4; m++) {
@@ -568,6 +568,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
 #pragma unroll
         for (int m = 0; m < 4; m++) {
             bad |= !(dq[m] >= 0.0f && dq[m] <= FLT_MAX);
+            odd |= dq[m] != 0.0f && !(dq[m] >= 0x1p-64f && dq[m] <= 0x1p96f);
             const double wd = half_value(wb[m]);
             a += static_cast<double>(dq[m]) * (wd * wd);  // exact: 24-bit d times 22-bit w^2
         }
@@ -590,10 +591,23 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         return;
     }
     float Af[E];
+    double amx = 0.0;
 #pragma unroll
     for (int e = 0; e < E; e++) {
         A[e] = warp_sum(A[e]);
         Af[e] = static_cast<float>(A[e]);
+        amx = fmax(amx, A[e]);
+    }
+    // The fp32 steps below bound their error relative to the terms, which holds
+    // while no fp32 value overflows or leaves the normal range.  Every objective
+    // is at most max_e A_e (each residual is at most |w|), screened values stay
+    // within 16 max_e A_e, and B = sum d|w||q| and C = sum d q^2 within
+    // 2^26 max d; so with every nonzero d in [2^-64, 2^96] and max_e A_e <= 2^120
+    // every nonzero fp32 value lies in [2^-112, 2^124].  Other groups take the
+    // fp64 exhaustive pass.
+    if (__any_sync(kFull, odd) || amx > 0x1p120) {
+        enqueue(p, g, lane, tl);
+        return;
     }
 
     // ---- 2. order the weights by |w|; stage w and d by rank ----------------

@@ -19,14 +19,23 @@
 //     Both are fp64 lower bounds of the exact objective, taken with a 2^-40
 //     margin that covers the rounding of either side (n <= 4096), so a scale
 //     they exclude has an objective above U and cannot be the minimum or tie it;
-//  4. the window in chunks of 32 scales, each with an interval lower bound
-//     (one lane per chunk); chunks whose bound exceeds U are skipped;
-//  5. every scale of the kept chunks, one lane per scale, evaluated in the
-//     definition's own order (i ascending, r = w - s q exact, r*r, d*rr and the
-//     running sum rounded separately, environments maxed in order), so each
-//     value equals the oracle's bit for bit; above the first all-zero scale j_z
-//     every scale has the same value, so only j_z is evaluated there;
-//  6. the (objective, pattern) minimum and its codes.
+//  4. the window in at most 256 chunks of C >= 8 scales (C a power of two),
+//     each with an fp32 interval lower bound of the objective, one lane per
+//     chunk; chunks whose bound exceeds U are dropped;
+//  5. best first: the chunks with the smallest bounds, 32 scales at a time,
+//     have every scale evaluated in the definition's own order (i ascending,
+//     r = w - s q exact, r*r, d*rr and the running sum rounded separately,
+//     environments maxed in order), so each value equals the oracle's bit for
+//     bit; a chunk is dropped once its bound exceeds the best value found so
+//     far, which leaves every scale in it strictly worse.  Above the first
+//     all-zero scale j_z every scale has the same value, so only j_z is
+//     evaluated there;
+//  6. the (objective, pattern) minimum over the evaluated scales and its codes.
+//
+// The fp32 bounds assume no fp32 overflow or subnormal result: every term is
+// d dist^2 with dist 0 or in [2^-24, 65504], so they are used only when every
+// nonzero d lies in [2^-64, 2^80] (terms 0 or in [2^-112, 2^112], sums below
+// 2^122); otherwise every chunk's bound is 0 and the scan covers the window.
 
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -41,9 +50,10 @@ namespace cq {
 namespace {
 
 constexpr int kCandidates = 7;
-constexpr uint32_t kChunk = 32;                                     // scales per interval bound (one per lane)
-constexpr int kMaxChunkWords = ((static_cast<int>(kLast) + 31) / 32 + 31) / 32;  // 31 words of chunk flags
-constexpr float kKeepChunk = 1.0f - 0x1p-12f;                        // covers the fp32 rounding of a bound
+constexpr int kLaneChunks = 8;                 // chunk bounds held per lane: at most 256 chunks
+constexpr uint32_t kMinChunk = 8;              // smallest chunk, in scales
+constexpr float kKeepChunk = 1.0f - 0x1p-12f;  // covers the fp32 rounding of a bound
+constexpr float kTrustLo = 0x1p-64f, kTrustHi = 0x1p80f;  // d range for the fp32 bounds
 
 struct SpecParams {
     const uint16_t *W;
@@ -84,6 +94,7 @@ struct Smem {
     float *wf;   // [n] exact weights
     double *wd;  // [n]
     double *dd;  // [E][n]
+    float *df;   // [E][n] the same diagonals in fp32 (exact), for the chunk bounds
 };
 
 // Objective at grid index j, in the definition's order; one thread.
@@ -239,7 +250,7 @@ __device__ float chunk_bound(const Smem &sm, int n, int qmin, int qmax, float s_
 #pragma unroll
         for (int e = 0; e < CQ_MAX_E; e++)
             if (e < E)
-                acc[e] = fmaf(static_cast<float>(sm.dd[e * n + i]), d2, acc[e]);
+                acc[e] = fmaf(sm.df[e * n + i], d2, acc[e]);
     }
     float best = 0.0f;
 #pragma unroll
@@ -253,20 +264,20 @@ template <int E>
 __global__ void __launch_bounds__(32) spec_kernel(SpecParams p)
 {
     extern __shared__ __align__(16) unsigned char dyn[];
-    __shared__ uint32_t keepw[kMaxChunkWords];
     const int n = p.n;
     const int lane = threadIdx.x & 31;
     Smem sm;
     sm.dd = reinterpret_cast<double *>(dyn);
     sm.wd = sm.dd + static_cast<size_t>(E) * n;
     sm.wf = reinterpret_cast<float *>(sm.wd + n);
+    sm.df = sm.wf + n;
     const int64_t gpr = p.K > 0 ? p.K / n : 1;
     constexpr double kKeep = 1.0 - 0x1p-40;
     for (int64_t g = blockIdx.x; g < p.G; g += gridDim.x) {
         __syncwarp();
         // 1. stage
         float am = 0.0f;
-        bool bad = false;
+        bool bad = false, odd = false;
         for (int i = lane; i < n; i += 32) {
             const uint32_t b = p.W[g * n + i];
             bad |= (b & 0x7FFFu) >= kBeyond;
@@ -278,10 +289,13 @@ __global__ void __launch_bounds__(32) spec_kernel(SpecParams p)
             for (int e = 0; e < E; e++) {
                 const float d = p.K > 0 ? p.D[e * p.K + (g % gpr) * n + i] : p.D[(e * p.G + g) * n + i];
                 bad |= !(d >= 0.0f && d <= FLT_MAX);
+                odd |= d != 0.0f && !(d >= kTrustLo && d <= kTrustHi);
                 sm.dd[e * n + i] = d;
+                sm.df[e * n + i] = d;
             }
         }
         bad = __any_sync(kFull, bad);
+        const bool trust = !__any_sync(kFull, odd);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
             am = fmaxf(am, __shfl_xor_sync(kFull, am, o));
@@ -354,40 +368,92 @@ __global__ void __launch_bounds__(32) spec_kernel(SpecParams p)
             hi = lo;
         }
         const uint32_t J1 = min(hi, jz);
-        // 4. chunks of 32 scales whose interval bound exceeds U are skipped; lane
-        // L bounds chunks L, L + 32, ...; bit c of the flag words marks chunk c kept
-        const int nch = static_cast<int>((J1 - J0) / kChunk + 1);
-        for (int c0 = 0; c0 < nch; c0 += 32) {
-            const int ch = c0 + lane;
-            bool k = false;
+        // 4. chunk bounds; lane L holds chunks L + 32 m in cb[m] (INFINITY when
+        // dropped; bit m of `gone` once taken).  C doubles from 8 until 256
+        // chunks cover the window.
+        const uint32_t len = J1 - J0 + 1;
+        uint32_t C = kMinChunk;
+        while (C * 32u * kLaneChunks < len)
+            C *= 2;
+        const int nch = static_cast<int>((len + C - 1) / C);
+        float cb[kLaneChunks];
+#pragma unroll
+        for (int m = 0; m < kLaneChunks; m++) {
+            const int ch = lane + 32 * m;
+            float v = INFINITY;
             if (ch < nch) {
-                const uint32_t a = J0 + static_cast<uint32_t>(ch) * kChunk;
-                const uint32_t b = min(a + kChunk - 1, J1);
-                k = chunk_bound<E>(sm, n, p.qmin, p.qmax, grid_value(a), grid_value(b)) * kKeepChunk <= U;
+                v = 0.0f;
+                if (trust) {
+                    const uint32_t a = J0 + static_cast<uint32_t>(ch) * C;
+                    const uint32_t b = min(a + C - 1, J1);
+                    v = chunk_bound<E>(sm, n, p.qmin, p.qmax, grid_value(a), grid_value(b));
+                    if (v * kKeepChunk > U)
+                        v = INFINITY;
+                }
             }
-            const unsigned bal = __ballot_sync(kFull, k);
-            if (lane == 0)
-                keepw[c0 >> 5] = bal;
+            cb[m] = v;
         }
-        __syncwarp();
-        // 5. scan the kept chunks in ascending order, one scale per lane, so each
-        // lane meets its scales in ascending order and strict < keeps the lowest
+        // 5. best first.  A batch takes up to 32 / C chunks (one for C >= 32, its
+        // scales in C / 32 passes), smallest bound first (lowest chunk on ties),
+        // while that bound times 1 - 2^-12 does not exceed thr: U, then the best
+        // objective evaluated.  A chunk left over has every objective above
+        // thr, so strictly above the minimum.  Per lane, the (objective,
+        // pattern) minimum in that order.
         double bf = INFINITY;
         uint32_t bj = 0xFFFFFFFFu;
-        for (int wi = 0; wi < (nch + 31) / 32; wi++) {
-            uint32_t bits = keepw[wi];
-            while (bits) {
-                const int ch = 32 * wi + __ffs(bits) - 1;
-                bits &= bits - 1;
-                const uint32_t j = J0 + static_cast<uint32_t>(ch) * kChunk + static_cast<uint32_t>(lane);
-                if (j <= J1) {
+        double thr = U;
+        const int per = C >= 32u ? 1 : static_cast<int>(32u / C);
+        const int passes = C >= 32u ? static_cast<int>(C / 32u) : 1;
+        uint32_t gone = 0;
+        for (;;) {
+            int mine = -1;
+            int taken = 0;
+            for (int t = 0; t < per; t++) {
+                float v = INFINITY;
+                int mi = 0;
+#pragma unroll
+                for (int m = 0; m < kLaneChunks; m++) {
+                    if (!((gone >> m) & 1u) && cb[m] < v) {
+                        v = cb[m];
+                        mi = m;
+                    }
+                }
+                int c = v < INFINITY ? lane + 32 * mi : 0x7FFFFFFF;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    const float ov = __shfl_xor_sync(kFull, v, o);
+                    const int oc = __shfl_xor_sync(kFull, c, o);
+                    if (ov < v || (ov == v && oc < c)) {
+                        v = ov;
+                        c = oc;
+                    }
+                }
+                if (c == 0x7FFFFFFF || v * kKeepChunk > thr)
+                    break;  // uniform: every lane holds the same (v, c)
+                if (lane == (c & 31))
+                    gone |= 1u << (c >> 5);
+                if (C >= 32u || lane / static_cast<int>(C) == t)
+                    mine = c;
+                taken++;
+            }
+            if (taken == 0)
+                break;
+            for (int ps = 0; ps < passes; ps++) {
+                const uint32_t off = C >= 32u ? static_cast<uint32_t>(ps * 32 + lane) : static_cast<uint32_t>(lane) % C;
+                const uint32_t j = J0 + static_cast<uint32_t>(mine) * C + off;
+                if (mine >= 0 && j <= J1) {
                     const double v = objective_at<E>(sm, n, p.qmin, p.qmax, j);
-                    if (v < bf) {
+                    if (v < bf || (v == bf && j < bj)) {
                         bf = v;
                         bj = j;
                     }
                 }
             }
+            double mf = bf;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                mf = fmin(mf, __shfl_xor_sync(kFull, mf, o));
+            thr = fmin(thr, mf);
         }
         warp_best(bf, bj);
         // 6. outputs
@@ -413,7 +479,8 @@ template <int E>
 cudaError_t launch_spec(const SpecParams &p, cudaStream_t st)
 {
     const int n = p.n;
-    const size_t smem = static_cast<size_t>(E) * n * sizeof(double) + n * sizeof(double) + n * sizeof(float);
+    const size_t smem = static_cast<size_t>(E) * n * (sizeof(double) + sizeof(float)) + n * sizeof(double) +
+                        n * sizeof(float);
     cudaError_t err = cudaSuccess;
     if (smem > 48 * 1024 &&
         (err = cudaFuncSetAttribute(spec_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
