@@ -476,7 +476,8 @@ def bench_spec(args, wl, dev):
                 "config": {"workload": f"sweep-rows0-{SPEC_ROWS}-q[{qmin},{qmax}]-n{n}", "groups": G, "E": wl.E,
                            "K": wl.cols, "qmin": qmin, "qmax": qmax, "group_size": n},
                 "roofline": {"bound": "alu", "achieved": ach, "peak": p32, "unit": "TFLOP/s", "frac": ach / p32,
-                             "traffic": None, "kernel": "spec_kernel", "fp32_flops": f32, "fp64_flops": f64,
+                             "traffic": recorded_kernel_traffic("spec_kernel<4>", W.size), "kernel": "spec_kernel",
+                             "fp32_flops": f32, "fp64_flops": f64,
                              "peak_note": psrc}}
         print(json.dumps(line), flush=True)
 

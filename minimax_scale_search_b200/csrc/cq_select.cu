@@ -107,6 +107,10 @@ __device__ __forceinline__ const float *diag_ptr(const Params &p, int64_t g, int
     return p.D + (static_cast<int64_t>(e) * p.G + g) * kGroup;
 }
 
+// fp32 bit patterns of 2^-64 and 2^81, the ends of the diagonal range the fp32
+// screens are sound for.
+constexpr uint32_t kDLowBits = 0x1F800000u, kDHighBits = 0x68000000u;
+
 // 1 / (k + 1/2), k = 0..7 (only an estimate's accuracy is needed).
 __constant__ float c_inv_half[8] = {2.0f, 2.0f / 3.0f, 2.0f / 5.0f, 2.0f / 7.0f,
                                     2.0f / 9.0f, 2.0f / 11.0f, 2.0f / 13.0f, 2.0f / 15.0f};
@@ -553,7 +557,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     const DiagView dv_g = diag_view(p, g);
     const uint2 wv = *reinterpret_cast<const uint2 *>(p.W + g * kGroup + 4 * lane);
     const uint32_t wb[4] = {wv.x & 0xFFFFu, wv.x >> 16, wv.y & 0xFFFFu, wv.y >> 16};
-    bool bad = false, nonzero = false, odd = false;
+    bool bad = false, nonzero = false, rare = false;
     double A[E];
 #pragma unroll
     for (int m = 0; m < 4; m++) {
@@ -567,12 +571,32 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         double a = 0.0;
 #pragma unroll
         for (int m = 0; m < 4; m++) {
-            bad |= !(dq[m] >= 0.0f && dq[m] <= FLT_MAX);
-            odd |= dq[m] != 0.0f && !(dq[m] >= 0x1p-64f && dq[m] <= 0x1p96f);
+            // d outside [2^-64, 2^81]: zero, negative, non-finite or extreme
+            rare |= __float_as_uint(dq[m]) - kDLowBits > kDHighBits - kDLowBits;
             const double wd = half_value(wb[m]);
             a += static_cast<double>(dq[m]) * (wd * wd);  // exact: 24-bit d times 22-bit w^2
         }
         A[e] = a;
+    }
+    // The fp32 steps below bound their error relative to the terms, which holds
+    // while no fp32 value overflows or leaves the normal range.  Every objective
+    // is at most max_e A_e <= 128 max d 65504^2 (each residual is at most |w|),
+    // screened values stay within 16 max_e A_e, and B = sum d|w||q| and
+    // C = sum d q^2 within 2^26 max d; so with every nonzero d in [2^-64, 2^81]
+    // every nonzero fp32 value lies in [2^-112, 2^124].  Groups with another
+    // nonzero d take the fp64 exhaustive pass.
+    bool odd = false;
+    if (__any_sync(kFull, rare)) {
+#pragma unroll
+        for (int e = 0; e < E; e++) {
+#pragma unroll
+            for (int m = 0; m < 4; m++) {
+                const float d = dv_g.base[e * dv_g.stride + 4 * lane + m];
+                bad |= !(d >= 0.0f && d <= FLT_MAX);
+                odd |= d != 0.0f && !(d >= 0x1p-64f && d <= 0x1p81f);
+            }
+        }
+        odd = __any_sync(kFull, odd);
     }
     bad = __any_sync(kFull, bad);
     nonzero = __any_sync(kFull, nonzero);
@@ -590,24 +614,15 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         enqueue(p, g, lane, tl);
         return;
     }
+    if (odd) {
+        enqueue(p, g, lane, tl);
+        return;
+    }
     float Af[E];
-    double amx = 0.0;
 #pragma unroll
     for (int e = 0; e < E; e++) {
         A[e] = warp_sum(A[e]);
         Af[e] = static_cast<float>(A[e]);
-        amx = fmax(amx, A[e]);
-    }
-    // The fp32 steps below bound their error relative to the terms, which holds
-    // while no fp32 value overflows or leaves the normal range.  Every objective
-    // is at most max_e A_e (each residual is at most |w|), screened values stay
-    // within 16 max_e A_e, and B = sum d|w||q| and C = sum d q^2 within
-    // 2^26 max d; so with every nonzero d in [2^-64, 2^96] and max_e A_e <= 2^120
-    // every nonzero fp32 value lies in [2^-112, 2^124].  Other groups take the
-    // fp64 exhaustive pass.
-    if (__any_sync(kFull, odd) || amx > 0x1p120) {
-        enqueue(p, g, lane, tl);
-        return;
     }
 
     // ---- 2. order the weights by |w|; stage w and d by rank ----------------

@@ -95,6 +95,7 @@ struct Smem {
     double *wd;  // [n]
     double *dd;  // [E][n]
     float *df;   // [E][n] the same diagonals in fp32 (exact), for the chunk bounds
+    float *cbs;  // [kLaneChunks * 32] chunk bounds
 };
 
 // Objective at grid index j, in the definition's order; one thread.
@@ -108,7 +109,7 @@ __device__ double objective_at(const Smem &sm, int n, int qmin, int qmax, uint32
 #pragma unroll
     for (int e = 0; e < CQ_MAX_E; e++)
         acc[e] = 0.0;
-    // the codes of 4 consecutive weights are computed independently; each
+    // the codes of 8 consecutive weights are computed independently; each
     // environment's running sum still takes the weights in ascending order
     auto term = [&](int i) {
         const float w = sm.wf[i];
@@ -122,9 +123,9 @@ __device__ double objective_at(const Smem &sm, int n, int qmin, int qmax, uint32
                 acc[e] = __dadd_rn(acc[e], __dmul_rn(sm.dd[e * n + i], rr));
     };
     int i = 0;
-    for (; i + 4 <= n; i += 4) {
+    for (; i + 8 <= n; i += 8) {
 #pragma unroll
-        for (int u = 0; u < 4; u++)
+        for (int u = 0; u < 8; u++)
             term(i + u);
     }
     for (; i < n; i++)
@@ -271,6 +272,7 @@ __global__ void __launch_bounds__(32) spec_kernel(SpecParams p)
     sm.wd = sm.dd + static_cast<size_t>(E) * n;
     sm.wf = reinterpret_cast<float *>(sm.wd + n);
     sm.df = sm.wf + n;
+    sm.cbs = sm.df + static_cast<size_t>(E) * n;
     const int64_t gpr = p.K > 0 ? p.K / n : 1;
     constexpr double kKeep = 1.0 - 0x1p-40;
     for (int64_t g = blockIdx.x; g < p.G; g += gridDim.x) {
@@ -342,32 +344,27 @@ __global__ void __launch_bounds__(32) spec_kernel(SpecParams p)
                 jb = j;
             }
         }
-        // 3. certified window [J0, J1]
-        uint32_t lo = 1, hi = jb;  // smallest index whose clipping bound does not exclude it
-        if (bound_at<E>(sm, n, p.qmin, p.qmax, 1, 0) * kKeep > U) {
-            while (hi - lo > 1) {  // invariant: lo excluded, hi not
-                const uint32_t mid = (lo + hi) / 2;
-                if (bound_at<E>(sm, n, p.qmin, p.qmax, mid, 0) * kKeep > U)
-                    lo = mid;
+        // 3. certified window [J0, J1]: side 0 bisects [1, jb] for the smallest
+        // index the clipping bound keeps (it falls as s rises), side 1 bisects
+        // [jb, kLast] for the largest the dead-zone bound keeps (it rises with
+        // s); jb is kept by both, and the indices 0 and kLast + 1 stand for
+        // excluded ends.
+        uint32_t J0 = jb, J1 = jb;
+#pragma unroll 1
+        for (int side = 0; side < 2; side++) {
+            uint32_t ex = side == 0 ? 0u : kLast + 1u, ok = jb;
+            while (ex + 1u != ok && ok + 1u != ex) {
+                const uint32_t mid = (ex + ok) / 2u;
+                if (bound_at<E>(sm, n, p.qmin, p.qmax, mid, side) * kKeep > U)
+                    ex = mid;
                 else
-                    hi = mid;
+                    ok = mid;
             }
-            lo = hi;
+            if (side == 0)
+                J0 = ok;
+            else
+                J1 = min(ok, jz);
         }
-        const uint32_t J0 = lo;
-        lo = jb;
-        hi = kLast;
-        if (bound_at<E>(sm, n, p.qmin, p.qmax, kLast, 1) * kKeep > U) {
-            while (hi - lo > 1) {  // invariant: lo not excluded, hi excluded
-                const uint32_t mid = (lo + hi) / 2;
-                if (bound_at<E>(sm, n, p.qmin, p.qmax, mid, 1) * kKeep > U)
-                    hi = mid;
-                else
-                    lo = mid;
-            }
-            hi = lo;
-        }
-        const uint32_t J1 = min(hi, jz);
         // 4. chunk bounds; lane L holds chunks L + 32 m in cb[m] (INFINITY when
         // dropped; bit m of `gone` once taken).  C doubles from 8 until 256
         // chunks cover the window.
@@ -376,22 +373,23 @@ __global__ void __launch_bounds__(32) spec_kernel(SpecParams p)
         while (C * 32u * kLaneChunks < len)
             C *= 2;
         const int nch = static_cast<int>((len + C - 1) / C);
+        for (int ch = lane; ch < nch; ch += 32) {
+            float v = 0.0f;
+            if (trust) {
+                const uint32_t a = J0 + static_cast<uint32_t>(ch) * C;
+                const uint32_t b = min(a + C - 1, J1);
+                v = chunk_bound<E>(sm, n, p.qmin, p.qmax, grid_value(a), grid_value(b));
+                if (v * kKeepChunk > U)
+                    v = INFINITY;
+            }
+            sm.cbs[ch] = v;
+        }
+        __syncwarp();
         float cb[kLaneChunks];
 #pragma unroll
         for (int m = 0; m < kLaneChunks; m++) {
             const int ch = lane + 32 * m;
-            float v = INFINITY;
-            if (ch < nch) {
-                v = 0.0f;
-                if (trust) {
-                    const uint32_t a = J0 + static_cast<uint32_t>(ch) * C;
-                    const uint32_t b = min(a + C - 1, J1);
-                    v = chunk_bound<E>(sm, n, p.qmin, p.qmax, grid_value(a), grid_value(b));
-                    if (v * kKeepChunk > U)
-                        v = INFINITY;
-                }
-            }
-            cb[m] = v;
+            cb[m] = ch < nch ? sm.cbs[ch] : INFINITY;
         }
         // 5. best first.  A batch takes up to 32 / C chunks (one for C >= 32, its
         // scales in C / 32 passes), smallest bound first (lowest chunk on ties),
@@ -480,7 +478,7 @@ cudaError_t launch_spec(const SpecParams &p, cudaStream_t st)
 {
     const int n = p.n;
     const size_t smem = static_cast<size_t>(E) * n * (sizeof(double) + sizeof(float)) + n * sizeof(double) +
-                        n * sizeof(float);
+                        n * sizeof(float) + kLaneChunks * 32 * sizeof(float);
     cudaError_t err = cudaSuccess;
     if (smem > 48 * 1024 &&
         (err = cudaFuncSetAttribute(spec_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
