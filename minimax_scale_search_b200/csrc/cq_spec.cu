@@ -90,11 +90,32 @@ __device__ __forceinline__ int spec_code(float aw, float s, float inv, int cap)
     return min(mi - below + above, cap);
 }
 
+// fp32 diagonals per weight, padded to whole float4 loads; fp64 ones padded
+// to whole double2 loads
+template <int E>
+constexpr int kPadE = E <= 4 ? 4 : 8;
+template <int E>
+constexpr int kPadD = (E + 1) & ~1;
+
+// The E fp64 diagonals of weight i, from kPadD<E> / 2 16-byte loads.
+template <int E>
+__device__ __forceinline__ void load_dd(const double *dd, int i, double (&d)[kPadD<E>])
+{
+    const double2 *dp = reinterpret_cast<const double2 *>(dd + i * kPadD<E>);
+#pragma unroll
+    for (int h = 0; h < kPadD<E> / 2; h++) {
+        const double2 v = dp[h];
+        d[2 * h] = v.x;
+        d[2 * h + 1] = v.y;
+    }
+}
+
 struct Smem {
     float *wf;   // [n] exact weights
     double *wd;  // [n]
-    double *dd;  // [E][n]
-    float *df;   // [E][n] the same diagonals in fp32 (exact), for the chunk bounds
+    double *dd;  // [n][kPadD]
+    float *df;   // [n][kPadE] the same diagonals in fp32 (exact), for the chunk bounds
+    float2 *ac;  // [n] (|w|, the code cap of w's sign)
     float *cbs;  // [kLaneChunks * 32] chunk bounds
 };
 
@@ -117,10 +138,11 @@ __device__ double objective_at(const Smem &sm, int n, int qmin, int qmax, uint32
         const int c = spec_code(fabsf(w), s, inv, neg ? -qmin : qmax);
         const double r = fma(nsd, static_cast<double>(neg ? -c : c), sm.wd[i]);
         const double rr = __dmul_rn(r, r);
+        double d[kPadD<E>];
+        load_dd<E>(sm.dd, i, d);
 #pragma unroll
-        for (int e = 0; e < CQ_MAX_E; e++)
-            if (e < E)
-                acc[e] = __dadd_rn(acc[e], __dmul_rn(sm.dd[e * n + i], rr));
+        for (int e = 0; e < E; e++)
+            acc[e] = __dadd_rn(acc[e], __dmul_rn(d[e], rr));
     };
     int i = 0;
     for (; i + 8 <= n; i += 8) {
@@ -178,9 +200,11 @@ __device__ double bound_at(const Smem &sm, int n, int qmin, int qmax, uint32_t j
         } else if (!code_at_least(aw, s, 1)) {
             t = sm.wd[i] * sm.wd[i];
         }
+        double d[kPadD<E>];
+        load_dd<E>(sm.dd, i, d);
 #pragma unroll
         for (int e = 0; e < E; e++)
-            acc[e] += sm.dd[e * n + i] * t;
+            acc[e] += d[e] * t;
     }
     double best = 0.0;
 #pragma unroll
@@ -209,9 +233,11 @@ __device__ double upper_at(const Smem &sm, int n, int qmin, int qmax, uint32_t j
         const int c = spec_code(fabsf(w), s, inv, neg ? -qmin : qmax);
         const double r = fma(nsd, static_cast<double>(neg ? -c : c), sm.wd[i]);
         const double rr = r * r;
+        double d[kPadD<E>];
+        load_dd<E>(sm.dd, i, d);
 #pragma unroll
         for (int e = 0; e < E; e++)
-            acc[e] = fma(sm.dd[e * n + i], rr, acc[e]);
+            acc[e] = fma(d[e], rr, acc[e]);
     }
     double f = 0.0;
 #pragma unroll
@@ -240,18 +266,26 @@ __device__ float chunk_bound(const Smem &sm, int n, int qmin, int qmax, float s_
     for (int e = 0; e < CQ_MAX_E; e++)
         acc[e] = 0.0f;
     for (int i = 0; i < n; i++) {
-        const float w = sm.wf[i];
-        const float aw = fabsf(w);
-        const float cap = static_cast<float>(w < 0.0f ? -qmin : qmax);
+        const float2 a = sm.ac[i];
+        const float aw = a.x, cap = a.y;
         const float k1 = fminf(floorf(aw * inv_hi), cap);
         const float e1 = fmaxf(fmaf(-k1, s_hi, aw), 0.0f);
         const float e2 = k1 < cap ? fmaxf(fmaf(k1 + 1.0f, s_lo, -aw), 0.0f) : INFINITY;
         const float dist = fminf(e1, e2);
         const float d2 = dist * dist;
+        const float4 *dv = reinterpret_cast<const float4 *>(sm.df + i * kPadE<E>);
+        float dq[kPadE<E>];
 #pragma unroll
-        for (int e = 0; e < CQ_MAX_E; e++)
-            if (e < E)
-                acc[e] = fmaf(sm.df[e * n + i], d2, acc[e]);
+        for (int h = 0; h < kPadE<E> / 4; h++) {
+            const float4 v = dv[h];
+            dq[4 * h] = v.x;
+            dq[4 * h + 1] = v.y;
+            dq[4 * h + 2] = v.z;
+            dq[4 * h + 3] = v.w;
+        }
+#pragma unroll
+        for (int e = 0; e < E; e++)
+            acc[e] = fmaf(dq[e], d2, acc[e]);
     }
     float best = 0.0f;
 #pragma unroll
@@ -268,11 +302,13 @@ __global__ void __launch_bounds__(32) spec_kernel(SpecParams p)
     const int n = p.n;
     const int lane = threadIdx.x & 31;
     Smem sm;
-    sm.dd = reinterpret_cast<double *>(dyn);
-    sm.wd = sm.dd + static_cast<size_t>(E) * n;
-    sm.wf = reinterpret_cast<float *>(sm.wd + n);
-    sm.df = sm.wf + n;
-    sm.cbs = sm.df + static_cast<size_t>(E) * n;
+    // 16-byte aligned first: df; then 8-byte items; then 4-byte items
+    sm.df = reinterpret_cast<float *>(dyn);
+    sm.dd = reinterpret_cast<double *>(sm.df + static_cast<size_t>(kPadE<E>) * n);
+    sm.wd = sm.dd + static_cast<size_t>(kPadD<E>) * n;
+    sm.ac = reinterpret_cast<float2 *>(sm.wd + n);
+    sm.wf = reinterpret_cast<float *>(sm.ac + n);
+    sm.cbs = sm.wf + n;
     const int64_t gpr = p.K > 0 ? p.K / n : 1;
     constexpr double kKeep = 1.0 - 0x1p-40;
     for (int64_t g = blockIdx.x; g < p.G; g += gridDim.x) {
@@ -286,15 +322,21 @@ __global__ void __launch_bounds__(32) spec_kernel(SpecParams p)
             const float w = half_value(b);
             sm.wf[i] = w;
             sm.wd[i] = w;
+            sm.ac[i] = make_float2(fabsf(w), static_cast<float>(w < 0.0f ? -p.qmin : p.qmax));
             am = fmaxf(am, fabsf(w));
 #pragma unroll
             for (int e = 0; e < E; e++) {
                 const float d = p.K > 0 ? p.D[e * p.K + (g % gpr) * n + i] : p.D[(e * p.G + g) * n + i];
                 bad |= !(d >= 0.0f && d <= FLT_MAX);
                 odd |= d != 0.0f && !(d >= kTrustLo && d <= kTrustHi);
-                sm.dd[e * n + i] = d;
-                sm.df[e * n + i] = d;
+                sm.dd[i * kPadD<E> + e] = d;
+                sm.df[i * kPadE<E> + e] = d;
             }
+            if (kPadD<E> > E)
+                sm.dd[i * kPadD<E> + E] = 0.0;
+#pragma unroll
+            for (int e = E; e < kPadE<E>; e++)
+                sm.df[i * kPadE<E> + e] = 0.0f;
         }
         bad = __any_sync(kFull, bad);
         const bool trust = !__any_sync(kFull, odd);
@@ -477,8 +519,9 @@ template <int E>
 cudaError_t launch_spec(const SpecParams &p, cudaStream_t st)
 {
     const int n = p.n;
-    const size_t smem = static_cast<size_t>(E) * n * (sizeof(double) + sizeof(float)) + n * sizeof(double) +
-                        n * sizeof(float) + kLaneChunks * 32 * sizeof(float);
+    const size_t smem = static_cast<size_t>(n) * (kPadE<E> * sizeof(float) + kPadD<E> * sizeof(double) + sizeof(double) +
+                                                  sizeof(float2) + sizeof(float)) +
+                        kLaneChunks * 32 * sizeof(float);
     cudaError_t err = cudaSuccess;
     if (smem > 48 * 1024 &&
         (err = cudaFuncSetAttribute(spec_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
