@@ -174,76 +174,152 @@ __device__ __forceinline__ void warp_best(double &f, uint32_t &j)
     }
 }
 
-// Max over environments of a per-environment sum of per-weight terms, the
-// lanes taking weights lane, lane + 32, ... (any order: a bound, used with a
-// margin).  kind 0: clipped weights' error at s; kind 1: error of the weights
-// that quantise to 0 at s.  Every lane gets the result.
+// max over e of the warp-wide sums of acc[e], on every lane.  A reduce-scatter
+// halves the values a lane carries at each of the first log2 N butterfly
+// steps (N = E rounded up to a power of two), so after the five steps the
+// block of 32 / N consecutive lanes j 32 / N ... holds sum j; the max over the
+// blocks follows.  The summation order differs from a plain butterfly; the
+// callers' margins cover any order.
 template <int E>
-__device__ double bound_at(const Smem &sm, int n, int qmin, int qmax, uint32_t j, int kind)
+__device__ __forceinline__ double warp_max_of_sums(const double (&acc)[E], int lane)
 {
-    const float s = grid_value(j);
-    const double sd = s;
-    double acc[E];
+    constexpr int N = E <= 1 ? 1 : E <= 2 ? 2 : E <= 4 ? 4 : 8;
+    double x[N];
 #pragma unroll
-    for (int e = 0; e < E; e++)
-        acc[e] = 0.0;
+    for (int i = 0; i < N; i++)
+        x[i] = i < E ? acc[i] : 0.0;
+    int o = 16;
+#pragma unroll
+    for (int h = N / 2; h >= 1; h /= 2, o >>= 1) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < h; i++) {
+            const double send = up ? x[i] : x[i + h];
+            const double keep = up ? x[i + h] : x[i];
+            x[i] = keep + __shfl_xor_sync(kFull, send, o);
+        }
+    }
+#pragma unroll
+    for (; o > 0; o >>= 1)
+        x[0] += __shfl_xor_sync(kFull, x[0], o);
+#pragma unroll
+    for (int b = 32 / N; b < 32; b <<= 1)
+        x[0] = fmax(x[0], __shfl_xor_sync(kFull, x[0], b));
+    return x[0];
+}
+
+// The same for two sets of E values at once: m0 = max over e of the sums of
+// a0[e], m1 = the same for a1[e].  After the reduce-scatter of the 2N values
+// lanes 0-15 hold the sums of a0 and lanes 16-31 those of a1.
+template <int E>
+__device__ __forceinline__ void warp_max_of_sums2(const double (&a0)[E], const double (&a1)[E], int lane, double &m0,
+                                                  double &m1)
+{
+    constexpr int N = E <= 1 ? 1 : E <= 2 ? 2 : E <= 4 ? 4 : 8;
+    constexpr int N2 = 2 * N;
+    double x[N2];
+#pragma unroll
+    for (int i = 0; i < N; i++) {
+        x[i] = i < E ? a0[i] : 0.0;
+        x[N + i] = i < E ? a1[i] : 0.0;
+    }
+    int o = 16;
+#pragma unroll
+    for (int h = N2 / 2; h >= 1; h /= 2, o >>= 1) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < h; i++) {
+            const double send = up ? x[i] : x[i + h];
+            const double keep = up ? x[i + h] : x[i];
+            x[i] = keep + __shfl_xor_sync(kFull, send, o);
+        }
+    }
+#pragma unroll
+    for (; o > 0; o >>= 1)
+        x[0] += __shfl_xor_sync(kFull, x[0], o);
+#pragma unroll
+    for (int b = 32 / N2; b < 16; b <<= 1)
+        x[0] = fmax(x[0], __shfl_xor_sync(kFull, x[0], b));
+    m0 = __shfl_sync(kFull, x[0], 0);
+    m1 = __shfl_sync(kFull, x[0], 16);
+}
+
+// Two window bounds in one pass over the weights, each the max over
+// environments of a per-environment sum of per-weight terms (the lanes take
+// weights lane, lane + 32, ...; any order: a bound, used with a margin):
+// b0 = the clipped weights' error at grid index j0, b1 = the error of the
+// weights that quantise to 0 at j1.  Every lane gets both.
+template <int E>
+__device__ void bound_pair(const Smem &sm, int n, int qmin, int qmax, uint32_t j0, uint32_t j1, double &b0,
+                           double &b1)
+{
+    const float s0 = grid_value(j0), s1 = grid_value(j1);
+    const double sd0 = s0;
+    double a0[E], a1[E];
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        a0[e] = 0.0;
+        a1[e] = 0.0;
+    }
     for (int i = threadIdx.x & 31; i < n; i += 32) {
         const float w = sm.wf[i];
         const float aw = fabsf(w);
-        double t = 0.0;
-        if (kind == 0) {
-            const int cap = w < 0.0f ? -qmin : qmax;
-            if (code_at_least(aw, s, cap + 1)) {
-                const double x = static_cast<double>(aw) - cap * sd;
-                t = x * x;
-            }
-        } else if (!code_at_least(aw, s, 1)) {
-            t = sm.wd[i] * sm.wd[i];
+        const int cap = w < 0.0f ? -qmin : qmax;
+        double t0 = 0.0, t1 = 0.0;
+        if (code_at_least(aw, s0, cap + 1)) {
+            const double x = static_cast<double>(aw) - cap * sd0;
+            t0 = x * x;
         }
+        if (!code_at_least(aw, s1, 1))
+            t1 = sm.wd[i] * sm.wd[i];
         double d[kPadD<E>];
         load_dd<E>(sm.dd, i, d);
 #pragma unroll
-        for (int e = 0; e < E; e++)
-            acc[e] += d[e] * t;
+        for (int e = 0; e < E; e++) {
+            a0[e] += d[e] * t0;
+            a1[e] += d[e] * t1;
+        }
     }
-    double best = 0.0;
-#pragma unroll
-    for (int e = 0; e < E; e++)
-        best = fmax(best, warp_sum(acc[e]));
-    return best;
+    warp_max_of_sums2<E>(a0, a1, threadIdx.x & 31, b0, b1);
 }
 
-// An upper bound of the objective at grid index j that the warp sums in any
-// order: the exact value's fp64 sums err by at most n 2^-53 relative either
-// way, so the warp sum times (1 + 2^-40) is at least the definition's own
-// value for n <= 4096.  Every lane gets the result.
+// Upper bounds of the objective at grid indices ja and jb, from one pass over
+// the weights, which the warp sums in any order: the exact value's fp64 sums
+// err by at most n 2^-53 relative either way, so the warp sum times
+// (1 + 2^-40) is at least the definition's own value for n <= 4096.  Every
+// lane gets both.
 template <int E>
-__device__ double upper_at(const Smem &sm, int n, int qmin, int qmax, uint32_t j)
+__device__ void upper_pair(const Smem &sm, int n, int qmin, int qmax, uint32_t ja, uint32_t jb, double &ua,
+                           double &ub)
 {
-    const float s = grid_value(j);
-    const float inv = 1.0f / s;
-    const double nsd = -static_cast<double>(s);
-    double acc[E];
+    const float sa = grid_value(ja), sb = grid_value(jb);
+    const float inva = 1.0f / sa, invb = 1.0f / sb;
+    const double nsa = -static_cast<double>(sa), nsb = -static_cast<double>(sb);
+    double a0[E], a1[E];
 #pragma unroll
-    for (int e = 0; e < E; e++)
-        acc[e] = 0.0;
+    for (int e = 0; e < E; e++) {
+        a0[e] = 0.0;
+        a1[e] = 0.0;
+    }
     for (int i = threadIdx.x & 31; i < n; i += 32) {
         const float w = sm.wf[i];
         const bool neg = w < 0.0f;
-        const int c = spec_code(fabsf(w), s, inv, neg ? -qmin : qmax);
-        const double r = fma(nsd, static_cast<double>(neg ? -c : c), sm.wd[i]);
-        const double rr = r * r;
+        const int cap = neg ? -qmin : qmax;
+        const int c0 = spec_code(fabsf(w), sa, inva, cap), c1 = spec_code(fabsf(w), sb, invb, cap);
+        const double r0 = fma(nsa, static_cast<double>(neg ? -c0 : c0), sm.wd[i]);
+        const double r1 = fma(nsb, static_cast<double>(neg ? -c1 : c1), sm.wd[i]);
+        const double rr0 = r0 * r0, rr1 = r1 * r1;
         double d[kPadD<E>];
         load_dd<E>(sm.dd, i, d);
 #pragma unroll
-        for (int e = 0; e < E; e++)
-            acc[e] = fma(d[e], rr, acc[e]);
+        for (int e = 0; e < E; e++) {
+            a0[e] = fma(d[e], rr0, a0[e]);
+            a1[e] = fma(d[e], rr1, a1[e]);
+        }
     }
-    double f = 0.0;
-#pragma unroll
-    for (int e = 0; e < E; e++)
-        f = fmax(f, warp_sum(acc[e]));
-    return f * (1.0 + 0x1p-40);
+    warp_max_of_sums2<E>(a0, a1, threadIdx.x & 31, ua, ub);
+    ua *= 1.0 + 0x1p-40;
+    ub *= 1.0 + 0x1p-40;
 }
 
 // A lower bound of the objective at every scale in [s_lo, s_hi]: at any such s
@@ -368,45 +444,60 @@ __global__ void __launch_bounds__(32) spec_kernel(SpecParams p)
         }
         double U = INFINITY;
         uint32_t jb = 1;
-        for (int t = 0; t < kCandidates; t++) {
-            uint32_t j;
-            if (t == kCandidates - 1) {
-                j = jz;
-            } else {
-                const double base = static_cast<double>(amax) / (t < 3 ? p.qmax : -p.qmin);
-                const int off = (t % 3) - 1;
-                const int jc = static_cast<int>(__half_as_ushort(__double2half(base))) + off;
-                j = static_cast<uint32_t>(min(max(jc, 1), static_cast<int>(kLast)));
+        // candidates in pairs (the last paired with itself; j_z dropped when
+        // above the grid); the first of equal bounds is kept
+        for (int t = 0; t < kCandidates; t += 2) {
+            uint32_t jp[2];
+#pragma unroll
+            for (int k = 0; k < 2; k++) {
+                const int tt = min(t + k, kCandidates - 1);
+                if (tt == kCandidates - 1) {
+                    jp[k] = jz;
+                } else {
+                    const double base = static_cast<double>(amax) / (tt < 3 ? p.qmax : -p.qmin);
+                    const int off = (tt % 3) - 1;
+                    const int jc = static_cast<int>(__half_as_ushort(__double2half(base))) + off;
+                    jp[k] = static_cast<uint32_t>(min(max(jc, 1), static_cast<int>(kLast)));
+                }
             }
-            if (j > kLast)
-                continue;
-            const double u = upper_at<E>(sm, n, p.qmin, p.qmax, j);
-            if (u < U) {
-                U = u;
-                jb = j;
+            double u[2];
+            upper_pair<E>(sm, n, p.qmin, p.qmax, min(jp[0], kLast), min(jp[1], kLast), u[0], u[1]);
+#pragma unroll
+            for (int k = 0; k < 2; k++) {
+                if (jp[k] <= kLast && u[k] < U) {
+                    U = u[k];
+                    jb = jp[k];
+                }
             }
         }
-        // 3. certified window [J0, J1]: side 0 bisects [1, jb] for the smallest
-        // index the clipping bound keeps (it falls as s rises), side 1 bisects
+        // 3. certified window [J0, J1]: one bisection over [1, jb] for the
+        // smallest index the clipping bound keeps (it falls as s rises), one over
         // [jb, kLast] for the largest the dead-zone bound keeps (it rises with
-        // s); jb is kept by both, and the indices 0 and kLast + 1 stand for
-        // excluded ends.
-        uint32_t J0 = jb, J1 = jb;
-#pragma unroll 1
-        for (int side = 0; side < 2; side++) {
-            uint32_t ex = side == 0 ? 0u : kLast + 1u, ok = jb;
-            while (ex + 1u != ok && ok + 1u != ex) {
-                const uint32_t mid = (ex + ok) / 2u;
-                if (bound_at<E>(sm, n, p.qmin, p.qmax, mid, side) * kKeep > U)
-                    ex = mid;
+        // s), advancing together with one pass over the weights per step.  jb
+        // is kept by both; the indices 0 and kLast + 1 stand for excluded ends.
+        uint32_t ex0 = 0u, ok0 = jb, ex1 = kLast + 1u, ok1 = jb;
+        for (;;) {
+            const bool go0 = ex0 + 1u != ok0, go1 = ok1 + 1u != ex1;
+            if (!go0 && !go1)
+                break;
+            const uint32_t m0 = go0 ? (ex0 + ok0) / 2u : ok0;
+            const uint32_t m1 = go1 ? (ex1 + ok1) / 2u : ok1;
+            double b0, b1;
+            bound_pair<E>(sm, n, p.qmin, p.qmax, m0, m1, b0, b1);
+            if (go0) {
+                if (b0 * kKeep > U)
+                    ex0 = m0;
                 else
-                    ok = mid;
+                    ok0 = m0;
             }
-            if (side == 0)
-                J0 = ok;
-            else
-                J1 = min(ok, jz);
+            if (go1) {
+                if (b1 * kKeep > U)
+                    ex1 = m1;
+                else
+                    ok1 = m1;
+            }
         }
+        const uint32_t J0 = ok0, J1 = min(ok1, jz);
         // 4. chunk bounds; lane L holds chunks L + 32 m in cb[m] (INFINITY when
         // dropped; bit m of `gone` once taken).  C doubles from 8 until 256
         // chunks cover the window.
