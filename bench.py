@@ -336,14 +336,25 @@ def bench_policies(args, wl, W, D, Wd, Dd, dev):
                     args.warmup, stream)
     bpg = 256 + 2 + 8 * wl.E + 8
     byt = G * bpg
+    # The definition fixes 2 + 2E fp64 operations per weight (r = w - s q, r*r,
+    # and d*rr plus the running sum per environment), each one FP64 lane-clock.
+    ops = G * 128 * (2 + 2 * wl.E)
+    _, _, mhz, csrc = peaks()
+    p64ops = SMS * FP64_LANES * mhz * 1e6 / 1e12
+    hbm_gbs = byt / ms / 1e6
+    ops_t = ops / ms / 1e9
+    if ops / p64ops >= byt / hbm * 1e3:  # the fp64 pipe binds
+        roof = {"bound": "alu", "achieved": ops_t, "peak": p64ops, "unit": "Top/s (fp64 operations)",
+                "frac": ops_t / p64ops, "hbm_achieved_gbs": hbm_gbs, "hbm_frac": hbm_gbs / hbm,
+                "peak_note": f"{SMS} SMs x {FP64_LANES} FP64 lanes x {mhz:.0f} MHz ({csrc})"}
+    else:
+        roof = {"bound": "hbm", "achieved": hbm_gbs, "peak": hbm, "unit": "GB/s", "frac": hbm_gbs / hbm,
+                "alu_frac": ops_t / p64ops, "peak_note": hsrc}
+    roof.update({"traffic": recorded_kernel_traffic("objective_kernel<4,", G),
+                 "kernel": "objective_kernel<4, per-column>", "bytes_per_group": bpg, "fp64_ops": ops})
     lines.append(dict(base, metric="objective of given scales groups/sec", op="objective", value=G / ms * 1e3,
                       unit="groups/s", ms_per_step=ms, higher_is_better=True, dtype="f64",
-                      gpu_launches=2 * args.steps,
-                      roofline={"bound": "hbm", "achieved": byt / ms / 1e6, "peak": hbm, "unit": "GB/s",
-                                "frac": byt / ms / 1e6 / hbm,
-                                "traffic": recorded_kernel_traffic("objective_kernel<4,", G),
-                                "kernel": "objective_kernel<4, per-column>", "bytes_per_group": bpg,
-                                "peak_note": hsrc}))
+                      gpu_launches=2 * args.steps, roofline=roof))
 
     Wp, Dp, offsets = synth.make_proxy_inputs()
     Wpd = torch.from_numpy(Wp.view(np.int16)).to(dev)
