@@ -9,11 +9,14 @@
 //
 // One warp per group (a grid of one-warp CTAs, grid-stride over groups; many
 // groups in flight per SM hide the latency of each group's serial steps):
-//  1. stage w (exact fp32 and fp64) and the group's diagonals (fp64);
+//  1. stage w (exact fp32 and fp64, and |w| with its code cap) and the group's
+//     diagonals per weight (fp64 for the exact sums, fp32 for the chunk bounds);
 //  2. U: an upper bound of the smallest objective, from warp-parallel sums at
 //     the AbsMax-type scales fp16(max|w|/qmax), fp16(max|w|/|qmin|), their
-//     grid neighbours and the first scale at which every code is 0;
-//  3. a certified window [J0, J1]: below a scale, the clipped weights' error
+//     grid neighbours and the first scale at which every code is 0, two
+//     scales per pass over the weights;
+//  3. a certified window [J0, J1], by two bisections that share one pass over
+//     the weights per step: below a scale, the clipped weights' error
 //     sum_e-max of sum d (|w| - c s)^2 only grows as s falls; above one, the
 //     error of the weights that round to 0, sum d w^2, only grows as s rises.
 //     Both are fp64 lower bounds of the exact objective, taken with a 2^-40
@@ -174,43 +177,13 @@ __device__ __forceinline__ void warp_best(double &f, uint32_t &j)
     }
 }
 
-// max over e of the warp-wide sums of acc[e], on every lane.  A reduce-scatter
-// halves the values a lane carries at each of the first log2 N butterfly
-// steps (N = E rounded up to a power of two), so after the five steps the
-// block of 32 / N consecutive lanes j 32 / N ... holds sum j; the max over the
-// blocks follows.  The summation order differs from a plain butterfly; the
-// callers' margins cover any order.
-template <int E>
-__device__ __forceinline__ double warp_max_of_sums(const double (&acc)[E], int lane)
-{
-    constexpr int N = E <= 1 ? 1 : E <= 2 ? 2 : E <= 4 ? 4 : 8;
-    double x[N];
-#pragma unroll
-    for (int i = 0; i < N; i++)
-        x[i] = i < E ? acc[i] : 0.0;
-    int o = 16;
-#pragma unroll
-    for (int h = N / 2; h >= 1; h /= 2, o >>= 1) {
-        const bool up = (lane & o) != 0;
-#pragma unroll
-        for (int i = 0; i < h; i++) {
-            const double send = up ? x[i] : x[i + h];
-            const double keep = up ? x[i + h] : x[i];
-            x[i] = keep + __shfl_xor_sync(kFull, send, o);
-        }
-    }
-#pragma unroll
-    for (; o > 0; o >>= 1)
-        x[0] += __shfl_xor_sync(kFull, x[0], o);
-#pragma unroll
-    for (int b = 32 / N; b < 32; b <<= 1)
-        x[0] = fmax(x[0], __shfl_xor_sync(kFull, x[0], b));
-    return x[0];
-}
-
-// The same for two sets of E values at once: m0 = max over e of the sums of
-// a0[e], m1 = the same for a1[e].  After the reduce-scatter of the 2N values
-// lanes 0-15 hold the sums of a0 and lanes 16-31 those of a1.
+// m0 = max over e of the warp-wide sums of a0[e], m1 = the same for a1[e], on
+// every lane.  A reduce-scatter halves the values a lane carries at each of
+// the first log2(2N) butterfly steps (N = E rounded up to a power of two), so
+// after the five steps the block of 32 / (2N) consecutive lanes starting at
+// lane j 32 / (2N) holds sum j: lanes 0-15 the sums of a0, lanes 16-31 those
+// of a1.  The max over the blocks of each half follows.  The summation order
+// differs from a plain butterfly; the callers' margins cover any order.
 template <int E>
 __device__ __forceinline__ void warp_max_of_sums2(const double (&a0)[E], const double (&a1)[E], int lane, double &m0,
                                                   double &m1)
