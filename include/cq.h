@@ -32,7 +32,7 @@
  *  - Results are deterministic: the same inputs give the same output bytes.
  *  - Non-finite or negative inputs never trap: the affected group gets scale
  *    0x0001 and all codes 0 (nibble 8), and the NONFINITE counter and flag are
- *    set; cq_read_counters() reports it as CQ_ERR_NONFINITE.
+ *    set; cq_get_status() and cq_read_counters() report it as CQ_ERR_NONFINITE.
  */
 #ifndef CQ_H
 #define CQ_H
@@ -272,6 +272,12 @@ cq_status cq_select_scales_noalloc(const uint16_t *W, int64_t G, const float *D,
  * memory).  Synchronises `stream`.  Returns CQ_ERR_NONFINITE when the last
  * call saw non-finite input, else CQ_OK (or CQ_ERR_CUDA / CQ_ERR_INVALID_ARG). */
 cq_status cq_read_counters(const void *workspace, uint32_t *host_counters, void *stream);
+
+/* Status of the last call that used `workspace`: synchronises `stream`, then
+ * returns CQ_ERR_NONFINITE when that call saw non-finite or negative input,
+ * CQ_ERR_CUDA when the stream reports an error, CQ_ERR_INVALID_ARG for a null
+ * workspace, else CQ_OK.  The same as cq_read_counters without the counts. */
+cq_status cq_get_status(const void *workspace, void *stream);
 
 /* Static, human-readable name of a status code. */
 const char *cq_status_string(cq_status status);

@@ -29,7 +29,7 @@ MAX_E = 8
 EXPORTS = ("cq_workspace_bytes", "cq_select_scales", "cq_select_scales_ex", "cq_select_scales_host",
            "cq_absmax_scales", "cq_pool_diagonals", "cq_group_objective", "cq_reconstruction_proxy",
            "cq_gptq_export", "cq_gptq_dequantize", "cq_estimate_diagonals", "cq_select_scales_spec",
-           "cq_select_scales_noalloc", "cq_read_counters", "cq_status_string", "cq_version")
+           "cq_select_scales_noalloc", "cq_read_counters", "cq_get_status", "cq_status_string", "cq_version")
 
 
 class CQError(RuntimeError):
@@ -86,6 +86,8 @@ def _load():
     L.cq_select_scales_noalloc.argtypes = [vp, i64, vp, i32, i64, vp, vp, vp]
     L.cq_read_counters.restype = i32
     L.cq_read_counters.argtypes = [vp, vp, vp]
+    L.cq_get_status.restype = i32
+    L.cq_get_status.argtypes = [vp, vp]
     L.cq_status_string.restype = ctypes.c_char_p
     L.cq_status_string.argtypes = [i32]
     L.cq_version.restype = i32
@@ -485,6 +487,15 @@ def read_counters(workspace, stream=None) -> dict:
     if st not in (CQ_OK, CQ_ERR_NONFINITE):
         raise CQError(st, "cq_read_counters")
     return {n: int(v) for n, v in zip(COUNTER_NAMES, host)}
+
+
+def get_status(workspace, stream=None) -> int:
+    """Synchronises ``stream``; CQ_OK, or CQ_ERR_NONFINITE when the last call
+    on ``workspace`` saw non-finite or negative input."""
+    st = lib.cq_get_status(_ptr(workspace), _stream_handle(stream))
+    if st not in (CQ_OK, CQ_ERR_NONFINITE):
+        raise CQError(st, "cq_get_status")
+    return st
 
 
 def to_numpy_bits(res: Result):

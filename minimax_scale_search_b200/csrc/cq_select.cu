@@ -1788,6 +1788,12 @@ cq_status cq_read_counters(const void *workspace, uint32_t *host_counters, void 
     return host_counters[CQ_CNT_NONFINITE] ? CQ_ERR_NONFINITE : CQ_OK;
 }
 
+cq_status cq_get_status(const void *workspace, void *stream)
+{
+    uint32_t counters[CQ_NUM_COUNTERS];
+    return cq_read_counters(workspace, counters, stream);
+}
+
 const char *cq_status_string(cq_status status)
 {
     switch (status) {

@@ -96,6 +96,7 @@ def test_plain_and_host_entry_points_validate(cq):
         cq.CQ_ERR_INVALID_ARG
     assert cq.lib.cq_select_scales_host(vp(None), 0, vp(None), 4, 0, vp(None), vp(None), vp(None)) == cq.CQ_OK
     assert cq.lib.cq_read_counters(vp(None), vp(FAKE), vp(None)) == cq.CQ_ERR_INVALID_ARG
+    assert cq.lib.cq_get_status(vp(None), vp(None)) == cq.CQ_ERR_INVALID_ARG
 
 
 def test_policy_entry_points_validate(cq):

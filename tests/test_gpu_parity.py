@@ -163,6 +163,10 @@ def test_nonfinite_inputs_are_flagged_not_trapped():
     st = cq.lib.cq_read_counters(ctypes.c_void_p(res.workspace.data_ptr()), ctypes.c_void_p(host.ctypes.data),
                                  ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == cq.CQ_ERR_NONFINITE and host[2] == 5
+    assert cq.get_status(res.workspace) == cq.CQ_ERR_NONFINITE
+    # a finite call on the same workspace resets the status
+    res2 = cq.select_scales(Wt[5:6].contiguous(), Dt[:, 5:6].contiguous(), workspace=res.workspace)
+    assert cq.get_status(res2.workspace) == cq.CQ_OK
 
 
 def test_exhaustive_path_matches_oracle_bit_for_bit():
