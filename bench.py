@@ -74,6 +74,30 @@ def peaks():
     return p32, p64, mhz, f"148 SMs x {FP32_LANES} FP32 / {FP64_LANES} FP64 lanes x 2 x {mhz:.0f} MHz ({src})"
 
 
+def objective_roofline(G: int, E: int, ms: float, hbm: float, hsrc: str = "") -> dict:
+    """Roofline of the objective of given scales over G groups in `ms`: the
+    slower of its bytes (256 + 2 + 8E + 8 per group) at the HBM peak `hbm`
+    (GB/s) and its fp64 operations at one per FP64 lane per clock.  The
+    definition fixes 2 + 2E of them per weight: r = w - s q, r*r, and d*rr plus
+    the running sum for each environment."""
+    bpg = 256 + 2 + 8 * E + 8
+    byt = G * bpg
+    ops = G * 128 * (2 + 2 * E)
+    _, _, mhz, csrc = peaks()
+    p64ops = SMS * FP64_LANES * mhz * 1e6 / 1e12  # T operations/s
+    hbm_gbs = byt / ms / 1e6
+    ops_t = ops / ms / 1e9
+    if ops / (p64ops * 1e12) >= byt / (hbm * 1e9):  # the fp64 pipe binds
+        roof = {"bound": "alu", "achieved": ops_t, "peak": p64ops, "unit": "Top/s (fp64 operations)",
+                "frac": ops_t / p64ops, "hbm_achieved_gbs": hbm_gbs, "hbm_frac": hbm_gbs / hbm,
+                "peak_note": f"{SMS} SMs x {FP64_LANES} FP64 lanes x {mhz:.0f} MHz ({csrc})"}
+    else:
+        roof = {"bound": "hbm", "achieved": hbm_gbs, "peak": hbm, "unit": "GB/s", "frac": hbm_gbs / hbm,
+                "alu_frac": ops_t / p64ops, "peak_note": hsrc}
+    roof.update({"bytes_per_group": bpg, "fp64_ops": ops})
+    return roof
+
+
 def kernel_source_hash() -> str:
     """Hash of the main kernel's sources (its file and the device header it includes)."""
     h = hashlib.sha256()
@@ -334,24 +358,9 @@ def bench_policies(args, wl, W, D, Wd, Dd, dev):
     obj = torch.empty(G, dtype=torch.float64, device=dev)
     ms = time_calls(lambda: cq.group_objective(Wd, Dd, scales, wl.cols, per_env=per_env, out=obj), args.steps,
                     args.warmup, stream)
-    bpg = 256 + 2 + 8 * wl.E + 8
-    byt = G * bpg
-    # The definition fixes 2 + 2E fp64 operations per weight (r = w - s q, r*r,
-    # and d*rr plus the running sum per environment), each one FP64 lane-clock.
-    ops = G * 128 * (2 + 2 * wl.E)
-    _, _, mhz, csrc = peaks()
-    p64ops = SMS * FP64_LANES * mhz * 1e6 / 1e12
-    hbm_gbs = byt / ms / 1e6
-    ops_t = ops / ms / 1e9
-    if ops / p64ops >= byt / hbm * 1e3:  # the fp64 pipe binds
-        roof = {"bound": "alu", "achieved": ops_t, "peak": p64ops, "unit": "Top/s (fp64 operations)",
-                "frac": ops_t / p64ops, "hbm_achieved_gbs": hbm_gbs, "hbm_frac": hbm_gbs / hbm,
-                "peak_note": f"{SMS} SMs x {FP64_LANES} FP64 lanes x {mhz:.0f} MHz ({csrc})"}
-    else:
-        roof = {"bound": "hbm", "achieved": hbm_gbs, "peak": hbm, "unit": "GB/s", "frac": hbm_gbs / hbm,
-                "alu_frac": ops_t / p64ops, "peak_note": hsrc}
+    roof = objective_roofline(G, wl.E, ms, hbm, hsrc)
     roof.update({"traffic": recorded_kernel_traffic("objective_kernel<4,", G),
-                 "kernel": "objective_kernel<4, per-column>", "bytes_per_group": bpg, "fp64_ops": ops})
+                 "kernel": "objective_kernel<4, per-column>"})
     lines.append(dict(base, metric="objective of given scales groups/sec", op="objective", value=G / ms * 1e3,
                       unit="groups/s", ms_per_step=ms, higher_is_better=True, dtype="f64",
                       gpu_launches=2 * args.steps, roofline=roof))

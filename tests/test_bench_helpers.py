@@ -45,3 +45,19 @@ def test_peaks_and_job_rate():
     assert abs(p64 - p32 / 2) < 1e-9
     # whole-job rate: all ranks' units over the slowest rank's time
     assert bench.job_rate(8, 1000, 0.5) == 16000.0
+
+
+def test_objective_roofline_picks_the_binding_bound():
+    p32, p64, mhz, _ = bench.peaks()
+    ops_peak = 148 * 64 * mhz * 1e6 / 1e12  # fp64 operations per second, T
+    G, E = 3_883_008, 4
+    # 10 fp64 operations per weight at E = 4, 298 bytes per group
+    r = bench.objective_roofline(G, E, 0.774, 6525.0)
+    assert r["fp64_ops"] == G * 128 * 10 and r["bytes_per_group"] == 298
+    assert r["bound"] == "alu"  # 0.267 ms of fp64 issue against 0.177 ms of HBM
+    assert abs(r["peak"] - ops_peak) < 1e-9
+    assert abs(r["frac"] - G * 1280 / 0.774e-3 / (ops_peak * 1e12)) < 1e-12
+    assert abs(r["hbm_frac"] - G * 298 / 0.774e-3 / 6525e9) < 1e-12
+    # with a slow memory the bytes bind instead
+    r2 = bench.objective_roofline(G, E, 0.774, 1000.0)
+    assert r2["bound"] == "hbm" and abs(r2["frac"] - G * 298 / 0.774e-3 / 1000e9) < 1e-12
