@@ -269,6 +269,7 @@ struct WarpSmem {
     float d[E][kGroup];       // diagonals by rank in ascending |w|
     float w[kGroup];          // signed weights by rank in ascending |w|
     uint8_t negpre[kGroup + 4];  // number of negative weights below each rank
+    uint8_t negidx[kGroup];      // rank of each negative weight, by its rank among negatives
     int lay[32];                 // window rank range of each transition layer; rank thresholds
     // A: transition layers -> level-2 lists -> per-run fp32 lower bounds ->
     //    survivor ranges + survivor results
@@ -651,7 +652,10 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
             sm.d[e][r] = dv_g.base[e * dv_g.stride + i];
         const bool neg = (k >> 7) != 0u && (bits & 0x8000u) != 0u;
         const unsigned bn = __ballot_sync(kFull, neg);
-        sm.negpre[r] = static_cast<uint8_t>(n7 + __popc(bn & ((1u << lane) - 1u)));
+        const int np = n7 + __popc(bn & ((1u << lane) - 1u));
+        sm.negpre[r] = static_cast<uint8_t>(np);
+        if (neg)
+            sm.negidx[np] = static_cast<uint8_t>(r);
         n7 += __popc(bn);
     }
     if (lane == 0)
@@ -856,14 +860,11 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         const int r = 32 * m + lane;
         const float wv = sm.w[r];
         const float aw = fabsf(wv);
-        // |q| at s_J0 and s_J1: the layers whose rank threshold r has passed
+        // |q| at s_J1: the layers whose rank threshold r has passed
         int ktop = (wv < 0.0f && r >= th[15]) ? 1 : 0;
-        int kbot = (wv < 0.0f && r >= th[7]) ? 1 : 0;
 #pragma unroll
-        for (int k = 0; k < 7; k++) {
+        for (int k = 0; k < 7; k++)
             ktop += r >= th[8 + k];
-            kbot += r >= th[k];
-        }
         const float fk = static_cast<float>(ktop);
 #pragma unroll
         for (int e = 0; e < E; e++) {
@@ -871,10 +872,30 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
             bb[e] = fmaf(dd, aw * fk, bb[e]);
             bc[e] = fmaf(dd, fk * fk, bc[e]);
         }
-        const uint32_t rb = static_cast<uint32_t>(r) << 3;
-        for (int k = ktop; k < kbot; k++) {
-            const int at = (k == 7) ? static_cast<int>(sm.negpre[r]) - off[7] : r - off[k];
-            layer[k * kLayerStride + at] = (transition_index(aw, k) << 10) | rb | static_cast<uint32_t>(k);
+    }
+    // The in-window transitions, layer after layer, spread evenly over the
+    // lanes: item t of layer k is its (t - pre_k)-th rank in the layer's range.
+    {
+        int pre[9];
+        pre[0] = 0;
+#pragma unroll
+        for (int k = 0; k < 8; k++)
+            pre[k + 1] = pre[k] + (off[k + 8] - off[k]);
+#pragma unroll 1
+        for (int t = lane; t < pre[8]; t += 32) {
+            int k = 0, base = 0;
+#pragma unroll
+            for (int kk = 1; kk < 8; kk++) {
+                if (t >= pre[kk]) {
+                    k = kk;
+                    base = pre[kk];
+                }
+            }
+            const int at = t - base;
+            const int r = (k == 7) ? static_cast<int>(sm.negidx[off[7] + at]) : off[k] + at;
+            const float aw = fabsf(sm.w[r]);
+            layer[k * kLayerStride + at] =
+                (transition_index(aw, k) << 10) | (static_cast<uint32_t>(r) << 3) | static_cast<uint32_t>(k);
         }
     }
     if (lane < 8)
