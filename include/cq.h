@@ -112,7 +112,9 @@ cq_status cq_select_scales(const uint16_t *W, int64_t G, const float *D, int E, 
  *  out_objective  nullable, fp64 [G]: the objective at the chosen scale.
  *  out_flags      nullable, uint8 [G]: CQ_FLAG_* bits.
  * The workspace counters are reset at the start of every call.  Calls that
- * share a workspace must be ordered on one stream. */
+ * share a workspace must be ordered on one stream.  The call only enqueues
+ * work on `stream` (no allocation, no host synchronisation), so it can be
+ * captured in a CUDA graph and replayed on new contents of the same buffers. */
 cq_status cq_select_scales_ex(const uint16_t *W, int64_t G, const float *D, int E, int64_t K,
                               uint16_t *out_scales, uint32_t *out_codes, void *stream,
                               const cq_opts *opts, void *workspace, size_t workspace_bytes,
