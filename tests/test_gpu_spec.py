@@ -60,7 +60,7 @@ def test_other_code_ranges(spec):
     _check(W, D, qmin, qmax, 128, where=f"spec {spec}")
 
 
-@pytest.mark.parametrize("n,E", [(1, 2), (32, 1), (64, 4), (100, 3), (256, 8), (1024, 2)])
+@pytest.mark.parametrize("n,E", [(1, 2), (32, 1), (64, 4), (100, 3), (256, 8), (1024, 2), (1024, 8)])
 def test_other_group_sizes(n, E):
     G = max(8, 4096 // n)
     W = _groups(G, n, seed=n)
