@@ -59,8 +59,9 @@ namespace cq {
 // code is ~110 KB; with independent CTAs per SM, instruction fetch was the top
 // stall).  20 warps of <= 96 registers fit the register file for E <= 4;
 // larger E needs more shared memory per warp and up to 128 registers: 16.
+// E = 1 needs at most 89 registers and less shared memory, so 23 warps fit.
 template <int E>
-constexpr int kWarpsPerCta = E <= 4 ? 20 : 16;
+constexpr int kWarpsPerCta = E == 1 ? 23 : (E <= 4 ? 20 : 16);
 constexpr uint32_t kInvalidKey = 0xFFFFFFFFu;
 constexpr int kMaxFinalists = 64;
 constexpr int kDefaultFinalists = 32;
