@@ -154,9 +154,11 @@ cq_status cq_pool_diagonals(const float *D, int E, int64_t n, float *out, void *
 /* Objective of given scales (the proxy's per-group term): per_env[g*E + e] =
  * sum_i d_{e,i} (w_i - s q_i(s))^2 in fp64, summed over i ascending without
  * fused multiply-adds, and out_objective[g] = max_e of those; s = scales[g]
- * (binary16 bits).  W and D as for cq_select_scales (both 16-byte aligned);
- * per_env [G][E] and out_objective [G] are fp64 and 8-byte aligned.  The
- * result is undefined for non-finite input. */
+ * (binary16 bits, a positive finite pattern 0x0001..0x7BFF).  W and D as for
+ * cq_select_scales (both 16-byte aligned); per_env [G][E] and out_objective
+ * [G] are fp64 and 8-byte aligned.  The values are unspecified for non-finite
+ * input or other scale patterns; the kernel reads and writes only the
+ * buffers above either way. */
 cq_status cq_group_objective(const uint16_t *W, int64_t G, const float *D, int E, int64_t K,
                              const uint16_t *scales, double *per_env, double *out_objective,
                              void *stream);
