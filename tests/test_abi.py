@@ -208,3 +208,17 @@ def test_no_cpu_fallback_in_binding():
             assert "import oracle" not in src and "from oracle" not in src, name
     src = open(os.path.join(pkg, "cq.py")).read()
     assert "raise ImportError" in src
+
+
+def test_binding_raises_without_its_library(tmp_path):
+    """Imported from a directory without libcq.so, the binding raises at import
+    instead of running anything on the CPU."""
+    import importlib.util
+    import shutil
+    src = os.path.join(ROOT, "minimax_scale_search_b200", "cq.py")
+    dst = tmp_path / "cq_copy.py"
+    shutil.copy(src, dst)
+    spec = importlib.util.spec_from_file_location("cq_copy_without_library", dst)
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError, match="libcq.so"):
+        spec.loader.exec_module(mod)
