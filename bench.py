@@ -200,6 +200,18 @@ def max_over_ranks(values, dist=None, device=None):
     return [float(v) for v in t.cpu()]
 
 
+def sum_over_ranks(counts: dict, dist=None, device=None) -> dict:
+    """Per-key sum of integer counters over ranks (every rank solves its own
+    matrix, so the job's counts are the sums)."""
+    if dist is None:
+        return {k: int(v) for k, v in counts.items()}
+    import torch
+    keys = sorted(counts)
+    t = torch.tensor([int(counts[k]) for k in keys], dtype=torch.int64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return {k: int(v) for k, v in zip(keys, t.cpu())}
+
+
 def job_rate(world: int, groups_per_rank: int, seconds: float) -> float:
     """Whole-job groups per second: every rank's groups over the slowest rank's time."""
     return world * groups_per_rank / seconds
@@ -566,7 +578,7 @@ def main():
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    counters = cq.read_counters(ws)
+    counters = sum_over_ranks(cq.read_counters(ws), dist, dev)  # one call per rank, summed over the job
 
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]

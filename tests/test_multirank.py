@@ -33,9 +33,10 @@ def _worker(rank, world, port, out):
         m = bench.rank_matrix(rank)
         W = synth.make_weights(5, 0, 4, matrix=m)  # first rows of this rank's matrix
         times = bench.max_over_ranks([10.0 + rank, 3.0 - rank], dist, "cpu")
+        counts = bench.sum_over_ranks({"fallback": rank + 1, "near_tie": 10 * rank}, dist, "cpu")
         dist.barrier()
         out[rank] = (m, int(W.astype(np.int64).sum()), times[0], times[1],
-                     bench.job_rate(world, 1000, times[0]))
+                     bench.job_rate(world, 1000, times[0]), counts)
     finally:
         dist.destroy_process_group()
 
@@ -51,7 +52,8 @@ def test_two_gloo_ranks_shard_and_take_max():
     for p in procs:
         p.join(120)
         assert p.exitcode == 0
-    (m0, s0, t0a, t0b, v0), (m1, s1, t1a, t1b, v1) = out[0], out[1]
+    (m0, s0, t0a, t0b, v0, c0), (m1, s1, t1a, t1b, v1, c1) = out[0], out[1]
     assert (m0, m1) == (0, 1) and s0 != s1          # different matrices per rank
     assert t0a == t1a == 11.0 and t0b == t1b == 3.0  # max over ranks, identical on every rank
     assert v0 == v1 == 2 * 1000 / 11.0
+    assert c0 == c1 == {"fallback": 3, "near_tie": 10}  # counters summed over ranks
