@@ -8,36 +8,45 @@
 // with an exact tie going to the lower bit pattern, and emit the codes packed
 // as (q+8) nibbles, 8 per uint32, low nibble first.
 //
-// Design (one warp per group, persistent grid of one CTA per SM whose 16-20
+// Design (one warp per group, persistent grid of one CTA per SM whose 16-23
 // warps start each group together; no tensor cores: the work is comparisons
-// and short fp64 dot products, not a dense contraction):
+// and short fp32/fp64 evaluations, not a dense contraction):
 //
-//  1. Load: 8-byte weight loads and 16-byte diagonal loads per lane; the
-//     group's w and d are staged in shared memory for indexed access.
-//  2. Code transitions ("candidates induced by code transitions"): weight i
-//     changes |q_i| from k+1 to k at the smallest grid index t_{i,k} where
-//     |w_i| < s (k + 1/2) (or equality with k even).  t is found from an fp32
-//     estimate and fixed by exact fp32 threshold tests (s * (k + 1/2) has at
-//     most 16 significant bits, so the product is exact).
-//  3. Ordering: the <= 1024 keys (t, i, k) are bitonic-sorted in registers.
-//  4. Coefficient scan: on a run of constant codes F_e(s) = A_e - 2 B_e s +
-//     C_e s^2 with B_e = sum d|w||q|, C_e = sum d q^2 ("quadratic"); B and C
-//     are exact-term fp64 suffix sums over the sorted transitions.
-//  5. Per run: max_e F_e is convex in s, so the leftmost grid minimiser is
-//     found by a binary search on the sign of f(s_{j+1}) - f(s_j).  Every
-//     comparison is certified against a rigorous bound on the fp64 evaluation
-//     error (2^-44 of sum_e-max of A + 2Bs + Cs^2); a run with an uncertified
-//     comparison falls back to a lower bound from its quadratic vertices
-//     ("quadratic vertices"), and the group goes to the exhaustive pass if
-//     that run could still hold the minimum.
-//  6. Finalists: the runs whose certified lower bound is within 2^-40 of the
-//     best certified upper bound; each is rescored with the direct fp64
-//     objective (exact codes, exact residuals) and the (objective, pattern)
-//     minimum wins.
-//  7. Exhaustive fallback (the page's conservative exhaustive-grid check):
-//     queued groups are solved over all 31,743 scales in the definition's
-//     own fp64 evaluation order by a second kernel, one CTA per group.
-//  8. Pack: each lane packs 4 codes; pairs of lanes form one uint32.
+//  1. Load: 8-byte weight and 16-byte diagonal loads per lane; A_e = sum d w^2
+//     in fp64.  Non-finite input is flagged, all-zero groups are trivial, and a
+//     nonzero d outside [2^-64, 2^81] (where the fp32 steps' error bounds could
+//     fail) sends the group to the exhaustive pass.
+//  2. Weights sorted by |w| (bitonic, 4 keys per lane); w, d staged by rank.
+//  3. U, an upper bound of the minimum, from the fp32 objective at three grid
+//     scales near the AbsMax scale.
+//  4. A certified window [J0, J1] of grid indices that can hold the minimum:
+//     below it the clipping error of the largest weights, above it the error
+//     of the weights in the dead zone, exceeds U.
+//  5. Code transitions inside the window ("candidates induced by code
+//     transitions"): weight i changes |q_i| from k+1 to k at the smallest grid
+//     index t_{i,k} where |w_i| < s (k + 1/2) (or equality with k even), from an
+//     fp32 estimate fixed by exact fp32 threshold tests.  With ranks in
+//     ascending |w| each code layer k is a rank range, so each layer's list is
+//     already sorted; the 8 layers are merged (merge path, 3 levels).
+//  6. fp32 screen: on a run of constant codes F_e(s) = A_e - 2 B_e s + C_e s^2
+//     ("quadratic"); suffix sums give B, C per run, and each run gets a lower
+//     bound (max over e at the clamped vertices, "quadratic vertices") and an
+//     upper bound, widened by a proved rounding margin.  Runs whose lower bound
+//     reaches the best upper bound survive.
+//  7. Survivors, fp64: exact coefficients (a direct warp sum, then exact
+//     delta walks); max_e F_e is convex on a run, so a certified strict local
+//     minimum at the vertex guess ends the search, else a binary search on the
+//     sign of f(s_{j+1}) - f(s_j).  Every comparison is certified against a
+//     bound on the fp64 evaluation error; an uncertified run that could still
+//     hold the minimum sends the group to the exhaustive pass.
+//  8. Finalists: runs whose certified lower bound is within 2^-40 of the best
+//     certified upper bound, rescored with the direct fp64 objective (exact
+//     codes, exact residuals); the (objective, pattern) minimum wins.
+//  9. Exhaustive fallback (the page's conservative exhaustive-grid check):
+//     queued groups are solved over their window (all 31,743 scales when
+//     forced or out of range) in the definition's own fp64 evaluation order by
+//     a second kernel, one CTA per group.
+// 10. Pack: each lane packs 4 codes; pairs of lanes form one uint32.
 
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
