@@ -21,6 +21,7 @@ namespace cq {
 namespace {
 
 constexpr int kStageWarps = 4;   // warps per CTA of the staged kernels
+constexpr int kStageCtas = 6;    // AbsMax: CTAs per SM its shared-memory staging allows (registers capped to fit)
 constexpr int kRowPitch = 272;   // bytes per staged 256-byte row: the 16-byte pad puts the 16-byte reads
                                  // of 8 consecutive rows (one shared-memory phase) on disjoint banks
 constexpr int kStageBytes = 32 * kRowPitch;
@@ -77,7 +78,7 @@ __device__ __forceinline__ int code_of(float aw, float s, float inv, int cap)
 // the quantiser's at s.  Non-finite weights give scale 0x0001 and zero codes,
 // as in the minimax kernel.  One thread per group; each warp stages 32
 // consecutive groups and writes their codes back as contiguous 16-byte stores.
-__global__ void __launch_bounds__(kStageWarps * 32) absmax_kernel(const uint16_t *__restrict__ W, int64_t G,
+__global__ void __launch_bounds__(kStageWarps * 32, kStageCtas) absmax_kernel(const uint16_t *__restrict__ W, int64_t G,
                                                                   uint16_t *__restrict__ out_scales,
                                                                   uint32_t *__restrict__ out_codes)
 {
