@@ -92,16 +92,39 @@ __global__ void __launch_bounds__(kTile * kTileRowsPerPass) dequant_kernel(const
     const int64_t tiles_r = (R + kTile - 1) / kTile;
     const int64_t tiles = ((K8 + kTile - 1) / kTile) * tiles_r;
     const int tx = threadIdx.x, ty = threadIdx.y;
+    // fp16 output: each thread's words of the next tile are loaded into
+    // registers while the current tile is dequantised and stored (the fp32
+    // output, twice the bytes per word, was faster without it)
+    constexpr int kPer = kTile / kTileRowsPerPass;
+    uint32_t nxt[kPer];
+    auto load = [&](int64_t t) {
+        const int64_t k0 = (t / tiles_r) * kTile, r0 = (t % tiles_r) * kTile;
+#pragma unroll
+        for (int k = 0; k < kPer; k++) {
+            const int64_t kk = k0 + ty + k * kTileRowsPerPass, r = r0 + tx;
+            nxt[k] = (kk < K8 && r < R) ? qweight[kk * R + r] : 0u;
+        }
+    };
+    if (kHalf && static_cast<int64_t>(blockIdx.x) < tiles)
+        load(blockIdx.x);
     for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
         const int64_t k0 = (t / tiles_r) * kTile, r0 = (t % tiles_r) * kTile;
         __syncthreads();
+        if (kHalf) {
 #pragma unroll
-        for (int k = 0; k < kTile; k += kTileRowsPerPass) {
-            const int64_t kk = k0 + ty + k, r = r0 + tx;
-            if (kk < K8 && r < R)
-                tile[ty + k][tx] = qweight[kk * R + r];
+            for (int k = 0; k < kPer; k++)
+                tile[ty + k * kTileRowsPerPass][tx] = nxt[k];
+        } else {
+#pragma unroll
+            for (int k = 0; k < kTile; k += kTileRowsPerPass) {
+                const int64_t kk = k0 + ty + k, r = r0 + tx;
+                if (kk < K8 && r < R)
+                    tile[ty + k][tx] = qweight[kk * R + r];
+            }
         }
         __syncthreads();
+        if (kHalf && t + gridDim.x < tiles)
+            load(t + gridDim.x);
         const int64_t kk = k0 + tx;
         if (kk >= K8)
             continue;
