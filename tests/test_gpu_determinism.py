@@ -3,7 +3,8 @@ bytes.  The selection queues fallback groups with an atomic counter and its
 warps finish in any order, so repeat it on a sample of the tie/stress workload
 (near ties, exact fits, zero groups, E = 8), on a second stream while another
 selection runs, and through the general-spec path.  Every output byte must
-match: scales, codes, objectives, flags and the counters."""
+match: scales, codes, objectives, flags and the counters.  Row blocks solved
+separately (as the ranks of a multi-GPU run do) concatenate to the whole."""
 import numpy as np
 import pytest
 
@@ -65,3 +66,21 @@ def test_general_spec_is_deterministic():
     torch.cuda.synchronize()
     ref = _bytes(runs[0])
     assert all(_bytes(r) == ref for r in runs[1:])
+
+
+def test_sharded_runs_concatenate_to_the_whole():
+    """Groups are independent: solving row blocks of a matrix separately (as
+    the ranks of a multi-GPU run do) and concatenating gives the whole
+    matrix's output byte for byte."""
+    import torch
+    from minimax_scale_search_b200 import cq
+    W, D = synth.make_inputs(2)  # 3,072 x 1,024, per-column diagonals
+    Wt = torch.from_numpy(W.view(np.int16)).cuda()
+    Dt = torch.from_numpy(D).cuda()
+    whole = _bytes(cq.select_scales(Wt, Dt, want_objective=True, want_flags=True))
+    for bounds in ((0, 1536, 3072), (0, 1000, 2048, 3071, 3072)):
+        parts = [cq.select_scales(Wt[a:b].contiguous(), Dt, want_objective=True, want_flags=True)
+                 for a, b in zip(bounds[:-1], bounds[1:])]
+        torch.cuda.synchronize()
+        joined = [b"".join(_bytes(p)[k] for p in parts) for k in range(4)]
+        assert joined == whole, bounds
