@@ -61,3 +61,23 @@ def test_objective_roofline_picks_the_binding_bound():
     # with a slow memory the bytes bind instead
     r2 = bench.objective_roofline(G, E, 0.774, 1000.0)
     assert r2["bound"] == "hbm" and abs(r2["frac"] - G * 298 / 0.774e-3 / 1000e9) < 1e-12
+
+
+def test_traffic_records_parse_and_match_their_summaries():
+    """The committed ncu records the benchmark reads: well formed, positive,
+    and the main kernel's hash is the one its profile summary cites."""
+    prof = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "profiles")
+    kv = dict(t.split("=", 1) for t in open(os.path.join(prof, "select_kernel_traffic.txt")).read().split())
+    assert int(kv["groups"]) > 0 and int(kv["dram_bytes"]) > 0
+    assert len(kv["kernel_sha"]) == 16
+    assert kv["kernel_sha"] in open(os.path.join(prof, kv["capture"])).read()
+    # bytes per group near the algorithmic 322 (some output still in L2): a sanity range
+    assert 250 <= int(kv["dram_bytes"]) / int(kv["groups"]) <= 340
+    names = set()
+    for ln in open(os.path.join(prof, "secondary_kernels_traffic.txt")).read().splitlines():
+        rec = dict(t.split("=", 1) for t in ln.split() if "=" in t)
+        assert {"kernel", "src", "sha", "units", "dram_bytes"} <= set(rec), ln
+        assert int(rec["units"]) > 0 and int(rec["dram_bytes"]) > 0
+        assert os.path.exists(os.path.join(os.path.dirname(prof), "minimax_scale_search_b200", "csrc", rec["src"]))
+        names.add(rec["kernel"])
+    assert {"absmax_kernel", "objective_kernel<4,", "spec_kernel<4>"} <= names
