@@ -41,7 +41,9 @@
 //     hold the minimum sends the group to the exhaustive pass.
 //  8. Finalists: runs whose certified lower bound is within 2^-40 of the best
 //     certified upper bound, rescored with the direct fp64 objective (exact
-//     codes, exact residuals); the (objective, pattern) minimum wins.
+//     codes, exact residuals); the (objective, pattern) minimum wins.  A single
+//     finalist is the answer by itself and is rescored only when the caller
+//     asks for the objective.
 //  9. Exhaustive fallback (the page's conservative exhaustive-grid check):
 //     queued groups are solved over their window (all 31,743 scales when
 //     forced or out of range) in the definition's own fp64 evaluation order by
@@ -1219,8 +1221,16 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     // ---- 9. fp64 rescoring of the finalists (lane L takes ranks 32m + L) -------
     double best = INFINITY, second = INFINITY;
     uint32_t bj = 0;
+    // One finalist is the minimum by itself: its fp64 objective is only an
+    // output, so it is computed when requested.  (best = 0 with second
+    // infinite is never a near tie, as with a rescored single finalist.)
+    const bool only = total == 1 && p.out_obj == nullptr;
+    if (only) {
+        bj = static_cast<uint32_t>(fin[0]);
+        best = 0.0;
+    }
 #pragma unroll 1
-    for (int f = 0; f < total; f++) {
+    for (int f = 0; f < (only ? 0 : total); f++) {
         const uint32_t j = static_cast<uint32_t>(fin[f]);
         const float s = grid_value(j);
         const double sd = s;
