@@ -8,8 +8,10 @@ inputs already resident in HBM.  Prints one JSON line (rank 0).
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cq|reference]
 
 N > 1 runs under torch.distributed (one process per GPU, NCCL used only for
-the barrier and the max-over-ranks time): every rank solves its own matrix of
-the same workload, so per-GPU work is fixed (weak scaling).
+the barrier and the max-over-ranks time): the sweep's 30,336 rows split into
+contiguous blocks of whole rows, one per rank, each rank holding the whole
+[4, 16384] diagonal set, so the job is the same 3,883,008 groups at every N
+(strong scaling) and no data crosses between ranks.
 The reference arm (--impl reference) times the exhaustive CPU oracle on the
 host cores over bounded samples of the same workload.
 """
@@ -185,11 +187,6 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(inside)}
 
 
-def rank_matrix(rank: int) -> int:
-    """Each rank solves its own matrix of the workload (weak scaling, no data exchange)."""
-    return rank
-
-
 def max_over_ranks(values, dist=None, device=None):
     """Elementwise max of per-rank timings (the job's time is its slowest rank)."""
     if dist is None:
@@ -212,9 +209,9 @@ def sum_over_ranks(counts: dict, dist=None, device=None) -> dict:
     return {k: int(v) for k, v in zip(keys, t.cpu())}
 
 
-def job_rate(world: int, groups_per_rank: int, seconds: float) -> float:
+def job_rate(groups_total: int, seconds: float) -> float:
     """Whole-job groups per second: every rank's groups over the slowest rank's time."""
-    return world * groups_per_rank / seconds
+    return groups_total / seconds
 
 
 def gpu_index_for(local_rank: int) -> str:
@@ -548,16 +545,18 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
 
-    from minimax_scale_search_b200 import cq
+    from minimax_scale_search_b200 import cq, shard
     if args.op in ("gptq", "diag", "spec"):
         if world > 1:
             ap.error(f"--op {args.op} runs on one GPU")
         {"gptq": bench_gptq, "diag": bench_diag, "spec": bench_spec}[args.op](args, wl, dev)
         return
-    W = synth.make_weights(WORKLOAD, matrix=rank_matrix(rank))
-    D = synth.make_diagonals(WORKLOAD, matrix=rank_matrix(rank))
+    r0, r1 = shard.row_block(rank, world, wl.rows)
+    W = synth.make_weights(WORKLOAD, r0, r1)
+    D = synth.make_diagonals(WORKLOAD)
     Wg = W.reshape(-1, 128)
     G = Wg.shape[0]
+    G_job = wl.groups_per_matrix
     f32, f64 = counted_flops(Wg, wl.E)
     Wd = torch.from_numpy(W.view(np.int16)).to(dev)
     Dd = torch.from_numpy(D).to(dev)
@@ -599,10 +598,10 @@ def main():
         dist.barrier()
     clocks = sampler.stop(w0, w1)
     ms_total = t_start.elapsed_time(t_end)
-    kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
-    ms_total, kernel_ms = max_over_ranks([ms_total, kernel_ms], dist, dev)
+    kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)  # this rank's own launches
+    ms_total = max_over_ranks([ms_total], dist, dev)[0]
     ms_step = ms_total / args.steps
-    value = job_rate(world, G, ms_step / 1e3)
+    value = job_rate(G_job, ms_step / 1e3)
 
     # ---- end to end through the host-buffer entry point (pinned host memory)
     e2e = None
@@ -623,8 +622,9 @@ def main():
         e2e_s = max_over_ranks([(time.perf_counter() - t0) / n_e2e], dist, dev)[0]
         dev_s = out_s.cpu().numpy().view(np.uint16)
         assert np.array_equal(dev_s, sn), "host entry point disagrees with the device entry point"
-        e2e = {"value": job_rate(world, G, e2e_s), "unit": "groups/s", "h2d_bytes_per_step": int(W.nbytes + D.nbytes),
-               "d2h_bytes_per_step": int(sn.nbytes + cn.nbytes), "ms_per_step": 1e3 * e2e_s, "steps": n_e2e}
+        io = sum_over_ranks({"h2d": W.nbytes + D.nbytes, "d2h": sn.nbytes + cn.nbytes}, dist, dev)
+        e2e = {"value": job_rate(G_job, e2e_s), "unit": "groups/s", "h2d_bytes_per_step": io["h2d"],
+               "d2h_bytes_per_step": io["d2h"], "ms_per_step": 1e3 * e2e_s, "steps": n_e2e}
 
     p32, p64, mhz, psrc = peaks()
     t_roof = f32 / (p32 * 1e12) + f64 / (p64 * 1e12)
@@ -640,11 +640,14 @@ def main():
 
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": "groups/s", "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong",
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": wl.name, "groups_per_gpu": G, "weights_per_gpu": G * 128, "E": wl.E,
-                           "K": wl.cols, "diagonals": "per-column [4, 16384] fp32",
-                           "l2": "inputs (994 MB of W per GPU) larger than the 126 MB L2; no flush"},
+                "config": {"workload": wl.name, "groups": G_job, "weights": G_job * 128, "E": wl.E,
+                           "K": wl.cols, "diagonals": "per-column [4, 16384] fp32, replicated on every rank",
+                           "parallelism": f"row blocks x{world}" if world > 1 else "one GPU",
+                           "rows_rank0": [r0, r1], "groups_rank0": G,
+                           "l2": f"inputs ({W.nbytes / 1e6:.0f} MB of W per GPU) larger than the 126 MB L2; "
+                                 "no flush"},
                 "weights_per_s": value * 128,
                 "roofline": {"bound": "alu", "achieved": achieved, "peak": p32, "unit": "TFLOP/s",
                              "frac": achieved / p32, "traffic": traffic,

@@ -27,3 +27,15 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    try:
+        import parity
+    except ImportError:
+        return
+    if not parity.REPORT:
+        return
+    terminalreporter.write_sep("-", "parity coverage (groups)")
+    for where, counts in parity.REPORT:
+        terminalreporter.write_line(f"{where}: " + ", ".join(f"{k}={v}" for k, v in counts.items()))

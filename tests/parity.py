@@ -7,6 +7,14 @@ import oracle
 
 NEAR_TIE = 1e-12
 
+# (workload, counts) of the parity checks run in this session, printed in the
+# terminal summary so a run's log shows how many groups met the oracle
+REPORT = []
+
+
+def record(where, **counts):
+    REPORT.append((where, counts))
+
 
 def oracle_threads():
     return max(1, os.cpu_count() or 1)

@@ -44,7 +44,7 @@ def test_peaks_and_job_rate():
     assert abs(p32 - 148 * 128 * 2 * mhz * 1e6 / 1e12) < 1e-9
     assert abs(p64 - p32 / 2) < 1e-9
     # whole-job rate: all ranks' units over the slowest rank's time
-    assert bench.job_rate(8, 1000, 0.5) == 16000.0
+    assert bench.job_rate(8000, 0.5) == 16000.0  # the job's groups over the slowest rank's seconds
 
 
 def test_objective_roofline_picks_the_binding_bound():

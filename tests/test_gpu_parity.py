@@ -7,18 +7,18 @@ oracle minimum.  Full-size workloads are compared on seeded samples plus every
 group the kernel flagged (near-tie or exhaustive fallback), and checked on all
 groups for code consistency and the AbsMax bound."""
 import ctypes
-import os
 
 import numpy as np
 import pytest
 
 import oracle
 import parity as P
+from oracle import exactfit
 from minimax_scale_search_b200 import synth
 
 pytestmark = pytest.mark.gpu
 
-SAMPLE = int(os.environ.get("CQ_PARITY_SAMPLE", "0")) or max(200, min(2000, 40 * (os.cpu_count() or 1)))
+SAMPLE = 10_000  # seeded groups per full-size workload, besides every flagged group
 
 
 def f16bits(x):
@@ -38,53 +38,92 @@ def test_tiny_workload_every_group():
     gpu = P.run_gpu(W, D)
     Wg, Dg = P.groups_and_diag(W, D, W.shape[1])
     P.check_against_oracle(Wg, Dg, gpu, where="tiny")
+    P.record(synth.workload(1).name, groups=Wg.shape[0], oracle=Wg.shape[0])
     assert np.array_equal(P.recompute_codes(Wg, gpu["scales"]), gpu["codes"])
     assert gpu["counters"]["nonfinite"] == 0
     assert absmax_bound_ok(Wg, Dg, gpu["scales"], gpu["obj"])
 
 
-def test_projection_workload_sample_and_flagged():
+def test_projection_workload_every_group():
+    """All 24,576 groups of the projection workload meet the oracle."""
     W, D = synth.make_inputs(2)
     gpu = P.run_gpu(W, D)
     gpu2 = P.run_gpu(W, D)
     assert np.array_equal(gpu["scales"], gpu2["scales"]) and np.array_equal(gpu["codes"], gpu2["codes"])
     Wg, Dg = P.groups_and_diag(W, D, W.shape[1])
-    flagged = np.nonzero(gpu["flags"] & (0x02 | 0x04))[0]
-    sel = np.union1d(synth.sample_groups(2, SAMPLE, seed=11), flagged[:500])
-    P.check_against_oracle(Wg, Dg, gpu, sel=sel, where="projection")
+    P.check_against_oracle(Wg, Dg, gpu, where="projection")
     assert np.array_equal(P.recompute_codes(Wg, gpu["scales"]), gpu["codes"])
     assert absmax_bound_ok(Wg, Dg, gpu["scales"], gpu["obj"])
     s = gpu["scales"]
     assert s.min() >= 0x0001 and s.max() <= 0x7BFF
+    flagged = int(np.count_nonzero(gpu["flags"] & (0x02 | 0x04)))
+    P.record(synth.workload(2).name, groups=Wg.shape[0], flagged=flagged, oracle=Wg.shape[0])
 
 
-@pytest.mark.parametrize("idx", [3, 4, 5])
-def test_full_size_workload_sampled(idx):
+def _check_full_matrix(idx, matrix, W, D, gpu, n_sample, where):
+    """North-star rule on one full-size matrix: every group's codes are the
+    codes of its scale; every group with an exact fit (zero objective) has the
+    lowest such scale bit for bit (closed form, all groups); the oracle checks a
+    seeded sample of n_sample groups plus every group the kernel flagged
+    (near-tie or exhaustive fallback) that the closed form does not settle."""
+    Wg = W.reshape(-1, 128)
+    G = Wg.shape[0]
+    for g0 in range(0, G, 1 << 18):
+        g1 = min(G, g0 + (1 << 18))
+        assert np.array_equal(P.recompute_codes(Wg[g0:g1], gpu["scales"][g0:g1]), gpu["codes"][g0:g1]), where
+    s = gpu["scales"]
+    assert s.min() >= 0x0001 and s.max() <= 0x7BFF
+    assert np.all(D > 0)  # the closed form needs every diagonal positive
+    fit = exactfit.lowest_exact_fit(Wg)
+    has_fit = fit > 0
+    assert np.array_equal(s[has_fit], fit[has_fit]), where
+    assert np.all(gpu["obj"][has_fit] == 0.0), where
+    flagged = np.nonzero(gpu["flags"] & (0x02 | 0x04))[0]
+    sample = synth.sample_groups(idx, n_sample, seed=13, matrix=matrix)
+    sel = np.union1d(sample, flagged[~has_fit[flagged]])
+    E = D.shape[0]
+    gpr = D.shape[1] // 128
+    Dsel = np.ascontiguousarray(D.reshape(E, gpr, 128)[:, sel % gpr, :])
+    sub = {k: v[sel] for k, v in gpu.items() if k != "counters"}
+    P.check_against_oracle(Wg[sel], Dsel, sub, where=where)
+    return dict(groups=G, sample=len(sample), flagged=len(flagged), exact_fit=int(has_fit.sum()),
+                flagged_by_closed_form=int(has_fit[flagged].sum()), oracle=len(sel))
+
+
+@pytest.mark.parametrize("idx", [3, 4])
+def test_full_size_workload_north_star_rule(idx):
     wl = synth.workload(idx)
     W, D = synth.make_inputs(idx, matrix=0)
     gpu = P.run_gpu(W, D)
-    Wg = W.reshape(-1, 128)
-    G = Wg.shape[0]
-    assert G == wl.groups_per_matrix
-    # every group: codes are the codes of the chosen scale; scale in range
-    for g0 in range(0, G, 1 << 18):
-        g1 = min(G, g0 + (1 << 18))
-        assert np.array_equal(P.recompute_codes(Wg[g0:g1], gpu["scales"][g0:g1]), gpu["codes"][g0:g1])
-    s = gpu["scales"]
-    assert s.min() >= 0x0001 and s.max() <= 0x7BFF
-    flagged = np.nonzero(gpu["flags"] & (0x02 | 0x04))[0]
-    n = SAMPLE // (2 if wl.E > 4 else 1)
-    sel = np.union1d(synth.sample_groups(idx, n, seed=13), flagged[:200])
-    Wsel, Dsel = synth.group_rows(idx, sel)
-    sub = {k: v[sel] for k, v in gpu.items() if k != "counters"}
-    P.check_against_oracle(Wsel, Dsel, sub, where=wl.name)
+    assert W.size // 128 == wl.groups_per_matrix
+    c = _check_full_matrix(idx, 0, W, D, gpu, SAMPLE, wl.name)
     if idx == 4:
         cls = synth.stress_classes()
         assert np.all(gpu["scales"][cls == 3] == 1)
         assert np.all(gpu["codes"][cls == 3] == 0x88888888)
         assert gpu["counters"]["trivial"] >= int((cls == 3).sum())
-        # exact-multiple and single-nonzero groups reach objective 0 exactly
-        assert np.all(gpu["obj"][(cls == 1) | (cls == 2) | (cls == 4)] == 0.0)
+        # every exact-multiple, all-zero and single-nonzero group is settled
+        # bit for bit by the closed form
+        fit = exactfit.lowest_exact_fit(W.reshape(-1, 128))
+        assert np.all(fit[cls != 0] > 0)
+    P.record(wl.name, **c)
+
+
+def test_large_workload_all_matrices_north_star_rule():
+    """All 32 matrices run one by one; the 10,000-group sample is spread over
+    them (313 or 312 per matrix) and every flagged group of every matrix meets
+    the oracle."""
+    wl = synth.workload(5)
+    per = [SAMPLE // wl.n_matrices + (1 if m < SAMPLE % wl.n_matrices else 0) for m in range(wl.n_matrices)]
+    tot = {}
+    for m in range(wl.n_matrices):
+        W, D = synth.make_inputs(5, matrix=m)
+        gpu = P.run_gpu(W, D)
+        c = _check_full_matrix(5, m, W, D, gpu, per[m], f"{wl.name} matrix {m}")
+        for k, v in c.items():
+            tot[k] = tot.get(k, 0) + v
+    assert tot["groups"] == wl.groups and tot["sample"] == SAMPLE
+    P.record(wl.name, **tot)
 
 
 @pytest.mark.parametrize("E", [1, 2, 3, 4, 5, 6, 7, 8])
