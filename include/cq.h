@@ -86,6 +86,11 @@ typedef struct {
     void *ev_main_begin;      /* nullable cudaEvent_t recorded on `stream` just before the main
                                  selection kernel (profiling hook) */
     void *ev_main_end;        /* nullable cudaEvent_t recorded just after it, before the fallback */
+    int32_t intersections;    /* nonzero: search each run that survives the screen with the
+                                 pairwise environment-intersection solver (the page's
+                                 "environment intersections" candidates) instead of a vertex
+                                 test and binary search; identical results, slower on the
+                                 0.8B-scale sweep, so off by default */
 } cq_opts;
 
 /* Bytes of device workspace cq_select_scales_ex needs for G groups.  The
@@ -102,7 +107,14 @@ size_t cq_workspace_bytes(int64_t G, int E);
  *  E          number of environments, 1..CQ_MAX_E.
  *  out_scales [G] binary16 bit patterns of the chosen scales (0x0001..0x7BFF).
  *  out_codes  [G][16] packed codes, 4-byte aligned.
- * Allocates its workspace with cudaMallocAsync/cudaFreeAsync on `stream`. */
+ * Unlike the other selection entry points this one allocates: it takes its
+ * workspace (cq_workspace_bytes(G, E), about 8 bytes per group) from a
+ * stream-ordered memory pool that the library creates for each device on
+ * first use, and frees it on `stream` after the kernels.  The pool's release
+ * threshold is unlimited, so freed blocks stay reserved for the next call and
+ * the pool keeps its high-water mark until the process exits or the caller
+ * calls cq_trim_memory().  For no allocation at all, pass a workspace to
+ * cq_select_scales_ex (or use cq_select_scales_noalloc). */
 cq_status cq_select_scales(const uint16_t *W, int64_t G, const float *D, int E, int64_t K,
                            uint16_t *out_scales, uint32_t *out_codes, void *stream);
 
@@ -122,9 +134,10 @@ cq_status cq_select_scales_ex(const uint16_t *W, int64_t G, const float *D, int 
 
 /* Host-buffer variant: W_host, D_host, out_scales_host and out_codes_host are
  * HOST pointers (page-locked memory gives overlapped copies).  The call
- * allocates device buffers, streams the groups through them in chunks with
- * host<->device copies overlapped with compute on `stream`, and returns
- * after the results are in the host buffers (it synchronises `stream`). */
+ * allocates device buffers (from the same library pool as cq_select_scales),
+ * streams the groups through them in chunks with host<->device copies
+ * overlapped with compute on `stream`, and returns after the results are in
+ * the host buffers (it synchronises `stream`). */
 cq_status cq_select_scales_host(const uint16_t *W_host, int64_t G, const float *D_host, int E,
                                 int64_t K, uint16_t *out_scales_host, uint32_t *out_codes_host,
                                 void *stream);
@@ -268,9 +281,20 @@ cq_status cq_select_scales_spec(const uint16_t *W, int64_t G, const float *D, in
  *  - Every call uses the same array; the counters in it are cleared on
  *    `stream` at the start of each call.  Calls whose work overlaps on the
  *    GPU (on different streams, or from different host threads without
- *    ordering) race on the array: order them on one stream or otherwise. */
+ *    ordering) race on the array: order them on one stream or otherwise.
+ *  - The return value is the only status this entry point reports: its
+ *    counters are not readable by the caller.  A group with non-finite or
+ *    negative input still gets scale 0x0001 and all codes 0, which looks
+ *    like an all-zero group; a caller that must detect such input checks it
+ *    first, or uses cq_select_scales_ex with its own workspace and out_flags. */
 cq_status cq_select_scales_noalloc(const uint16_t *W, int64_t G, const float *D, int E, int64_t K,
                                    uint16_t *out_scales, uint32_t *out_codes, void *stream);
+
+/* Release the memory that cq_select_scales and cq_select_scales_host keep
+ * cached in the current device's library pool (cudaMemPoolTrimTo to zero).
+ * Blocks still in use by enqueued work are kept.  A no-op when the pool was
+ * never created.  Returns CQ_ERR_CUDA when a CUDA call fails. */
+cq_status cq_trim_memory(void);
 
 /* Copy the workspace counters to host_counters[CQ_NUM_COUNTERS] (host
  * memory).  Synchronises `stream`.  Returns CQ_ERR_NONFINITE when the last

@@ -29,7 +29,8 @@ MAX_E = 8
 EXPORTS = ("cq_workspace_bytes", "cq_select_scales", "cq_select_scales_ex", "cq_select_scales_host",
            "cq_absmax_scales", "cq_pool_diagonals", "cq_group_objective", "cq_reconstruction_proxy",
            "cq_gptq_export", "cq_gptq_dequantize", "cq_estimate_diagonals", "cq_select_scales_spec",
-           "cq_select_scales_noalloc", "cq_read_counters", "cq_get_status", "cq_status_string", "cq_version")
+           "cq_select_scales_noalloc", "cq_trim_memory", "cq_read_counters", "cq_get_status", "cq_status_string",
+           "cq_version")
 
 
 class CQError(RuntimeError):
@@ -49,7 +50,7 @@ SPEC_MAX_GROUP = 1024
 class Opts(ctypes.Structure):
     _fields_ = [("finalist_cap", ctypes.c_int32), ("force_exhaustive", ctypes.c_int32),
                 ("flag_rel_gap", ctypes.c_double), ("ev_main_begin", ctypes.c_void_p),
-                ("ev_main_end", ctypes.c_void_p)]
+                ("ev_main_end", ctypes.c_void_p), ("intersections", ctypes.c_int32)]
 
 
 def _load():
@@ -84,6 +85,8 @@ def _load():
     L.cq_select_scales_spec.argtypes = [vp, i64, vp, i32, i64, ctypes.POINTER(QuantizerSpec), vp, vp, vp, vp, vp]
     L.cq_select_scales_noalloc.restype = i32
     L.cq_select_scales_noalloc.argtypes = [vp, i64, vp, i32, i64, vp, vp, vp]
+    L.cq_trim_memory.restype = i32
+    L.cq_trim_memory.argtypes = []
     L.cq_read_counters.restype = i32
     L.cq_read_counters.argtypes = [vp, vp, vp]
     L.cq_get_status.restype = i32
@@ -164,14 +167,17 @@ def _shapes(W, D, K):
 def select_scales(W, D, K: int | None = None, *, stream=None, finalist_cap: int = 0,
                   force_exhaustive: bool = False, flag_rel_gap: float = 0.0,
                   out_scales=None, out_codes=None, want_objective: bool = False,
-                  want_flags: bool = False, workspace=None, main_events=None) -> Result:
+                  want_flags: bool = False, workspace=None, main_events=None,
+                  intersections: bool = False) -> Result:
     """Exact minimax FP16 scales and packed W4 codes for every 128-weight group.
 
     W: CUDA tensor of binary16 bit patterns (int16/uint16/float16), [R, K] grouped
        along rows or [G, 128].  D: CUDA float32, per column [E, K] or per group
        [E, G, 128].  Runs asynchronously on ``stream`` (default: current).
        main_events: optional pair of torch.cuda.Event (enable_timing=True)
-       recorded just before and after the main selection kernel."""
+       recorded just before and after the main selection kernel.
+       intersections: search surviving runs with the pairwise
+       environment-intersection solver (same results)."""
     import torch
     if not (W.is_cuda and D.is_cuda):
         raise ValueError("W and D must be CUDA tensors")
@@ -198,7 +204,8 @@ def select_scales(W, D, K: int | None = None, *, stream=None, finalist_cap: int 
             if not e.cuda_event:
                 e.record(stream)
         ev0, ev1 = (ctypes.c_void_p(e.cuda_event) for e in main_events)
-    opts = Opts(int(finalist_cap), int(bool(force_exhaustive)), float(flag_rel_gap), ev0, ev1)
+    opts = Opts(int(finalist_cap), int(bool(force_exhaustive)), float(flag_rel_gap), ev0, ev1,
+                int(bool(intersections)))
     st = lib.cq_select_scales_ex(_ptr(W), G, _ptr(D), E, K, _ptr(out_scales), _ptr(out_codes),
                                  _stream_handle(stream), ctypes.byref(opts), _ptr(workspace), wsb,
                                  _ptr(obj), _ptr(flags))
@@ -487,6 +494,14 @@ def read_counters(workspace, stream=None) -> dict:
     if st not in (CQ_OK, CQ_ERR_NONFINITE):
         raise CQError(st, "cq_read_counters")
     return {n: int(v) for n, v in zip(COUNTER_NAMES, host)}
+
+
+def trim_memory() -> None:
+    """Return the device memory that select_scales_plain and the host-buffer
+    path keep cached in the library's pool on the current device."""
+    st = lib.cq_trim_memory()
+    if st != CQ_OK:
+        raise CQError(st, "cq_trim_memory")
 
 
 def get_status(workspace, stream=None) -> int:

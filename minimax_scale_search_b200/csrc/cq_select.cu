@@ -94,6 +94,7 @@ struct Params {
     uint2 *queue;  // fallback entries: group, then J0 | J1 << 16 (the grid range to scan)
     int finalist_cap;
     int force_exhaustive;
+    int intersections;  // search surviving runs with the environment-intersection solver
     double flag_rel_gap;
     cudaEvent_t ev_begin;
     cudaEvent_t ev_end;
@@ -294,6 +295,8 @@ struct WarpSmem {
     __device__ SurvEntry *ent() { return reinterpret_cast<SurvEntry *>(bufA); }
     __device__ float *res_lb() { return reinterpret_cast<float *>(bufA + 4 * kMaxSurvivors); }
     __device__ uint16_t *res_j() { return reinterpret_cast<uint16_t *>(bufA + 5 * kMaxSurvivors); }
+    // one run's shifted fp32 coefficients for the intersection stage (E float4)
+    __device__ float4 *icoef() { return reinterpret_cast<float4 *>(bufA + 6 * kMaxSurvivors); }
     __device__ int *fin() { return reinterpret_cast<int *>(bufB); }
 };
 
@@ -310,24 +313,35 @@ struct RunResult {
     bool uncertain;
 };
 
+// max_e (A_e - 2 B_e s + C_e s^2) in fp64 (-2B is exact).
 template <int E>
-__device__ __forceinline__ double screen(const double (&A)[E], const double (&nb2)[E], const double (&C)[E],
-                                         double s)
+__device__ __forceinline__ double screen(const double (&A)[E], const double (&B)[E], const double (&C)[E], double s)
 {
-    double f = fma(fma(C[0], s, nb2[0]), s, A[0]);
+    double f = fma(fma(C[0], s, -2.0 * B[0]), s, A[0]);
 #pragma unroll
     for (int e = 1; e < E; e++)
-        f = fmax(f, fma(fma(C[e], s, nb2[e]), s, A[e]));
+        f = fmax(f, fma(fma(C[e], s, -2.0 * B[e]), s, A[e]));
     return f;
 }
 
-// Leftmost grid minimiser of max_e (A_e - 2 B_e s + C_e s^2) over grid
-// indices [ja, jb], with a certified bracket (see the file comment, step 5).
-template <int E>
-__device__ RunResult solve_run(const double (&A)[E], const double (&B)[E], const double (&C)[E],
-                               uint32_t ja, uint32_t jb, uint32_t guess)
+__device__ __forceinline__ void store_run(const RunResult &r, int at, float *res_lb, uint16_t *res_j, double &ub_min)
 {
-    RunResult r;
+    res_lb[at] = r.lb;
+    res_j[at] = static_cast<uint16_t>(r.j | (r.uncertain ? kUncertainBit : 0u));
+    ub_min = fmin(ub_min, r.ub);
+}
+
+// Search of one run's grid minimiser of f = max_e (A_e - 2 B_e s + C_e s^2)
+// over grid indices [ja, jb], in three certified stages (file comment, step
+// 7): a strict local minimum at a guess, the bracket of the continuous
+// minimiser from the environment intersections, and a binary search.
+
+// Common set-up of a run: delta >= |screen - exact| anywhere on the run.  A run on which every coefficient C is zero (every code with d > 0
+// is zero) has the constant objective max_e A_e: resolved here (true).
+template <int E>
+__device__ __forceinline__ bool run_prepare(const double (&A)[E], const double (&B)[E], const double (&C)[E],
+                                            uint32_t ja, uint32_t jb, double &delta, RunResult &r)
+{
     double cmax = C[0], amax = A[0];
 #pragma unroll
     for (int e = 1; e < E; e++) {
@@ -335,50 +349,95 @@ __device__ RunResult solve_run(const double (&A)[E], const double (&B)[E], const
         amax = fmax(amax, A[e]);
     }
     if (cmax == 0.0) {
-        // every code with d > 0 is zero: f is the constant max_e A_e (exact terms)
-        const double delta = amax * 0x1p-44;
+        delta = amax * 0x1p-44;
         r.j = ja;
         r.ub = amax + delta;
         r.lb = __double2float_rd(amax - delta);
         r.uncertain = false;
-        return r;
+        return true;
     }
-    const double sa = grid_value(ja), sb = grid_value(jb);
-    double P = 0.0, nb2[E];
+    const double sb = grid_value(jb);
+    double P = 0.0;
 #pragma unroll
-    for (int e = 0; e < E; e++) {
-        nb2[e] = -2.0 * B[e];
+    for (int e = 0; e < E; e++)
         P = fmax(P, fma(fma(C[e], sb, 2.0 * B[e]), sb, A[e]));
+    delta = P * 0x1p-44;
+    return false;
+}
+
+// A certified strict local minimum at grid index j is the run's unique grid
+// minimiser (max_e F_e is convex on the run).  True and r filled when certified.
+template <int E>
+__device__ __forceinline__ bool certify_local_min(const double (&A)[E], const double (&B)[E], const double (&C)[E],
+                                                  uint32_t ja, uint32_t jb, uint32_t j, double delta, RunResult &r)
+{
+    j = min(max(j, ja), jb);
+    const double Sj = screen<E>(A, B, C, grid_value(j));
+    bool ok = true;
+    if (j > ja) {
+        const double Sl = screen<E>(A, B, C, grid_value(j - 1));
+        ok = Sl - Sj > 2.0 * delta + 0x1p-40 * fmax(fabs(Sl), fabs(Sj));
     }
-    const double delta = P * 0x1p-44;  // >= |screen - exact| anywhere on the run
-    // A certified strict local minimum at the guess is the run's unique
-    // minimiser (convexity); otherwise fall back to the binary search.
-    {
-        const uint32_t j = min(max(guess, ja), jb);
-        const double Sj = screen<E>(A, nb2, C, grid_value(j));
-        bool ok = true;
-        if (j > ja) {
-            const double Sl = screen<E>(A, nb2, C, grid_value(j - 1));
-            ok = Sl - Sj > 2.0 * delta + 0x1p-40 * fmax(fabs(Sl), fabs(Sj));
-        }
-        if (ok && j < jb) {
-            const double Sr = screen<E>(A, nb2, C, grid_value(j + 1));
-            ok = Sr - Sj > 2.0 * delta + 0x1p-40 * fmax(fabs(Sr), fabs(Sj));
-        }
-        if (ok) {
-            r.j = j;
-            r.ub = Sj + delta;
-            r.lb = __double2float_rd(Sj - delta);
-            r.uncertain = false;
-            return r;
-        }
+    if (ok && j < jb) {
+        const double Sr = screen<E>(A, B, C, grid_value(j + 1));
+        ok = Sr - Sj > 2.0 * delta + 0x1p-40 * fmax(fabs(Sr), fabs(Sj));
     }
+    if (ok) {
+        r.j = j;
+        r.ub = Sj + delta;
+        r.lb = __double2float_rd(Sj - delta);
+        r.uncertain = false;
+    }
+    return ok;
+}
+
+// The grid minimiser of a run is one of the two grid points that bracket the
+// continuous minimiser of max_e F_e (convexity on the run).  Given the lower
+// one, j, this evaluates j and j + 1, takes the smaller (j on a tie) and
+// certifies it as a strict local minimum against both its neighbours, which
+// makes it the run's unique grid minimiser.  Three evaluations, as many as a
+// local-minimum test of one guess.  True and r filled when certified.
+template <int E>
+__device__ __forceinline__ bool certify_bracket(const double (&A)[E], const double (&B)[E], const double (&C)[E],
+                                                uint32_t ja, uint32_t jb, uint32_t j, double delta, RunResult &r)
+{
+    j = min(max(j, ja), jb);
+    const double S0 = screen<E>(A, B, C, grid_value(j));
+    const double S1 = j < jb ? screen<E>(A, B, C, grid_value(j + 1)) : INFINITY;
+    const bool up = S1 < S0;
+    const uint32_t w = up ? j + 1 : j;          // the smaller of the pair
+    const double Sw = up ? S1 : S0;
+    const double Sp = up ? S0 : S1;             // its partner (INFINITY: none)
+    // the far neighbour, on the side away from the partner
+    double Sf = INFINITY;
+    if (up ? w < jb : w > ja)
+        Sf = screen<E>(A, B, C, grid_value(up ? w + 1 : w - 1));
+    const double m = 2.0 * delta;
+    const bool ok = (Sp == INFINITY || Sp - Sw > m + 0x1p-40 * fmax(fabs(Sp), fabs(Sw))) &&
+                    (Sf == INFINITY || Sf - Sw > m + 0x1p-40 * fmax(fabs(Sf), fabs(Sw)));
+    if (ok) {
+        r.j = w;
+        r.ub = Sw + delta;
+        r.lb = __double2float_rd(Sw - delta);
+        r.uncertain = false;
+    }
+    return ok;
+}
+
+// Leftmost grid minimiser by a binary search on the sign of f(s_{j+1}) -
+// f(s_j); a comparison within the evaluation error marks the run uncertain,
+// and its lower bound then falls back to a bound over the whole run.
+template <int E>
+__device__ RunResult bisect_run(const double (&A)[E], const double (&B)[E], const double (&C)[E], uint32_t ja,
+                                uint32_t jb, double delta)
+{
+    RunResult r;
     uint32_t lo = ja, hi = jb;
     bool unc = false;
     while (lo < hi) {
         const uint32_t mid = (lo + hi) >> 1;
-        const double S0 = screen<E>(A, nb2, C, grid_value(mid));
-        const double S1 = screen<E>(A, nb2, C, grid_value(mid + 1));
+        const double S0 = screen<E>(A, B, C, grid_value(mid));
+        const double S1 = screen<E>(A, B, C, grid_value(mid + 1));
         const double Dd = S1 - S0;
         if (fabs(Dd) <= 2.0 * delta + 0x1p-40 * fmax(fabs(S0), fabs(S1)))
             unc = true;
@@ -387,7 +446,7 @@ __device__ RunResult solve_run(const double (&A)[E], const double (&B)[E], const
         else
             lo = mid + 1;
     }
-    const double Sf = screen<E>(A, nb2, C, grid_value(lo));
+    const double Sf = screen<E>(A, B, C, grid_value(lo));
     r.j = lo;
     r.ub = Sf + delta;
     r.uncertain = unc;
@@ -397,17 +456,111 @@ __device__ RunResult solve_run(const double (&A)[E], const double (&B)[E], const
         // max_e of a lower bound of each environment's minimum over [sa, sb]:
         // a convex quadratic with curvature C lies at most C (sb - sa)^2 / 4
         // below the smaller of its end values anywhere between them
+        const double sa = grid_value(ja), sb = grid_value(jb);
         const double h = sb - sa;
         double L = -INFINITY;
 #pragma unroll
         for (int e = 0; e < E; e++) {
-            const double Fa = fma(fma(C[e], sa, nb2[e]), sa, A[e]);
-            const double Fb = fma(fma(C[e], sb, nb2[e]), sb, A[e]);
+            const double Fa = fma(fma(C[e], sa, -2.0 * B[e]), sa, A[e]);
+            const double Fb = fma(fma(C[e], sb, -2.0 * B[e]), sb, A[e]);
             L = fmax(L, fmin(Fa, Fb) - 0.25 * C[e] * h * h);
         }
         r.lb = __double2float_rd(L - 2.0 * delta);
     }
     return r;
+}
+
+// max_e F_e at sa + t, with F_e(sa + t) = F0_e + t (g_e + C_e t) and
+// q[e] = {F0_e, g_e, C_e, -} in shared memory (every lane reads the same words).
+template <int E>
+__device__ __forceinline__ float shifted_max(const float4 *q, float t)
+{
+    float f = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < E; e++) {
+        const float4 c = q[e];
+        f = fmaxf(f, fmaf(fmaf(c.z, t, c.y), t, c.x));
+    }
+    return f;
+}
+
+// Pairwise environment intersections ("candidates induced by code transitions,
+// quadratic vertices, and environment intersections").  On one run every F_e
+// is a convex quadratic, so the continuous minimiser of max_e F_e over
+// [sa, sa + len] is a run end, the vertex of one F_e, or a point where two of
+// them cross.  The warp enumerates all of them: slot p < E(E-1)/2 is the pair
+// (e, f) with both roots of (F_e - F_f)(t) = 0 from the cancellation-free
+// quadratic formula, then the E clamped vertices, then the two ends; lane l
+// takes slots l and l + 32.  Every candidate's max_e F_e is evaluated in the
+// shifted fp32 form and a warp argmin (ties to the smaller t) gives the
+// minimiser's offset t* from sa.  The result only seeds the certified fp64
+// check, so its rounding cannot change the answer.
+template <int E>
+__device__ float intersect_minimiser(const float4 *q, float len, int lane)
+{
+    constexpr int kPairs = E * (E - 1) / 2;
+    constexpr int kSlots = kPairs + E + 2;
+    float best = INFINITY, bt = 0.0f;
+#pragma unroll
+    for (int rep = 0; rep < (kSlots + 31) / 32; rep++) {
+        const int slot = lane + 32 * rep;
+        float t1 = -1.0f, t2 = -1.0f;  // negative: no candidate
+        if (slot < kPairs) {
+            int e = 0, p = slot;
+#pragma unroll
+            for (int k = 0; k < E - 1; k++) {
+                if (p >= E - 1 - e) {
+                    p -= E - 1 - e;
+                    e++;
+                }
+            }
+            const float4 ce = q[e], cf = q[e + 1 + p];
+            // (F_e - F_f)(t) = c + b t + a t^2
+            const float a = ce.z - cf.z, b = ce.y - cf.y, c = ce.x - cf.x;
+            if (a == 0.0f) {
+                if (b != 0.0f)
+                    t1 = __fdividef(-c, b);
+            } else {
+                const float disc = fmaf(b, b, -4.0f * a * c);
+                if (disc >= 0.0f) {
+                    const float r = -0.5f * (b + copysignf(disc > 0.0f ? disc * rsqrtf(disc) : 0.0f, b));
+                    t1 = __fdividef(r, a);
+                    if (r != 0.0f)
+                        t2 = __fdividef(c, r);
+                }
+            }
+        } else if (slot < kPairs + E) {
+            const float4 ce = q[slot - kPairs];
+            const float v = ce.z > 0.0f ? __fdividef(-ce.y, 2.0f * ce.z) : (ce.y < 0.0f ? len : 0.0f);
+            t1 = fminf(fmaxf(v, 0.0f), len);
+        } else if (slot < kSlots) {
+            t1 = slot == kPairs + E ? 0.0f : len;
+        }
+        if (t1 >= 0.0f && t1 <= len) {
+            const float f1 = shifted_max<E>(q, t1);
+            if (f1 < best || (f1 == best && t1 < bt)) {
+                best = f1;
+                bt = t1;
+            }
+        }
+        if (t2 >= 0.0f && t2 <= len) {
+            const float f2 = shifted_max<E>(q, t2);
+            if (f2 < best || (f2 == best && t2 < bt)) {
+                best = f2;
+                bt = t2;
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float ob = __shfl_xor_sync(kFull, best, o);
+        const float ot = __shfl_xor_sync(kFull, bt, o);
+        if (ob < best || (ob == best && ot < bt)) {
+            best = ob;
+            bt = ot;
+        }
+    }
+    return bt;
 }
 
 // fp32 screen of one run [ja, jb]: a lower bound of min_s max_e F_e (the max
@@ -563,7 +716,7 @@ __device__ __forceinline__ void direct_coefficients(const WarpSmem<E> &sm, float
     }
 }
 
-template <int E>
+template <int E, bool kIntersect>
 __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int lane, Tally &tl)
 {
     // ---- 1. load ---------------------------------------------------------
@@ -1154,27 +1307,144 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
                 }
             }
         }
-        if (lane < nb) {
-            const SurvEntry en = ent[base + lane];
-            // starting guess: the grid point nearest the clamped vertex of the
-            // environment whose own minimum on the run is largest
-            const float sa = grid_value(en.ja), sb = grid_value(en.jb);
-            float L = -INFINITY, vstar = sa;
+        if constexpr (!kIntersect) {
+            // One lane per survivor: a certified strict local minimum at the grid
+            // point nearest the clamped vertex of the environment whose own
+            // minimum on the run is largest, else a binary search.
+            if (lane < nb) {
+                const SurvEntry en = ent[base + lane];
+                const float sa = grid_value(en.ja), sb = grid_value(en.jb);
+                float L = -INFINITY, vstar = sa;
 #pragma unroll
-            for (int e = 0; e < E; e++) {
-                const float Bf = static_cast<float>(myB[e]), Cf = static_cast<float>(myC[e]);
-                const float v = fminf(fmaxf(__fdividef(Bf, Cf), sa), sb);
-                const float f = fmaf(fmaf(Cf, v, -2.0f * Bf), v, Af[e]);
-                if (f > L) {
-                    L = f;
-                    vstar = v;
+                for (int e = 0; e < E; e++) {
+                    const float Bf = static_cast<float>(myB[e]), Cf = static_cast<float>(myC[e]);
+                    const float v = fminf(fmaxf(__fdividef(Bf, Cf), sa), sb);
+                    const float f = fmaf(fmaf(Cf, v, -2.0f * Bf), v, Af[e]);
+                    if (f > L) {
+                        L = f;
+                        vstar = v;
+                    }
+                }
+                const uint32_t guess = __half_as_ushort(__float2half_rn(vstar));
+                double delta;
+                RunResult rr;
+                if (!run_prepare<E>(A, myB, myC, en.ja, en.jb, delta, rr) &&
+                    !certify_local_min<E>(A, myB, myC, en.ja, en.jb, guess, delta, rr))
+                    rr = bisect_run<E>(A, myB, myC, en.ja, en.jb, delta);
+                store_run(rr, base + lane, res_lb, res_j, ub_min);
+            }
+        } else {
+            // Stage 1, one lane per survivor, in fp32 (the result only seeds the
+            // certified fp64 check).  The environment whose own minimum on the run
+            // is largest binds at its clamped vertex v* unless another one, m, is
+            // above it there; then the minimiser of the pair's maximum is where
+            // the two cross between v* and m's vertex (the pairwise environment
+            // intersection of the page's solver outline, a root of
+            // (C_e - C_m) s^2 - 2 (B_e - B_m) s + (A_e - A_m) by the
+            // cancellation-free quadratic formula).  The two grid points that
+            // bracket the guess are then certified.
+            SurvEntry en{0u, 0u, 0, 0};
+            double delta = 0.0;
+            bool need = false;
+            if (lane < nb) {
+                en = ent[base + lane];
+                const float sa = grid_value(en.ja), sb = grid_value(en.jb);
+                float Bf[E], Cf[E];
+                float L = -INFINITY, vstar = sa;
+                int eb = 0;
+#pragma unroll
+                for (int e = 0; e < E; e++) {
+                    Bf[e] = static_cast<float>(myB[e]);
+                    Cf[e] = static_cast<float>(myC[e]);
+                    const float v = fminf(fmaxf(__fdividef(Bf[e], Cf[e]), sa), sb);
+                    const float f = fmaf(fmaf(Cf[e], v, -2.0f * Bf[e]), v, Af[e]);
+                    if (f > L) {
+                        L = f;
+                        vstar = v;
+                        eb = e;
+                    }
+                }
+                float top = -INFINITY;
+                int m = eb;
+                float a = 0.0f, b = 0.0f, c = 0.0f, vm = vstar;  // (F_eb - F_m)(s) = a s^2 + b s + c
+#pragma unroll
+                for (int e = 0; e < E; e++) {
+                    const float f = fmaf(fmaf(Cf[e], vstar, -2.0f * Bf[e]), vstar, Af[e]);
+                    if (f > top) {
+                        top = f;
+                        m = e;
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < E; e++) {
+                    const float sg = e == eb ? 1.0f : (e == m ? -1.0f : 0.0f);
+                    a = fmaf(sg, Cf[e], a);
+                    b = fmaf(sg, -2.0f * Bf[e], b);
+                    c = fmaf(sg, Af[e], c);
+                    if (e == m)
+                        vm = fminf(fmaxf(__fdividef(Bf[e], Cf[e]), sa), sb);
+                }
+                float sg = vstar;
+                if (m != eb) {
+                    const float lo = fminf(vstar, vm), hi = fmaxf(vstar, vm);
+                    float r1 = -1.0f, r2 = -1.0f;
+                    if (a == 0.0f) {
+                        if (b != 0.0f)
+                            r1 = __fdividef(-c, b);
+                    } else {
+                        const float disc = fmaf(b, b, -4.0f * a * c);
+                        if (disc >= 0.0f) {
+                            const float q = -0.5f * (b + copysignf(disc > 0.0f ? disc * rsqrtf(disc) : 0.0f, b));
+                            r1 = __fdividef(q, a);
+                            if (q != 0.0f)
+                                r2 = __fdividef(c, q);
+                        }
+                    }
+                    if (r1 >= lo && r1 <= hi)
+                        sg = r1;
+                    else if (r2 >= lo && r2 <= hi)
+                        sg = r2;
+                }
+                const uint32_t j = __half_as_ushort(__float2half_rd(sg));
+                RunResult rr;
+                need = !run_prepare<E>(A, myB, myC, en.ja, en.jb, delta, rr) &&
+                       !certify_bracket<E>(A, myB, myC, en.ja, en.jb, j, delta, rr);
+                if (!need)
+                    store_run(rr, base + lane, res_lb, res_j, ub_min);
+            }
+            // Stage 2, the whole warp per survivor that is still open (three or
+            // more environments meet, or a near tie): the continuous minimiser
+            // from every pairwise environment intersection, vertex and end of the
+            // run, then the same bracket certificate.
+            unsigned pend = __ballot_sync(kFull, need);
+            while (pend) {
+                const int src = __ffs(pend) - 1;
+                pend &= pend - 1;
+                float4 *qc = sm.icoef();
+                const double sa = grid_value(en.ja);
+                if (lane == src) {
+#pragma unroll
+                    for (int e = 0; e < E; e++)
+                        qc[e] = make_float4(static_cast<float>(fma(fma(myC[e], sa, -2.0 * myB[e]), sa, A[e])),
+                                            static_cast<float>(2.0 * fma(myC[e], sa, -myB[e])),
+                                            static_cast<float>(myC[e]), 0.0f);
+                }
+                __syncwarp();
+                // exact: both ends are binary16 values
+                const float len = __shfl_sync(kFull, grid_value(en.jb) - static_cast<float>(sa), src);
+                const float t = intersect_minimiser<E>(qc, len, lane);
+                __syncwarp();
+                if (lane == src) {
+                    const uint32_t j = __half_as_ushort(__float2half_rd(static_cast<float>(sa) + t));
+                    RunResult rr;
+                    need = !certify_bracket<E>(A, myB, myC, en.ja, en.jb, j, delta, rr);
+                    if (!need)
+                        store_run(rr, base + lane, res_lb, res_j, ub_min);
                 }
             }
-            const uint32_t guess = __half_as_ushort(__float2half_rn(vstar));
-            const RunResult rr = solve_run<E>(A, myB, myC, en.ja, en.jb, guess);
-            res_lb[base + lane] = rr.lb;
-            res_j[base + lane] = static_cast<uint16_t>(rr.j | (rr.uncertain ? kUncertainBit : 0u));
-            ub_min = fmin(ub_min, rr.ub);
+            // Stage 3 (rare): binary search, which marks a near-flat run uncertain.
+            if (need)
+                store_run(bisect_run<E>(A, myB, myC, en.ja, en.jb, delta), base + lane, res_lb, res_j, ub_min);
         }
     }
     __syncwarp();
@@ -1286,7 +1556,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     tl.finalists += static_cast<uint32_t>(total);
 }
 
-template <int E>
+template <int E, bool kIntersect>
 __global__ void __launch_bounds__(kWarpsPerCta<E> * 32, 1) select_kernel(Params p)
 {
     constexpr int kWarps = kWarpsPerCta<E>;
@@ -1302,7 +1572,7 @@ __global__ void __launch_bounds__(kWarpsPerCta<E> * 32, 1) select_kernel(Params 
         if (g < p.G) {
             if (lane < 2 && g + stride < p.G)
                 asm volatile("prefetch.global.L2 [%0];" ::"l"(p.W + (g + stride) * kGroup + 64 * lane));
-            process_group<E>(p, sm, g, lane, tl);
+            process_group<E, kIntersect>(p, sm, g, lane, tl);
         }
         __syncthreads();  // the warps start the next group together
     }
@@ -1503,22 +1773,17 @@ cudaError_t pool_alloc(void **ptr, size_t bytes, cudaStream_t st)
     return cudaMallocFromPoolAsync(ptr, bytes, g_pool[dev], st);
 }
 
-template <int E>
-cudaError_t launch(const Params &p, cudaStream_t st)
+template <int E, bool kIntersect>
+cudaError_t launch_main(const Params &p, cudaStream_t st, int sms)
 {
-    int dev = 0;
-    cudaError_t err = cudaGetDevice(&dev);
-    if (err != cudaSuccess)
-        return err;
-    const int sms = sm_count(dev);
     constexpr int kWarps = kWarpsPerCta<E>;
     const size_t smem = sizeof(WarpSmem<E>) * kWarps;
-    err = cudaFuncSetAttribute(select_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
+    cudaError_t err = cudaFuncSetAttribute(select_kernel<E, kIntersect>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
     if (err != cudaSuccess)
         return err;
     int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel<E>, kWarps * 32, smem);
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel<E, kIntersect>, kWarps * 32, smem);
     if (err != cudaSuccess)
         return err;
     if (per_sm < 1)
@@ -1527,11 +1792,25 @@ cudaError_t launch(const Params &p, cudaStream_t st)
     const int64_t grid = need < static_cast<int64_t>(sms) * per_sm ? need : static_cast<int64_t>(sms) * per_sm;
     if (p.ev_begin && (err = cudaEventRecord(p.ev_begin, st)) != cudaSuccess)
         return err;
-    select_kernel<E><<<static_cast<unsigned>(grid), kWarps * 32, smem, st>>>(p);
+    select_kernel<E, kIntersect><<<static_cast<unsigned>(grid), kWarps * 32, smem, st>>>(p);
     err = cudaGetLastError();
     if (err != cudaSuccess)
         return err;
     if (p.ev_end && (err = cudaEventRecord(p.ev_end, st)) != cudaSuccess)
+        return err;
+    return cudaSuccess;
+}
+
+template <int E>
+cudaError_t launch(const Params &p, cudaStream_t st)
+{
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess)
+        return err;
+    const int sms = sm_count(dev);
+    err = p.intersections ? launch_main<E, true>(p, st, sms) : launch_main<E, false>(p, st, sms);
+    if (err != cudaSuccess)
         return err;
     exhaustive_kernel<E><<<static_cast<unsigned>(2 * sms), kExThreads, 0, st>>>(p);
     return cudaGetLastError();
@@ -1646,6 +1925,7 @@ cq_status cq_select_scales_ex(const uint16_t *W, int64_t G, const float *D, int 
     p.queue = reinterpret_cast<uint2 *>(static_cast<unsigned char *>(workspace) + kHeaderBytes);
     p.finalist_cap = kDefaultFinalists;
     p.force_exhaustive = 0;
+    p.intersections = 0;
     p.flag_rel_gap = 1e-12;
     p.ev_begin = nullptr;
     p.ev_end = nullptr;
@@ -1657,6 +1937,7 @@ cq_status cq_select_scales_ex(const uint16_t *W, int64_t G, const float *D, int 
         if (opts->finalist_cap > 0)
             p.finalist_cap = opts->finalist_cap;
         p.force_exhaustive = opts->force_exhaustive != 0;
+        p.intersections = opts->intersections != 0;
         if (opts->flag_rel_gap < 0.0 || !(opts->flag_rel_gap == opts->flag_rel_gap))
             return CQ_ERR_INVALID_ARG;
         if (opts->flag_rel_gap > 0.0)
@@ -1814,6 +2095,23 @@ cq_status cq_select_scales_noalloc(const uint16_t *W, int64_t G, const float *D,
         return CQ_ERR_CUDA;
     return cq_select_scales_ex(W, G, D, E, K, out_scales, out_codes, stream, nullptr, ws, workspace_bytes(G), nullptr,
                                nullptr);
+}
+
+cq_status cq_trim_memory(void)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return CQ_ERR_CUDA;
+    if (dev < 0 || dev >= 64)
+        return CQ_ERR_CUDA;
+    cudaMemPool_t pool;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!g_pool_init[dev])
+            return CQ_OK;
+        pool = g_pool[dev];
+    }
+    return cudaMemPoolTrimTo(pool, 0) == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
 }
 
 cq_status cq_read_counters(const void *workspace, uint32_t *host_counters, void *stream)

@@ -40,6 +40,19 @@ def test_library_exports_every_declared_symbol(cq):
         assert hasattr(cq.lib, name)
 
 
+def test_allocating_entry_points_document_the_pool(cq):
+    """cq_select_scales says that it allocates, from which pool, that the pool
+    keeps its blocks, and how to return them; the trim call is exported."""
+    src = open(HEADER).read()
+    head = src[:src.index("cq_status cq_select_scales(")]
+    doc = head[head.rindex("/*"):]
+    for phrase in ("allocates", "pool", "release", "cq_trim_memory", "cq_select_scales_ex"):
+        assert phrase in doc, phrase
+    assert hasattr(cq.lib, "cq_trim_memory")
+    noalloc = src[src.index("Allocation-free variant"):src.index("cq_status cq_select_scales_noalloc(")]
+    assert "only status" in noalloc  # the allocation-free call reports no counters
+
+
 def test_status_strings_and_version(cq):
     assert cq.status_string(0) == "CQ_OK"
     for st in range(1, 6):

@@ -287,3 +287,47 @@ def test_host_entry_point_ragged_chunks():
     torch.cuda.synchronize()
     assert np.array_equal(hs2, r.scales.cpu().numpy().view(np.uint16))
     assert np.array_equal(hc2, r.codes.cpu().numpy().view(np.uint32))
+
+
+# ---- the pairwise environment-intersection solver (cq_opts.intersections) ----
+
+@pytest.mark.parametrize("idx", [1, 2])
+def test_intersection_solver_every_group(idx):
+    """Surviving runs searched by the environment-intersection solver: every
+    group of the tiny and projection workloads against the oracle."""
+    W, D = synth.make_inputs(idx)
+    gpu = P.run_gpu(W, D, intersections=True)
+    Wg, Dg = P.groups_and_diag(W, D, W.shape[1])
+    P.check_against_oracle(Wg, Dg, gpu, where=f"intersections {synth.workload(idx).name}")
+    assert np.array_equal(P.recompute_codes(Wg, gpu["scales"]), gpu["codes"])
+
+
+@pytest.mark.parametrize("E", [1, 2, 3, 4, 5, 6, 7, 8])
+def test_intersection_solver_each_environment_count(E):
+    rng = np.random.default_rng(140 + E)
+    G = 301
+    W = f16bits(rng.normal(0, 0.02, (G, 128)) * np.where(rng.random((G, 128)) < 0.02, 9, 1))
+    D = rng.lognormal(0, 2.0, (E, G, 128)).astype(np.float32)
+    gpu = P.run_gpu(W, D, intersections=True)
+    P.check_against_oracle(W, D, gpu, where=f"intersections E={E}")
+
+
+@pytest.mark.parametrize("idx,rows", [(3, 8192), (4, 8192)])
+def test_intersection_solver_same_output_as_default(idx, rows):
+    """Both run searches certify the unique grid minimiser of every run, so
+    the outputs (scales, codes, objectives, flags) are the same bytes; a
+    sample of the groups also meets the oracle."""
+    W = synth.make_weights(idx, 0, rows)
+    D = synth.make_diagonals(idx)
+    a = P.run_gpu(W, D)
+    b = P.run_gpu(W, D, intersections=True)
+    for k in ("scales", "codes", "obj", "flags"):
+        assert np.array_equal(a[k], b[k]), k
+    assert a["counters"] == b["counters"]
+    Wg = W.reshape(-1, 128)
+    sel = synth.sample_groups(idx, 1000, seed=19)
+    sel = sel[sel < Wg.shape[0]]
+    E = D.shape[0]
+    Dsel = np.ascontiguousarray(D.reshape(E, -1, 128)[:, sel % (D.shape[1] // 128), :])
+    P.check_against_oracle(Wg[sel], Dsel, {k: v[sel] for k, v in b.items() if k != "counters"},
+                           where=f"intersections {synth.workload(idx).name}")
