@@ -108,9 +108,9 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(groups: int):
-    """DRAM bytes per launch of the main kernel from the committed ncu summary,
-    scaled to `groups`; None when the kernel changed since the capture."""
+def main_kernel_record():
+    """The committed ncu record of the main kernel (profiles/select_kernel_traffic.txt)
+    as a dict, or None when the kernel's source changed since the capture."""
     path = os.path.join(ROOT, "profiles", "select_kernel_traffic.txt")
     try:
         kv = dict(tok.split("=", 1) for tok in open(path).read().split() if "=" in tok)
@@ -118,7 +118,32 @@ def recorded_traffic(groups: int):
         return None
     if kv.get("kernel_sha") != kernel_source_hash():
         return None
+    return kv
+
+
+def recorded_traffic(groups: int):
+    """DRAM bytes per launch of the main kernel from the committed ncu summary,
+    scaled to `groups`; None when the kernel changed since the capture."""
+    kv = main_kernel_record()
+    if kv is None:
+        return None
     return float(kv["dram_bytes"]) / float(kv["groups"]) * groups
+
+
+def recorded_issue():
+    """The main kernel's hardware utilisation from the same ncu capture: issue
+    slots active, pipe utilisation and warp instructions per group; None when
+    the kernel changed since the capture.  The counted-FLOP fraction compares
+    the kernel with the pages' candidate method; these say how busy the SMs
+    actually are."""
+    kv = main_kernel_record()
+    if kv is None or "issue_active_pct" not in kv:
+        return None
+    keys = ("issue_active_pct", "fma_pipe_pct", "fp64_pipe_pct", "alu_pipe_pct", "lsu_pipe_pct",
+            "warp_inst_per_group")
+    out = {k: float(kv[k]) for k in keys if k in kv}
+    out["source"] = "profiles/" + kv.get("capture", "select_kernel_sweep.md")
+    return out
 
 
 def recorded_kernel_traffic(kernel: str, units: int):
@@ -653,7 +678,13 @@ def main():
                              "frac": achieved / p32, "traffic": traffic,
                              "kernel": f"select_kernel<{wl.E}>", "kernel_ms": kernel_ms,
                              "roofline_ms": 1e3 * t_roof, "fp32_flops": f32, "fp64_flops": f64,
-                             "peak_note": f"fp32-equivalent (fp64 flops weighted x{p32 / p64:.0f}); {psrc}"},
+                             "peak_note": f"fp32-equivalent (fp64 flops weighted x{p32 / p64:.0f}); {psrc}",
+                             "count_basis": "the pages' candidate method on every constant-code run of every "
+                                            "group (vertices, pairwise environment intersections, closed-form "
+                                            "max), not the kernel's own instructions: the kernel skips most runs "
+                                            "by a certified window and screen, so frac compares it with that "
+                                            "method; 'issue' gives the hardware utilisation",
+                             "issue": recorded_issue()},
                 "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps,
                 "clocks": clocks, "counters": counters}
         print(json.dumps(line), flush=True)

@@ -28,7 +28,9 @@ namespace cq {
 namespace {
 
 constexpr int kTile = 32;
-constexpr int kTileRowsPerPass = 8;  // CTA of 32 x 8 threads, 4 elements per thread
+constexpr int kTileRowsPerPass = 8;  // transpose: CTA of 32 x 8 threads, 4 elements per thread
+constexpr int kDequantRows = 4;      // dequantisation: CTA of 32 x 4 threads, 8 words per thread, so 16 CTAs
+                                     // (twice the loads in flight) fit per SM
 
 // dst[c][r] = src[r][c] for an [rows][cols] matrix, one 32 x 32 tile per CTA
 // iteration (grid-stride over tiles).
@@ -81,7 +83,7 @@ __device__ __forceinline__ int64_t clamp_group(int g, int64_t ngroups)
 // lane writes the 8 values of one word, so a warp stores 256 consecutive
 // values of one output row.  Group indices outside [0, K/128) are clamped.
 template <bool kHalf>
-__global__ void __launch_bounds__(kTile * kTileRowsPerPass) dequant_kernel(const uint32_t *__restrict__ qweight,
+__global__ void __launch_bounds__(kTile * kDequantRows) dequant_kernel(const uint32_t *__restrict__ qweight,
                                                                           const uint32_t *__restrict__ qzeros,
                                                                           const uint16_t *__restrict__ scales,
                                                                           const int32_t *__restrict__ g_idx,
@@ -95,13 +97,13 @@ __global__ void __launch_bounds__(kTile * kTileRowsPerPass) dequant_kernel(const
     // fp16 output: each thread's words of the next tile are loaded into
     // registers while the current tile is dequantised and stored (the fp32
     // output, twice the bytes per word, was faster without it)
-    constexpr int kPer = kTile / kTileRowsPerPass;
+    constexpr int kPer = kTile / kDequantRows;
     uint32_t nxt[kPer];
     auto load = [&](int64_t t) {
         const int64_t k0 = (t / tiles_r) * kTile, r0 = (t % tiles_r) * kTile;
 #pragma unroll
         for (int k = 0; k < kPer; k++) {
-            const int64_t kk = k0 + ty + k * kTileRowsPerPass, r = r0 + tx;
+            const int64_t kk = k0 + ty + k * kDequantRows, r = r0 + tx;
             nxt[k] = (kk < K8 && r < R) ? qweight[kk * R + r] : 0u;
         }
     };
@@ -113,10 +115,10 @@ __global__ void __launch_bounds__(kTile * kTileRowsPerPass) dequant_kernel(const
         if (kHalf) {
 #pragma unroll
             for (int k = 0; k < kPer; k++)
-                tile[ty + k * kTileRowsPerPass][tx] = nxt[k];
+                tile[ty + k * kDequantRows][tx] = nxt[k];
         } else {
 #pragma unroll
-            for (int k = 0; k < kTile; k += kTileRowsPerPass) {
+            for (int k = 0; k < kTile; k += kDequantRows) {
                 const int64_t kk = k0 + ty + k, r = r0 + tx;
                 if (kk < K8 && r < R)
                     tile[ty + k][tx] = qweight[kk * R + r];
@@ -137,7 +139,7 @@ __global__ void __launch_bounds__(kTile * kTileRowsPerPass) dequant_kernel(const
             uniform = uniform && gi[j] == gi[0];
         const int64_t g0 = clamp_group(gi[0], ngroups);
 #pragma unroll
-        for (int k = 0; k < kTile; k += kTileRowsPerPass) {
+        for (int k = 0; k < kTile; k += kDequantRows) {
             const int64_t r = r0 + ty + k;
             if (r >= R)
                 continue;
@@ -247,7 +249,7 @@ cq_status cq_gptq_dequantize(const int32_t *qweight, const int32_t *qzeros, cons
     if (!qweight || !qzeros || !gptq_scales || !g_idx || !out || !aligned(qweight, 4) || !aligned(qzeros, 4) ||
         !aligned(gptq_scales, 2) || !aligned(g_idx, 16) || !aligned(out, 16))
         return CQ_ERR_INVALID_ARG;
-    const dim3 block(kTile, kTileRowsPerPass);
+    const dim3 block(kTile, kDequantRows);
     const unsigned grid = tile_grid(((R + 31) / 32) * ((K / 8 + 31) / 32));
     const uint32_t *qw = reinterpret_cast<const uint32_t *>(qweight);
     const uint32_t *qz = reinterpret_cast<const uint32_t *>(qzeros);

@@ -73,6 +73,42 @@ __device__ __forceinline__ int code_of(float aw, float s, float inv, int cap)
     return min(ni - below + above, cap);
 }
 
+// Codes of the 8 weights in one 16-byte chunk (binary16 bits, two per word)
+// at scale s, packed as (q + 8) nibbles low first.  Fast path: the signed
+// estimate x = w * (1/s) is within 9 * 2^-23 of w / s, and adding 1.5 * 2^23
+// rounds it to the nearest integer n (ties even) in the low mantissa bits; away
+// from a half-integer that n is the exact round-half-even of w / s, and the
+// clip to [-8, 7] follows.  When any of the 8 lies within 2^-12 of a
+// half-integer, the chunk is redone with the exact threshold tests of code_of.
+__device__ __forceinline__ uint32_t code_word(uint4 v, float s, float inv)
+{
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+    const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+    uint32_t word = 0;
+    bool near = false;
+#pragma unroll
+    for (int h = 0; h < 8; h++) {
+        const uint32_t b = (wd[h >> 1] >> (16 * (h & 1))) & 0xFFFFu;
+        const float x = __half2float(__ushort_as_half(static_cast<unsigned short>(b))) * inv;
+        const float y = x + kRound;
+        const int n = __float_as_int(y) - 0x4B400000;
+        near |= fabsf(fabsf(x - (y - kRound)) - 0.5f) <= 0x1p-12f;
+        const int q = min(max(n, -8), 7);
+        word |= static_cast<uint32_t>((q & 0xF) ^ 8) << (4 * h);
+    }
+    if (near) {
+        word = 0;
+#pragma unroll
+        for (int h = 0; h < 8; h++) {
+            const uint32_t b = (wd[h >> 1] >> (16 * (h & 1))) & 0xFFFFu;
+            const bool neg = b & 0x8000u;
+            const int c = code_of(half_value(b & 0x7FFFu), s, inv, neg ? 8 : 7);
+            word |= static_cast<uint32_t>(((neg ? -c : c) + 8) & 0xF) << (4 * h);
+        }
+    }
+    return word;
+}
+
 // AbsMax: s = binary16 nearest (ties even) to max_i |w_i| / 7 computed in
 // fp64, raised to the smallest positive pattern when it rounds to 0; codes are
 // the quantiser's at s.  Non-finite weights give scale 0x0001 and zero codes,
@@ -93,6 +129,12 @@ __global__ void __launch_bounds__(kStageWarps * 32, kStageCtas) absmax_kernel(co
         const int n = static_cast<int>(min(static_cast<int64_t>(32), G - g0));
         __syncwarp();
         stage_rows(sm, W, n, lane, [g0](int r) { return g0 + r; });
+        {
+            // the warp's next chunk into L2 while this one is computed
+            const int64_t gn = g0 + static_cast<int64_t>(gridDim.x) * kStageWarps * 32;
+            if (gn + 32 <= G)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(W + gn * kGroup + 64 * lane));
+        }
         __syncwarp();
         if (lane < n) {
             uint32_t m2 = 0;
@@ -114,19 +156,7 @@ __global__ void __launch_bounds__(kStageWarps * 32, kStageCtas) absmax_kernel(co
 #pragma unroll 4
             for (int j = 0; j < 16; j++) {
                 const uint4 v = *reinterpret_cast<const uint4 *>(row + j * 16);
-                const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
-                uint32_t word = 0x88888888u;
-                if (mag < kBeyond) {
-                    word = 0;
-#pragma unroll
-                    for (int h = 0; h < 8; h++) {
-                        const uint32_t b = (wd[h >> 1] >> (16 * (h & 1))) & 0xFFFFu;
-                        const bool neg = b & 0x8000u;
-                        const int c = code_of(half_value(b & 0x7FFFu), s, inv, neg ? 8 : 7);
-                        word |= static_cast<uint32_t>(((neg ? -c : c) + 8) & 0xF) << (4 * h);
-                    }
-                }
-                *reinterpret_cast<uint32_t *>(row + 4 * j) = word;
+                *reinterpret_cast<uint32_t *>(row + 4 * j) = mag < kBeyond ? code_word(v, s, inv) : 0x88888888u;
             }
             out_scales[g0 + lane] = static_cast<uint16_t>(sbits);
         }

@@ -2149,7 +2149,7 @@ const char *cq_status_string(cq_status status)
 
 int cq_version(void)
 {
-    return 100;
+    return 200;  // 2.0.0: cq_opts gained `intersections`, cq_trim_memory added
 }
 
 }  // extern "C"
