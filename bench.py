@@ -504,12 +504,20 @@ def bench_diag(args, wl, dev):
 
 
 SPEC_ROWS = 4096
-SPEC_CASES = ((-8, 7, 128), (-4, 3, 128), (-8, 7, 64), (-16, 15, 128))
+SPEC_CASES = ((-8, 7, 128), (-4, 3, 128), (-2, 1, 128), (-8, 7, 64), (-16, 15, 128))
+
+
+def spec_uses_w4_search(qmin: int, qmax: int, n: int) -> bool:
+    """Whether cq_select_scales_spec runs the W4 kernel's search for this spec
+    (group size 128, |qmin| = qmax or qmax + 1, at most 8)."""
+    return n == 128 and qmax >= 1 and -qmin <= 8 and -qmin in (qmax, qmax + 1)
 
 
 def bench_spec(args, wl, dev):
     """The general-spec path on the first 4,096 rows of the sweep (524,288
-    groups of 128; 1,048,576 of 64), one JSON line per spec."""
+    groups of 128; 1,048,576 of 64), one JSON line per spec and kernel: specs
+    the W4 kernel's search serves get a second line forced onto the general
+    kernel, for comparison."""
     import torch
     from minimax_scale_search_b200 import cq, synth
     stream = torch.cuda.current_stream()
@@ -520,20 +528,26 @@ def bench_spec(args, wl, dev):
     p32, p64, _, psrc = peaks()
     for qmin, qmax, n in SPEC_CASES:
         G = W.size // n
-        ms = time_calls(lambda: cq.select_scales_spec(Wd, Dd, wl.cols, qmin=qmin, qmax=qmax, group_size=n),
-                        args.steps, args.warmup, stream)
         f32, f64 = counted_flops(W.reshape(-1, n), wl.E, qmin, qmax)
-        ach = (f32 + f64 * p32 / p64) / (ms / 1e3) / 1e12
-        line = {"metric": "general-spec minimax scale selection groups/sec", "op": "spec", "value": G / ms * 1e3,
-                "unit": "groups/s", "ms_per_step": ms, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
-                "higher_is_better": True, "dtype": "f64", "data": "synthetic", "gpu_launches": args.steps,
-                "config": {"workload": f"sweep-rows0-{SPEC_ROWS}-q[{qmin},{qmax}]-n{n}", "groups": G, "E": wl.E,
-                           "K": wl.cols, "qmin": qmin, "qmax": qmax, "group_size": n},
-                "roofline": {"bound": "alu", "achieved": ach, "peak": p32, "unit": "TFLOP/s", "frac": ach / p32,
-                             "traffic": recorded_kernel_traffic("spec_kernel<4>", W.size), "kernel": "spec_kernel",
-                             "fp32_flops": f32, "fp64_flops": f64,
-                             "peak_note": psrc}}
-        print(json.dumps(line), flush=True)
+        kernels = (False, True) if spec_uses_w4_search(qmin, qmax, n) else (True,)
+        for general in kernels:
+            ms = time_calls(lambda: cq.select_scales_spec(Wd, Dd, wl.cols, qmin=qmin, qmax=qmax, group_size=n,
+                                                          general_kernel=general),
+                            args.steps, args.warmup, stream)
+            ach = (f32 + f64 * p32 / p64) / (ms / 1e3) / 1e12
+            kname = "spec_kernel" if general else f"select_kernel<{wl.E}, false, true> (W4 search)"
+            traffic = recorded_kernel_traffic("spec_kernel<4>", W.size) if general else None
+            line = {"metric": "general-spec minimax scale selection groups/sec", "op": "spec",
+                    "value": G / ms * 1e3, "unit": "groups/s", "ms_per_step": ms, "n_gpus": 1,
+                    "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "dtype": "f64",
+                    "data": "synthetic", "gpu_launches": args.steps * (1 if general else 2),
+                    "config": {"workload": f"sweep-rows0-{SPEC_ROWS}-q[{qmin},{qmax}]-n{n}", "groups": G,
+                               "E": wl.E, "K": wl.cols, "qmin": qmin, "qmax": qmax, "group_size": n,
+                               "kernel": "general" if general else "w4-search"},
+                    "roofline": {"bound": "alu", "achieved": ach, "peak": p32, "unit": "TFLOP/s",
+                                 "frac": ach / p32, "traffic": traffic, "kernel": kname,
+                                 "fp32_flops": f32, "fp64_flops": f64, "peak_note": psrc}}
+            print(json.dumps(line), flush=True)
 
 
 def main():

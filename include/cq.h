@@ -244,13 +244,23 @@ cq_status cq_estimate_diagonals(const void *X, int dtype, int64_t K, const int64
  * of rows) or per group [E][G][n] (K == 0).  Outputs: out_scales [G],
  * out_codes int8 [G][n] (the codes q themselves), optional out_objective fp64
  * [G] (8-byte aligned) and out_flags [G] (CQ_FLAG_TRIVIAL / CQ_FLAG_NONFINITE;
- * such groups get scale 0x0001, zero codes and objective 0).  The kernel is a
- * certified window plus an exact scan, slower than cq_select_scales, which
- * serves (-8, 7, 128). */
+ * such groups get scale 0x0001, zero codes and objective 0).  Scales, codes
+ * and objectives are the definition's own fp64 values, bit for bit.
+ *
+ * Two kernels serve it.  Group size 128 with a code range [-m, m] or
+ * [-m, m - 1], m <= 8 (the 2-, 3- and 4-bit ranges and the symmetric ones),
+ * and W, D 16-byte aligned, out_codes 4-byte aligned: the W4 kernel's search
+ * with that range's caps, its finalists rescored in the definition's order;
+ * this takes a workspace from the library pool, like cq_select_scales.  Any
+ * other spec: a certified window plus an exact best-first scan of the grid
+ * (no allocation).  spec->kernel = CQ_SPEC_KERNEL_GENERAL forces the second. */
+#define CQ_SPEC_KERNEL_AUTO 0
+#define CQ_SPEC_KERNEL_GENERAL 1
 typedef struct cq_quantizer_spec {
     int32_t qmin;
     int32_t qmax;
     int32_t group_size;
+    int32_t kernel;  /* CQ_SPEC_KERNEL_AUTO (0) or CQ_SPEC_KERNEL_GENERAL */
 } cq_quantizer_spec;
 #define CQ_SPEC_MAX_GROUP 1024
 cq_status cq_select_scales_spec(const uint16_t *W, int64_t G, const float *D, int E, int64_t K,

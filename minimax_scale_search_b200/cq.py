@@ -41,7 +41,8 @@ class CQError(RuntimeError):
 
 class QuantizerSpec(ctypes.Structure):
     """Codes in [qmin, qmax], groups of group_size weights (the pages' QuantizerSpec)."""
-    _fields_ = [("qmin", ctypes.c_int32), ("qmax", ctypes.c_int32), ("group_size", ctypes.c_int32)]
+    _fields_ = [("qmin", ctypes.c_int32), ("qmax", ctypes.c_int32), ("group_size", ctypes.c_int32),
+                ("kernel", ctypes.c_int32)]
 
 
 SPEC_MAX_GROUP = 1024
@@ -424,12 +425,14 @@ def gptq_dequantize(t: GPTQTensors, *, half: bool = False, stream=None):
 
 
 def select_scales_spec(W, D, K: int | None = None, *, qmin: int = -8, qmax: int = 7, group_size: int = 128,
-                       stream=None, want_objective: bool = False, want_flags: bool = False) -> Result:
+                       stream=None, want_objective: bool = False, want_flags: bool = False,
+                       general_kernel: bool = False) -> Result:
     """Exact minimax scales for a general spec (codes in [qmin, qmax], groups of
     group_size weights).  W: CUDA 16-bit binary16 patterns whose last dimension
     is a multiple of group_size; D: float32 per column [E, K] or per group
     [E, G, group_size].  Returns scales int16 [G] and codes int8 [G, group_size]
-    (the q values).  (-8, 7, 128) is served faster by select_scales."""
+    (the q values).  Group size 128 with qmin = -qmax or -qmax - 1 (|qmin| <= 8)
+    runs the W4 kernel's search; general_kernel=True forces the general one."""
     import torch
     n = int(group_size)
     if not (W.is_cuda and D.is_cuda and W.is_contiguous() and D.is_contiguous()):
@@ -453,7 +456,7 @@ def select_scales_spec(W, D, K: int | None = None, *, qmin: int = -8, qmax: int 
     codes = torch.empty((G, n), dtype=torch.int8, device=dev)
     obj = torch.empty(G, dtype=torch.float64, device=dev) if want_objective else None
     flags = torch.empty(G, dtype=torch.uint8, device=dev) if want_flags else None
-    spec = QuantizerSpec(int(qmin), int(qmax), n)
+    spec = QuantizerSpec(int(qmin), int(qmax), n, 1 if general_kernel else 0)
     _check(lib.cq_select_scales_spec(_ptr(W), G, _ptr(D), E, K, ctypes.byref(spec), _ptr(scales), _ptr(codes),
                                      _ptr(obj), _ptr(flags), _stream_handle(stream)), "cq_select_scales_spec")
     return Result(scales, codes, obj, flags)

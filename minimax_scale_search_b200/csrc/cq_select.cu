@@ -95,6 +95,9 @@ struct Params {
     int finalist_cap;
     int force_exhaustive;
     int intersections;  // search surviving runs with the environment-intersection solver
+    int qmax;           // general spec (kSpec kernels): largest positive code
+    int nmax;           // general spec: largest negative code magnitude, -qmin (qmax or qmax + 1, <= 8)
+    int8_t *out_q;      // general spec: codes q, int8 [G][128]
     double flag_rel_gap;
     cudaEvent_t ev_begin;
     cudaEvent_t ev_end;
@@ -620,9 +623,12 @@ __device__ __forceinline__ uint32_t pack_lane_codes(const int (&q)[4], int lane)
     return h | (up << 16);  // valid on even lanes: codes 8*(lane/2) .. +7
 }
 
+template <bool kSpec>
 __device__ __forceinline__ void write_constant_group(const Params &p, int64_t g, int lane, uint8_t flag)
 {
-    if (lane < 16)
+    if constexpr (kSpec)
+        reinterpret_cast<uint32_t *>(p.out_q + g * kGroup)[lane] = 0u;
+    else if (lane < 16)
         p.out_codes[g * 16 + lane] = 0x88888888u;
     if (lane == 0) {
         p.out_scales[g] = 0x0001;
@@ -681,7 +687,7 @@ __device__ __forceinline__ void add_delta64(const WarpSmem<E> &sm, uint32_t kk, 
 // the group (lane L takes ranks 32m + L); every lane gets the same totals.
 template <int E>
 __device__ __forceinline__ void direct_coefficients(const WarpSmem<E> &sm, float s, int lane, double (&B)[E],
-                                                    double (&C)[E])
+                                                    double (&C)[E], int qp, int qn)
 {
 #pragma unroll
     for (int e = 0; e < E; e++) {
@@ -692,7 +698,7 @@ __device__ __forceinline__ void direct_coefficients(const WarpSmem<E> &sm, float
     for (int m = 0; m < 4; m++) {
         const int r = 32 * m + lane;
         const float wv = sm.w[r];
-        const int aq = abs_code(fabsf(wv), s, wv < 0.0f ? 8 : 7);
+        const int aq = abs_code(fabsf(wv), s, wv < 0.0f ? qn : qp);
         const double bw = static_cast<double>(fabsf(wv)) * static_cast<double>(aq);  // exact
         const double cq = static_cast<double>(aq * aq);
 #pragma unroll
@@ -716,9 +722,15 @@ __device__ __forceinline__ void direct_coefficients(const WarpSmem<E> &sm, float
     }
 }
 
-template <int E, bool kIntersect>
+template <int E, bool kIntersect, bool kSpec>
 __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int lane, Tally &tl)
 {
+    // Code range: W4 clips at 7 and -8; a general spec (kSpec) at qmax and
+    // -nmax, with nmax = qmax or qmax + 1 and at most 8 code layers.  When
+    // nmax > qmax the last layer, k = qmax, holds negative weights only.
+    const int QP = kSpec ? p.qmax : 7;
+    const int QN = kSpec ? p.nmax : 8;
+    const bool negx = QN > QP;
     // ---- 1. load ---------------------------------------------------------
     const DiagView dv_g = diag_view(p, g);
     const uint2 wv = *reinterpret_cast<const uint2 *>(p.W + g * kGroup + 4 * lane);
@@ -767,12 +779,12 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     bad = __any_sync(kFull, bad);
     nonzero = __any_sync(kFull, nonzero);
     if (bad) {
-        write_constant_group(p, g, lane, CQ_FLAG_NONFINITE);
+        write_constant_group<kSpec>(p, g, lane, CQ_FLAG_NONFINITE);
         tl.nonfinite++;
         return;
     }
     if (!nonzero) {
-        write_constant_group(p, g, lane, CQ_FLAG_TRIVIAL);
+        write_constant_group<kSpec>(p, g, lane, CQ_FLAG_TRIVIAL);
         tl.trivial++;
         return;
     }
@@ -831,14 +843,16 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     // The fp32 objective at three grid scales near the AbsMax scale |w|max/7,
     // widened by 2^-18 (>= 12 fp32 roundings of nonnegative terms).
     const float amax = fabsf(sm.w[kGroup - 1]);
-    const uint32_t ja0 = min(max(static_cast<uint32_t>(__half_as_ushort(__float2half_rn(amax * (1.0f / 7.0f)))), 1u),
-                             kLast);
+    const float invq = kSpec ? 1.0f / static_cast<float>(QP) : (1.0f / 7.0f);
+    const uint32_t ja0 = min(max(static_cast<uint32_t>(__half_as_ushort(__float2half_rn(amax * invq))), 1u), kLast);
     float U;
     {
         const uint32_t jc[3] = {ja0, min(max(static_cast<uint32_t>(
-                                              __half_as_ushort(__float2half_rn(amax * (0.9f / 7.0f)))), 1u), kLast),
+                                              __half_as_ushort(__float2half_rn(
+                                                  amax * (kSpec ? 0.9f * invq : 0.9f / 7.0f)))), 1u), kLast),
                                 min(max(static_cast<uint32_t>(
-                                        __half_as_ushort(__float2half_rn(amax * (0.8f / 7.0f)))), 1u), kLast)};
+                                        __half_as_ushort(__float2half_rn(
+                                            amax * (kSpec ? 0.8f * invq : 0.8f / 7.0f)))), 1u), kLast)};
         float acc[3][E];
 #pragma unroll
         for (int c = 0; c < 3; c++)
@@ -860,7 +874,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         for (int m = 0; m < 4; m++) {
             const float wv = wq[m];
             const float aw = fabsf(wv);
-            const int K = wv < 0.0f ? 8 : 7;
+            const int K = wv < 0.0f ? QN : QP;
 #pragma unroll
             for (int c = 0; c < 3; c++) {
                 const float s = grid_value(jc[c]);
@@ -936,7 +950,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
 #pragma unroll 1
             for (int r = kGroup - 8; r < kGroup; r++) {
                 const float wv = sm.w[r];
-                const float ex = fmaxf(fmaf(-(wv < 0.0f ? 8.0f : 7.0f), sl, fabsf(wv)), 0.0f);
+                const float ex = fmaxf(fmaf(-static_cast<float>(wv < 0.0f ? QN : QP), sl, fabsf(wv)), 0.0f);
                 const float e2 = ex * ex;
 #pragma unroll
                 for (int e = 0; e < E; e++)
@@ -999,8 +1013,9 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
             else
                 hi = mid;
         }
-        sm.lay[lane] = (k == 7) ? sm.negpre[lo] : lo;  // lanes 0..7: F0_k, lanes 8..15: F1_k
-        sm.lay[16 + lane] = lo;                         // the same as rank thresholds
+        const bool empty = k >= QN;  // no code layer k in this range
+        sm.lay[lane] = empty ? 0 : ((negx && k == QP) ? sm.negpre[lo] : lo);  // lanes 0..7: F0_k, 8..15: F1_k
+        sm.lay[16 + lane] = empty ? kGroup : lo;                               // the same as rank thresholds
     }
     __syncwarp();
     const int *off = sm.lay;  // layer k holds ranks [off[k], off[k + 8]) (layer 7: negative ranks)
@@ -1026,10 +1041,14 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         const float wv = sm.w[r];
         const float aw = fabsf(wv);
         // |q| at s_J1: the layers whose rank threshold r has passed
-        int ktop = (wv < 0.0f && r >= th[15]) ? 1 : 0;
+        int ktop = 0;
 #pragma unroll
-        for (int k = 0; k < 7; k++)
-            ktop += r >= th[8 + k];
+        for (int k = 0; k < 8; k++) {
+            if (k < QP)
+                ktop += r >= th[8 + k];
+            else if (negx && k == QP && wv < 0.0f)
+                ktop += r >= th[8 + k];
+        }
         const float fk = static_cast<float>(ktop);
 #pragma unroll
         for (int e = 0; e < E; e++) {
@@ -1057,7 +1076,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
                 }
             }
             const int at = t - base;
-            const int r = (k == 7) ? static_cast<int>(sm.negidx[off[7] + at]) : off[k] + at;
+            const int r = (negx && k == QP) ? static_cast<int>(sm.negidx[off[k] + at]) : off[k] + at;
             const float aw = fabsf(sm.w[r]);
             layer[k * kLayerStride + at] =
                 (transition_index(aw, k) << 10) | (static_cast<uint32_t>(r) << 3) | static_cast<uint32_t>(k);
@@ -1285,7 +1304,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         for (int si = 0; si < nb; si++) {
             const SurvEntry en = ent[base + si];
             if (cur == -2 || cur - en.pos > kWalkMax) {
-                direct_coefficients<E>(sm, grid_value(en.ja), lane, Bc, Cc);
+                direct_coefficients<E>(sm, grid_value(en.ja), lane, Bc, Cc, QP, QN);
             } else {
                 // add the deltas of positions cur, cur-1, ..., en.pos+1
                 int lp = cur / c, x = cur - lp * c;
@@ -1499,37 +1518,96 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         bj = static_cast<uint32_t>(fin[0]);
         best = 0.0;
     }
+    if constexpr (kSpec) {
+        // A general spec returns the definition's own fp64 values: each
+        // finalist's objective is summed in weight order (i ascending, one
+        // rounding per multiply and add, as the oracle does), so the
+        // (objective, pattern) choice among several finalists and the
+        // reported objective are the oracle's bit for bit.  Lane L forms the
+        // terms of weights 4L..4L+3; lanes 0..3 sum four environments' 128
+        // terms in order through shared memory.
+        double *terms = reinterpret_cast<double *>(sm.bufA);  // [4][kGroup]
 #pragma unroll 1
-    for (int f = 0; f < (only ? 0 : total); f++) {
-        const uint32_t j = static_cast<uint32_t>(fin[f]);
-        const float s = grid_value(j);
-        const double sd = s;
-        double acc[E];
+        for (int f = 0; f < (only ? 0 : total); f++) {
+            const uint32_t j = static_cast<uint32_t>(fin[f]);
+            const float s = grid_value(j);
+            const double sd = s;
+            double rr[4];
 #pragma unroll
-        for (int e = 0; e < E; e++)
-            acc[e] = 0.0;
+            for (int m = 0; m < 4; m++) {
+                const bool neg = (wb[m] & 0x8000u) != 0u;
+                const int aq = abs_code(half_value(wb[m] & 0x7FFFu), s, neg ? QN : QP);
+                const double r_ = static_cast<double>(half_value(wb[m])) - sd * static_cast<double>(neg ? -aq : aq);
+                rr[m] = __dmul_rn(r_, r_);  // r is exact
+            }
+            double acc[E];
+#pragma unroll
+            for (int e0 = 0; e0 < E; e0 += 4) {
+#pragma unroll
+                for (int e = e0; e < E && e < e0 + 4; e++) {
+                    const float4 dv = *reinterpret_cast<const float4 *>(dv_g.base + e * dv_g.stride + 4 * lane);
+                    const float dq[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+                    for (int m = 0; m < 4; m++)
+                        terms[(e - e0) * kGroup + 4 * lane + m] = __dmul_rn(static_cast<double>(dq[m]), rr[m]);
+                }
+                __syncwarp();
+                double a = 0.0;
+                if (lane < 4 && e0 + lane < E) {
+#pragma unroll 8
+                    for (int i = 0; i < kGroup; i++)
+                        a = __dadd_rn(a, terms[lane * kGroup + i]);
+                }
+#pragma unroll
+                for (int e = e0; e < E && e < e0 + 4; e++)
+                    acc[e] = __shfl_sync(kFull, a, e - e0);
+                __syncwarp();
+            }
+            double v = acc[0];
+#pragma unroll
+            for (int e = 1; e < E; e++)
+                v = fmax(v, acc[e]);
+            if (v < best || (v == best && j < bj)) {
+                second = best;
+                best = v;
+                bj = j;
+            } else if (v < second) {
+                second = v;
+            }
+        }
+    } else {
 #pragma unroll 1
-        for (int m = 0; m < 4; m++) {
-            const int r = 32 * m + lane;
-            const float wv = sm.w[r];
-            const int aq = abs_code(fabsf(wv), s, wv < 0.0f ? 8 : 7);
-            const double r_ = static_cast<double>(fabsf(wv)) - sd * static_cast<double>(aq);  // exact
-            const double rr = __dmul_rn(r_, r_);
+        for (int f = 0; f < (only ? 0 : total); f++) {
+            const uint32_t j = static_cast<uint32_t>(fin[f]);
+            const float s = grid_value(j);
+            const double sd = s;
+            double acc[E];
 #pragma unroll
             for (int e = 0; e < E; e++)
-                acc[e] = __dadd_rn(acc[e], __dmul_rn(static_cast<double>(sm.d[e][r]), rr));
-        }
-        warp_sum_all(acc, lane);
-        double v = -INFINITY;
+                acc[e] = 0.0;
+#pragma unroll 1
+            for (int m = 0; m < 4; m++) {
+                const int r = 32 * m + lane;
+                const float wv = sm.w[r];
+                const int aq = abs_code(fabsf(wv), s, wv < 0.0f ? 8 : 7);
+                const double r_ = static_cast<double>(fabsf(wv)) - sd * static_cast<double>(aq);  // exact
+                const double rr = __dmul_rn(r_, r_);
 #pragma unroll
-        for (int e = 0; e < E; e++)
-            v = fmax(v, acc[e]);
-        if (v < best || (v == best && j < bj)) {
-            second = best;
-            best = v;
-            bj = j;
-        } else if (v < second) {
-            second = v;
+                for (int e = 0; e < E; e++)
+                    acc[e] = __dadd_rn(acc[e], __dmul_rn(static_cast<double>(sm.d[e][r]), rr));
+            }
+            warp_sum_all(acc, lane);
+            double v = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < E; e++)
+                v = fmax(v, acc[e]);
+            if (v < best || (v == best && j < bj)) {
+                second = best;
+                best = v;
+                bj = j;
+            } else if (v < second) {
+                second = v;
+            }
         }
     }
 
@@ -1538,25 +1616,33 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     int q[4];
 #pragma unroll
     for (int m = 0; m < 4; m++) {
-        const int aq = abs_code(half_value(wb[m] & 0x7FFFu), s, (wb[m] & 0x8000u) ? 8 : 7);
+        const int aq = abs_code(half_value(wb[m] & 0x7FFFu), s, (wb[m] & 0x8000u) ? QN : QP);
         q[m] = (wb[m] & 0x8000u) ? -aq : aq;
     }
-    const uint32_t word = pack_lane_codes(q, lane);
-    if ((lane & 1) == 0)
-        p.out_codes[g * 16 + (lane >> 1)] = word;
     const bool near = near_tie(best, second, p.flag_rel_gap);
+    if constexpr (kSpec) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int m = 0; m < 4; m++)
+            word |= static_cast<uint32_t>(q[m] & 0xFF) << (8 * m);
+        reinterpret_cast<uint32_t *>(p.out_q + g * kGroup)[lane] = word;  // the codes q as int8
+    } else {
+        const uint32_t word = pack_lane_codes(q, lane);
+        if ((lane & 1) == 0)
+            p.out_codes[g * 16 + (lane >> 1)] = word;
+    }
     if (lane == 0) {
         p.out_scales[g] = static_cast<uint16_t>(bj);
         if (p.out_obj)
             p.out_obj[g] = best;
         if (p.out_flags)
-            p.out_flags[g] = near ? CQ_FLAG_NEAR_TIE : 0;
+            p.out_flags[g] = (!kSpec && near) ? CQ_FLAG_NEAR_TIE : 0;
     }
     tl.near_tie += near ? 1u : 0u;
     tl.finalists += static_cast<uint32_t>(total);
 }
 
-template <int E, bool kIntersect>
+template <int E, bool kIntersect, bool kSpec>
 __global__ void __launch_bounds__(kWarpsPerCta<E> * 32, 1) select_kernel(Params p)
 {
     constexpr int kWarps = kWarpsPerCta<E>;
@@ -1572,7 +1658,7 @@ __global__ void __launch_bounds__(kWarpsPerCta<E> * 32, 1) select_kernel(Params 
         if (g < p.G) {
             if (lane < 2 && g + stride < p.G)
                 asm volatile("prefetch.global.L2 [%0];" ::"l"(p.W + (g + stride) * kGroup + 64 * lane));
-            process_group<E, kIntersect>(p, sm, g, lane, tl);
+            process_group<E, kIntersect, kSpec>(p, sm, g, lane, tl);
         }
         __syncthreads();  // the warps start the next group together
     }
@@ -1607,9 +1693,10 @@ __device__ __forceinline__ Best3 combine(Best3 a, Best3 b)
     return b;
 }
 
-template <int E>
+template <int E, bool kSpec>
 __global__ void __launch_bounds__(kExThreads) exhaustive_kernel(Params p)
 {
+    const int QP = kSpec ? p.qmax : 7, QN = kSpec ? p.nmax : 8;
     __shared__ float ws[kGroup];
     __shared__ double wsd[kGroup];
     __shared__ double ds[E][kGroup];
@@ -1640,7 +1727,7 @@ __global__ void __launch_bounds__(kExThreads) exhaustive_kernel(Params p)
             // the definition's own order: i ascending, one sum per environment
             for (int i = 0; i < kGroup; i++) {
                 const float w = ws[i];
-                const int aq = abs_code(fabsf(w), s, w < 0.0f ? 8 : 7);
+                const int aq = abs_code(fabsf(w), s, w < 0.0f ? QN : QP);
                 const double q = (w < 0.0f) ? -static_cast<double>(aq) : static_cast<double>(aq);
                 const double r = wsd[i] - sd * q;
                 const double rr = __dmul_rn(r, r);
@@ -1682,12 +1769,15 @@ __global__ void __launch_bounds__(kExThreads) exhaustive_kernel(Params p)
         if (tid < kGroup) {
             const float w = ws[tid];
             const float s = grid_value(r.j);
-            const int aq = abs_code(fabsf(w), s, w < 0.0f ? 8 : 7);
+            const int aq = abs_code(fabsf(w), s, w < 0.0f ? QN : QP);
             const int q = (w < 0.0f) ? -aq : aq;
-            nib[tid] = static_cast<uint32_t>((q + 8) & 0xF);
+            if constexpr (kSpec)
+                p.out_q[g * kGroup + tid] = static_cast<int8_t>(q);
+            else
+                nib[tid] = static_cast<uint32_t>((q + 8) & 0xF);
         }
         __syncthreads();
-        if (tid < 16) {
+        if (!kSpec && tid < 16) {
             uint32_t word = 0;
 #pragma unroll
             for (int t = 0; t < 8; t++)
@@ -1700,7 +1790,7 @@ __global__ void __launch_bounds__(kExThreads) exhaustive_kernel(Params p)
                 p.out_obj[g] = r.best;
             const bool near = near_tie(r.best, r.second, p.flag_rel_gap);
             if (p.out_flags)
-                p.out_flags[g] = CQ_FLAG_FALLBACK | (near ? CQ_FLAG_NEAR_TIE : 0);
+                p.out_flags[g] = kSpec ? 0 : (CQ_FLAG_FALLBACK | (near ? CQ_FLAG_NEAR_TIE : 0));
             if (near)
                 atomicAdd(&p.counters[CQ_CNT_NEAR_TIE], 1u);
         }
@@ -1773,17 +1863,17 @@ cudaError_t pool_alloc(void **ptr, size_t bytes, cudaStream_t st)
     return cudaMallocFromPoolAsync(ptr, bytes, g_pool[dev], st);
 }
 
-template <int E, bool kIntersect>
+template <int E, bool kIntersect, bool kSpec>
 cudaError_t launch_main(const Params &p, cudaStream_t st, int sms)
 {
     constexpr int kWarps = kWarpsPerCta<E>;
     const size_t smem = sizeof(WarpSmem<E>) * kWarps;
-    cudaError_t err = cudaFuncSetAttribute(select_kernel<E, kIntersect>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t err = cudaFuncSetAttribute(select_kernel<E, kIntersect, kSpec>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
     if (err != cudaSuccess)
         return err;
     int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel<E, kIntersect>, kWarps * 32, smem);
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel<E, kIntersect, kSpec>, kWarps * 32, smem);
     if (err != cudaSuccess)
         return err;
     if (per_sm < 1)
@@ -1792,7 +1882,7 @@ cudaError_t launch_main(const Params &p, cudaStream_t st, int sms)
     const int64_t grid = need < static_cast<int64_t>(sms) * per_sm ? need : static_cast<int64_t>(sms) * per_sm;
     if (p.ev_begin && (err = cudaEventRecord(p.ev_begin, st)) != cudaSuccess)
         return err;
-    select_kernel<E, kIntersect><<<static_cast<unsigned>(grid), kWarps * 32, smem, st>>>(p);
+    select_kernel<E, kIntersect, kSpec><<<static_cast<unsigned>(grid), kWarps * 32, smem, st>>>(p);
     err = cudaGetLastError();
     if (err != cudaSuccess)
         return err;
@@ -1809,10 +1899,16 @@ cudaError_t launch(const Params &p, cudaStream_t st)
     if (err != cudaSuccess)
         return err;
     const int sms = sm_count(dev);
-    err = p.intersections ? launch_main<E, true>(p, st, sms) : launch_main<E, false>(p, st, sms);
+    if (p.out_q) {  // a general spec (the W4 search's code range from p.qmax, p.nmax)
+        if ((err = launch_main<E, false, true>(p, st, sms)) != cudaSuccess)
+            return err;
+        exhaustive_kernel<E, true><<<static_cast<unsigned>(2 * sms), kExThreads, 0, st>>>(p);
+        return cudaGetLastError();
+    }
+    err = p.intersections ? launch_main<E, true, false>(p, st, sms) : launch_main<E, false, false>(p, st, sms);
     if (err != cudaSuccess)
         return err;
-    exhaustive_kernel<E><<<static_cast<unsigned>(2 * sms), kExThreads, 0, st>>>(p);
+    exhaustive_kernel<E, false><<<static_cast<unsigned>(2 * sms), kExThreads, 0, st>>>(p);
     return cudaGetLastError();
 }
 
@@ -1888,6 +1984,57 @@ cudaError_t noalloc_scratch(void **ptr)
     return cudaSuccess;
 }
 
+// A general spec through the W4 kernel's search, for group size 128 and a
+// code range [-nmax, qmax] with nmax = qmax or qmax + 1 and nmax <= 8 (the
+// 2-, 3- and 4-bit ranges and the symmetric ones): the same transitions,
+// window, screen and certified run search with the range's caps, the
+// finalists rescored in the definition's order, codes written as int8.
+// CQ_ERR_UNSUPPORTED when the spec or the buffers' alignment do not fit, so
+// the caller can take the general kernel.  Shapes are validated by the caller.
+// The workspace comes from the library pool, like cq_select_scales.
+cq_status select_spec_fast(const uint16_t *W, int64_t G, const float *D, int E, int64_t K, int qmin, int qmax,
+                           uint16_t *out_scales, int8_t *out_q, double *out_obj, uint8_t *out_flags,
+                           cudaStream_t st)
+{
+    const int nmax = -qmin;
+    if (!(qmax >= 1 && nmax <= 8 && (nmax == qmax || nmax == qmax + 1)))
+        return CQ_ERR_UNSUPPORTED;
+    if (!aligned(W, 16) || !aligned(D, 16) || !aligned(out_q, 4) || !aligned(out_scales, 2) ||
+        (out_obj && !aligned(out_obj, 8)))
+        return CQ_ERR_UNSUPPORTED;
+    Params p;
+    p.W = W;
+    p.D = D;
+    p.G = G;
+    p.K = K;
+    p.gpr = K > 0 ? K / kGroup : 1;
+    p.out_scales = out_scales;
+    p.out_codes = nullptr;
+    p.out_obj = out_obj;
+    p.out_flags = out_flags;
+    p.finalist_cap = kDefaultFinalists;
+    p.force_exhaustive = 0;
+    p.intersections = 0;
+    p.qmax = qmax;
+    p.nmax = nmax;
+    p.out_q = out_q;
+    p.flag_rel_gap = 1e-12;
+    p.ev_begin = nullptr;
+    p.ev_end = nullptr;
+    void *ws = nullptr;
+    const size_t bytes = workspace_bytes(G);
+    if (pool_alloc(&ws, bytes, st) != cudaSuccess)
+        return CQ_ERR_CUDA;
+    p.counters = static_cast<uint32_t *>(ws);
+    p.queue = reinterpret_cast<uint2 *>(static_cast<unsigned char *>(ws) + kHeaderBytes);
+    cq_status out = CQ_OK;
+    if (cudaMemsetAsync(ws, 0, kHeaderBytes, st) != cudaSuccess || dispatch(E, p, st) != cudaSuccess)
+        out = CQ_ERR_CUDA;
+    if (cudaFreeAsync(ws, st) != cudaSuccess && out == CQ_OK)
+        out = CQ_ERR_CUDA;
+    return out;
+}
+
 }  // namespace cq
 
 using namespace cq;
@@ -1926,6 +2073,9 @@ cq_status cq_select_scales_ex(const uint16_t *W, int64_t G, const float *D, int 
     p.finalist_cap = kDefaultFinalists;
     p.force_exhaustive = 0;
     p.intersections = 0;
+    p.qmax = 7;
+    p.nmax = 8;
+    p.out_q = nullptr;
     p.flag_rel_gap = 1e-12;
     p.ev_begin = nullptr;
     p.ev_end = nullptr;

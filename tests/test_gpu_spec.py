@@ -95,3 +95,47 @@ def test_per_column_layout_and_edge_groups():
     s, c, f, fl = _run(Wb, _diag(2, 6, 64), -4, 3, 64)
     assert list(fl[:4]) == [0, 8, 1, 8]
     assert np.all(s[1:4] == 1) and np.all(c[1:4] == 0) and np.all(f[1:4] == 0)
+
+
+def _run_kernel(W, D, qmin, qmax, n, K, general):
+    import torch
+    from minimax_scale_search_b200 import cq
+    Wt = torch.from_numpy(np.ascontiguousarray(W).view(np.int16)).cuda()
+    Dt = torch.from_numpy(np.ascontiguousarray(D, dtype=np.float32)).cuda()
+    r = cq.select_scales_spec(Wt, Dt, K, qmin=qmin, qmax=qmax, group_size=n, want_objective=True,
+                              want_flags=True, general_kernel=general)
+    torch.cuda.synchronize()
+    return (r.scales.cpu().numpy().view(np.uint16), r.codes.cpu().numpy(), r.objective.cpu().numpy(),
+            r.flags.cpu().numpy())
+
+
+@pytest.mark.parametrize("spec", [(-8, 7), (-4, 3), (-2, 1), (-1, 1), (-8, 8), (-5, 4)])
+def test_w4_search_and_general_kernel_same_bytes(spec):
+    """Group size 128 with |qmin| = qmax or qmax + 1 runs the W4 kernel's
+    search; the general kernel is the other implementation of the same
+    definition.  On 262,144 sweep groups every scale, code, objective and flag
+    is the same, and a sample meets the oracle."""
+    qmin, qmax = spec
+    wl = synth.workload(3)
+    W = synth.make_weights(3, 0, 2048)
+    D = synth.make_diagonals(3)
+    a = _run_kernel(W, D, qmin, qmax, 128, wl.cols, general=False)
+    b = _run_kernel(W, D, qmin, qmax, 128, wl.cols, general=True)
+    for x, y, name in zip(a, b, ("scales", "codes", "objective", "flags")):
+        assert np.array_equal(x.view(np.uint8), y.view(np.uint8)), (spec, name)
+    sel = synth.sample_groups(3, 20_000, seed=29)
+    sel = sel[sel < W.size // 128][:600]
+    Wg = W.reshape(-1, 128)[sel]
+    Dg = np.ascontiguousarray(D.reshape(4, -1, 128)[:, sel % wl.groups_per_row, :])
+    o = oracle.solve(Wg, Dg, qmin=qmin, qmax=qmax, threads=oracle_threads())
+    assert np.array_equal(a[0][sel], o["best_bits"]), spec
+    assert np.array_equal(a[1][sel], o["codes"][:, :128]), spec
+    assert np.array_equal(a[2][sel].view(np.uint64), o["best_obj"].view(np.uint64)), spec
+
+
+@pytest.mark.parametrize("E", [1, 2, 3, 5, 8])
+def test_w4_search_each_environment_count(E):
+    W = _groups(160, 128, seed=200 + E)
+    D = _diag(E, 160, 128, seed=300 + E, sigma=2.0)
+    for qmin, qmax in ((-4, 3), (-2, 1), (-8, 8)):
+        _check(W, D, qmin, qmax, 128, where=f"E={E} spec ({qmin}, {qmax})")
