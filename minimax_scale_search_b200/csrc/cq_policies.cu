@@ -109,6 +109,34 @@ __device__ __forceinline__ uint32_t code_word(uint4 v, float s, float inv)
     return word;
 }
 
+// The signed codes q of the 8 weights of one 16-byte chunk at scale s, by the
+// fast path of code_word (estimate, magic-constant rounding, clip to [-8, 7]),
+// redone with the exact threshold tests when any lies within 2^-12 of a
+// half-integer.
+__device__ __forceinline__ void codes8(uint4 v, float s, float inv, int (&q)[8])
+{
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+    const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+    bool near = false;
+#pragma unroll
+    for (int h = 0; h < 8; h++) {
+        const uint32_t b = (wd[h >> 1] >> (16 * (h & 1))) & 0xFFFFu;
+        const float x = __half2float(__ushort_as_half(static_cast<unsigned short>(b))) * inv;
+        const float y = x + kRound;
+        near |= fabsf(fabsf(x - (y - kRound)) - 0.5f) <= 0x1p-12f;
+        q[h] = min(max(__float_as_int(y) - 0x4B400000, -8), 7);
+    }
+    if (near) {
+#pragma unroll
+        for (int h = 0; h < 8; h++) {
+            const uint32_t b = (wd[h >> 1] >> (16 * (h & 1))) & 0xFFFFu;
+            const bool neg = b & 0x8000u;
+            const int c = code_of(half_value(b & 0x7FFFu), s, inv, neg ? 8 : 7);
+            q[h] = neg ? -c : c;
+        }
+    }
+}
+
 // AbsMax: s = binary16 nearest (ties even) to max_i |w_i| / 7 computed in
 // fp64, raised to the smallest positive pattern when it rounds to 0; codes are
 // the quantiser's at s.  Non-finite weights give scale 0x0001 and zero codes,
@@ -247,12 +275,12 @@ __global__ void __launch_bounds__(kStageWarps * 32) objective_kernel(const uint1
         for (int j = 0; j < 16; j++) {
             const uint4 v = *reinterpret_cast<const uint4 *>(row + j * 16);
             const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+            int qc[8];
+            codes8(v, s, inv, qc);
 #pragma unroll
             for (int h = 0; h < 8; h++) {
                 const uint32_t bits = (wd[h >> 1] >> (16 * (h & 1))) & 0xFFFFu;
-                const bool neg = bits & 0x8000u;
-                const int c = code_of(half_value(bits & 0x7FFFu), s, inv, neg ? 8 : 7);
-                const double r = fma(nsd, static_cast<double>(neg ? -c : c), static_cast<double>(half_value(bits)));
+                const double r = fma(nsd, static_cast<double>(qc[h]), static_cast<double>(half_value(bits)));
                 const double rr = __dmul_rn(r, r);
 #pragma unroll
                 for (int e = 0; e < E; e++) {
