@@ -137,6 +137,31 @@ __device__ __forceinline__ void codes8(uint4 v, float s, float inv, int (&q)[8])
     }
 }
 
+// code_word for an AbsMax scale in the normal binary16 range: then
+// |w| / s <= 7 / (1 - 2^-11) < 7.5 for every weight of the group, so every code
+// is already in [-7, 7] and needs no clip.  Two weights go through each step:
+// their estimates' rounded integers sit in the low halves of y, which one byte
+// permute packs; (n & 15) ^ 8 forms both nibbles at once.  near is set when a
+// weight lies within 2^-12 of a half-integer (the caller then takes code_word).
+__device__ __forceinline__ uint32_t code_word_unclipped(uint4 v, float inv, bool &near)
+{
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+    const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+    float dmax = 0.0f;
+    uint32_t b[4];
+#pragma unroll
+    for (int p = 0; p < 4; p++) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&wd[p]));
+        const float x0 = f.x * inv, x1 = f.y * inv;
+        const float y0 = x0 + kRound, y1 = x1 + kRound;
+        dmax = fmaxf(dmax, fmaxf(fabsf(x0 - (y0 - kRound)), fabsf(x1 - (y1 - kRound))));
+        const uint32_t nb = (__byte_perm(__float_as_uint(y0), __float_as_uint(y1), 0x5410) & 0x000F000Fu) ^ 0x00080008u;
+        b[p] = nb | (nb >> 12);  // byte 0: the pair's two nibbles, low weight first
+    }
+    near = dmax >= 0.5f - 0x1p-12f;
+    return __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+}
+
 // AbsMax: s = binary16 nearest (ties even) to max_i |w_i| / 7 computed in
 // fp64, raised to the smallest positive pattern when it rounds to 0; codes are
 // the quantiser's at s.  Non-finite weights give scale 0x0001 and zero codes,
@@ -181,10 +206,22 @@ __global__ void __launch_bounds__(kStageWarps * 32, kStageCtas) absmax_kernel(co
             const float s = grid_value(sbits);
             const float inv = 1.0f / s;
             // code word j (8 nibbles) overwrites bytes 4j..4j+3 of the row, which chunk j has already passed
+            if (sbits >= 0x400u && mag < kBeyond) {
 #pragma unroll 4
-            for (int j = 0; j < 16; j++) {
-                const uint4 v = *reinterpret_cast<const uint4 *>(row + j * 16);
-                *reinterpret_cast<uint32_t *>(row + 4 * j) = mag < kBeyond ? code_word(v, s, inv) : 0x88888888u;
+                for (int j = 0; j < 16; j++) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(row + j * 16);
+                    bool near;
+                    uint32_t word = code_word_unclipped(v, inv, near);
+                    if (near)
+                        word = code_word(v, s, inv);
+                    *reinterpret_cast<uint32_t *>(row + 4 * j) = word;
+                }
+            } else {
+#pragma unroll 4
+                for (int j = 0; j < 16; j++) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(row + j * 16);
+                    *reinterpret_cast<uint32_t *>(row + 4 * j) = mag < kBeyond ? code_word(v, s, inv) : 0x88888888u;
+                }
             }
             out_scales[g0 + lane] = static_cast<uint16_t>(sbits);
         }

@@ -42,8 +42,10 @@ def test_absmax_matches_oracle():
     pick = np.concatenate([np.nonzero(cls == c)[0][:300] for c in range(5)])
     W4, _ = synth.group_rows(4, np.sort(pick))
     Wp, _, _ = synth.make_proxy_inputs()
+    # tiny weights: max|w| / 7 lands in the subnormal range, where codes reach the clip
+    sub = (np.random.default_rng(8).integers(-40, 41, (96, 128)) * 2.0 ** -24).astype(np.float16).view(np.uint16)
     for name, W in (("tiny", synth.make_weights(1).reshape(-1, 128)), ("stress", W4),
-                    ("proxy", Wp), ("nonfinite", _with_nonfinite(Wp[:40]))):
+                    ("proxy", Wp), ("nonfinite", _with_nonfinite(Wp[:40])), ("subnormal scales", sub)):
         s, c = cq.absmax_scales(_cuda(W))
         gs, gc = _host_bits(s, c)
         es, ec = OP.absmax_policy(W)
