@@ -509,8 +509,8 @@ SPEC_CASES = ((-8, 7, 128), (-4, 3, 128), (-2, 1, 128), (-8, 7, 64), (-16, 15, 1
 
 def spec_uses_w4_search(qmin: int, qmax: int, n: int) -> bool:
     """Whether cq_select_scales_spec runs the W4 kernel's search for this spec
-    (group size 128, |qmin| = qmax or qmax + 1, at most 8)."""
-    return n == 128 and qmax >= 1 and -qmin <= 8 and -qmin in (qmax, qmax + 1)
+    (group size 128 or 64, |qmin| = qmax or qmax + 1, at most 8)."""
+    return n in (128, 64) and qmax >= 1 and -qmin <= 8 and -qmin in (qmax, qmax + 1)
 
 
 def bench_spec(args, wl, dev):
@@ -535,7 +535,7 @@ def bench_spec(args, wl, dev):
                                                           general_kernel=general),
                             args.steps, args.warmup, stream)
             ach = (f32 + f64 * p32 / p64) / (ms / 1e3) / 1e12
-            kname = "spec_kernel" if general else f"select_kernel<{wl.E}, false, true> (W4 search)"
+            kname = "spec_kernel" if general else f"select_kernel<{wl.E}, false, true, {n}> (W4 search)"
             traffic = recorded_kernel_traffic("spec_kernel<4>", W.size) if general else None
             line = {"metric": "general-spec minimax scale selection groups/sec", "op": "spec",
                     "value": G / ms * 1e3, "unit": "groups/s", "ms_per_step": ms, "n_gpus": 1,

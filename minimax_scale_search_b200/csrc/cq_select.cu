@@ -97,30 +97,69 @@ struct Params {
     int intersections;  // search surviving runs with the environment-intersection solver
     int qmax;           // general spec (kSpec kernels): largest positive code
     int nmax;           // general spec: largest negative code magnitude, -qmin (qmax or qmax + 1, <= 8)
-    int8_t *out_q;      // general spec: codes q, int8 [G][128]
+    int8_t *out_q;      // general spec: codes q, int8 [G][group]
+    int group;          // weights per group: 128, or 64 for a general spec
     double flag_rel_gap;
     cudaEvent_t ev_begin;
     cudaEvent_t ev_end;
 };
 
-// Diagonals of group g: environment e's 128 values start at base + e * stride.
+// Diagonals of group g (N weights): environment e's N values start at
+// base + e * stride.
 struct DiagView {
     const float *base;
     int64_t stride;
 };
 
+template <int N>
 __device__ __forceinline__ DiagView diag_view(const Params &p, int64_t g)
 {
     if (p.K > 0)
-        return DiagView{p.D + (g % p.gpr) * kGroup, p.K};
-    return DiagView{p.D + g * kGroup, p.G * kGroup};
+        return DiagView{p.D + (g % p.gpr) * N, p.K};
+    return DiagView{p.D + g * N, p.G * N};
 }
 
+template <int N>
 __device__ __forceinline__ const float *diag_ptr(const Params &p, int64_t g, int e)
 {
     if (p.K > 0)
-        return p.D + static_cast<int64_t>(e) * p.K + (g % p.gpr) * kGroup;
-    return p.D + (static_cast<int64_t>(e) * p.G + g) * kGroup;
+        return p.D + static_cast<int64_t>(e) * p.K + (g % p.gpr) * N;
+    return p.D + (static_cast<int64_t>(e) * p.G + g) * N;
+}
+
+// KW consecutive binary16 patterns (one 8- or 4-byte load) and KW consecutive
+// floats (one 16- or 8-byte load): a lane's share of a group of 32 * KW weights.
+template <int KW>
+__device__ __forceinline__ void load_bits(const uint16_t *src, uint32_t (&wb)[KW])
+{
+    if constexpr (KW == 4) {
+        const uint2 v = *reinterpret_cast<const uint2 *>(src);
+        wb[0] = v.x & 0xFFFFu;
+        wb[1] = v.x >> 16;
+        wb[2] = v.y & 0xFFFFu;
+        wb[3] = v.y >> 16;
+    } else {
+        static_assert(KW == 2, "4 or 2 weights per lane");
+        const uint32_t v = *reinterpret_cast<const uint32_t *>(src);
+        wb[0] = v & 0xFFFFu;
+        wb[1] = v >> 16;
+    }
+}
+
+template <int KW>
+__device__ __forceinline__ void load_f(const float *src, float (&v)[KW])
+{
+    if constexpr (KW == 4) {
+        const float4 t = *reinterpret_cast<const float4 *>(src);
+        v[0] = t.x;
+        v[1] = t.y;
+        v[2] = t.z;
+        v[3] = t.w;
+    } else {
+        const float2 t = *reinterpret_cast<const float2 *>(src);
+        v[0] = t.x;
+        v[1] = t.y;
+    }
 }
 
 // fp32 bit patterns of 2^-64 and 2^81, the ends of the diagonal range the fp32
@@ -232,6 +271,44 @@ __device__ __forceinline__ void bitonic_sort_128(uint32_t (&key)[4], int lane)
 #pragma unroll
         for (int x = 0; x < 4; x++)
             key[x] ^= flip;
+    }
+}
+
+// Ascending bitonic sort of 32 * KW keys, lane L holding positions KW*L ..
+// KW*L + KW - 1: block size k doubles from 2; within a block, element p and
+// p ^ j meet for j = k/2 .. 1, in ascending order when p & k == 0.  Partners
+// at distance j >= KW are in lane L ^ (j / KW).  (128 keys use the tuned
+// bitonic_sort_128 above.)
+template <int KW>
+__device__ __forceinline__ void bitonic_sort_lanes(uint32_t (&key)[KW], int lane)
+{
+    constexpr int NK = 32 * KW;
+#pragma unroll
+    for (int k = 2; k <= NK; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            if (j >= KW) {
+                const int lm = j / KW;
+                const bool upper = (lane & lm) != 0;
+#pragma unroll
+                for (int x = 0; x < KW; x++) {
+                    const bool asc = ((KW * lane + x) & k) == 0;
+                    const uint32_t o = __shfl_xor_sync(kFull, key[x], lm);
+                    key[x] = (asc != upper) ? min(key[x], o) : max(key[x], o);
+                }
+            } else {
+#pragma unroll
+                for (int x = 0; x < KW; x++) {
+                    if ((x & j) == 0) {
+                        const int y = x | j;
+                        const bool asc = ((KW * lane + x) & k) == 0;
+                        const uint32_t lo = min(key[x], key[y]), hi = max(key[x], key[y]);
+                        key[x] = asc ? lo : hi;
+                        key[y] = asc ? hi : lo;
+                    }
+                }
+            }
+        }
     }
 }
 
@@ -623,11 +700,13 @@ __device__ __forceinline__ uint32_t pack_lane_codes(const int (&q)[4], int lane)
     return h | (up << 16);  // valid on even lanes: codes 8*(lane/2) .. +7
 }
 
-template <bool kSpec>
+template <bool kSpec, int N>
 __device__ __forceinline__ void write_constant_group(const Params &p, int64_t g, int lane, uint8_t flag)
 {
-    if constexpr (kSpec)
-        reinterpret_cast<uint32_t *>(p.out_q + g * kGroup)[lane] = 0u;
+    if constexpr (kSpec && N == 128)
+        reinterpret_cast<uint32_t *>(p.out_q + g * N)[lane] = 0u;
+    else if constexpr (kSpec)
+        reinterpret_cast<uint16_t *>(p.out_q + g * N)[lane] = 0u;
     else if (lane < 16)
         p.out_codes[g * 16 + lane] = 0x88888888u;
     if (lane == 0) {
@@ -685,7 +764,7 @@ __device__ __forceinline__ void add_delta64(const WarpSmem<E> &sm, uint32_t kk, 
 
 // B_e = sum_i d |w| |q_i(s)| and C_e = sum_i d q_i(s)^2 summed directly over
 // the group (lane L takes ranks 32m + L); every lane gets the same totals.
-template <int E>
+template <int E, int KW>
 __device__ __forceinline__ void direct_coefficients(const WarpSmem<E> &sm, float s, int lane, double (&B)[E],
                                                     double (&C)[E], int qp, int qn)
 {
@@ -695,7 +774,7 @@ __device__ __forceinline__ void direct_coefficients(const WarpSmem<E> &sm, float
         C[e] = 0.0;
     }
 #pragma unroll 1
-    for (int m = 0; m < 4; m++) {
+    for (int m = 0; m < KW; m++) {
         const int r = 32 * m + lane;
         const float wv = sm.w[r];
         const int aq = abs_code(fabsf(wv), s, wv < 0.0f ? qn : qp);
@@ -722,9 +801,10 @@ __device__ __forceinline__ void direct_coefficients(const WarpSmem<E> &sm, float
     }
 }
 
-template <int E, bool kIntersect, bool kSpec>
+template <int E, bool kIntersect, bool kSpec, int N>
 __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int lane, Tally &tl)
 {
+    constexpr int KW = N / 32;  // weights per lane: 4 for groups of 128, 2 for 64
     // Code range: W4 clips at 7 and -8; a general spec (kSpec) at qmax and
     // -nmax, with nmax = qmax or qmax + 1 and at most 8 code layers.  When
     // nmax > qmax the last layer, k = qmax, holds negative weights only.
@@ -732,23 +812,23 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     const int QN = kSpec ? p.nmax : 8;
     const bool negx = QN > QP;
     // ---- 1. load ---------------------------------------------------------
-    const DiagView dv_g = diag_view(p, g);
-    const uint2 wv = *reinterpret_cast<const uint2 *>(p.W + g * kGroup + 4 * lane);
-    const uint32_t wb[4] = {wv.x & 0xFFFFu, wv.x >> 16, wv.y & 0xFFFFu, wv.y >> 16};
+    const DiagView dv_g = diag_view<N>(p, g);
+    uint32_t wb[KW];
+    load_bits<KW>(p.W + g * N + KW * lane, wb);
     bool bad = false, nonzero = false, rare = false;
     double A[E];
 #pragma unroll
-    for (int m = 0; m < 4; m++) {
+    for (int m = 0; m < KW; m++) {
         bad |= (wb[m] & 0x7C00u) == 0x7C00u;
         nonzero |= (wb[m] & 0x7FFFu) != 0u;
     }
 #pragma unroll
     for (int e = 0; e < E; e++) {
-        const float4 dv = *reinterpret_cast<const float4 *>(dv_g.base + e * dv_g.stride + 4 * lane);
-        const float dq[4] = {dv.x, dv.y, dv.z, dv.w};
+        float dq[KW];
+        load_f<KW>(dv_g.base + e * dv_g.stride + KW * lane, dq);
         double a = 0.0;
 #pragma unroll
-        for (int m = 0; m < 4; m++) {
+        for (int m = 0; m < KW; m++) {
             // d outside [2^-64, 2^81]: zero, negative, non-finite or extreme
             rare |= __float_as_uint(dq[m]) - kDLowBits > kDHighBits - kDLowBits;
             const double wd = half_value(wb[m]);
@@ -768,8 +848,8 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
 #pragma unroll
         for (int e = 0; e < E; e++) {
 #pragma unroll
-            for (int m = 0; m < 4; m++) {
-                const float d = dv_g.base[e * dv_g.stride + 4 * lane + m];
+            for (int m = 0; m < KW; m++) {
+                const float d = dv_g.base[e * dv_g.stride + KW * lane + m];
                 bad |= !(d >= 0.0f && d <= FLT_MAX);
                 odd |= d != 0.0f && !(d >= 0x1p-64f && d <= 0x1p81f);
             }
@@ -779,12 +859,12 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     bad = __any_sync(kFull, bad);
     nonzero = __any_sync(kFull, nonzero);
     if (bad) {
-        write_constant_group<kSpec>(p, g, lane, CQ_FLAG_NONFINITE);
+        write_constant_group<kSpec, N>(p, g, lane, CQ_FLAG_NONFINITE);
         tl.nonfinite++;
         return;
     }
     if (!nonzero) {
-        write_constant_group<kSpec>(p, g, lane, CQ_FLAG_TRIVIAL);
+        write_constant_group<kSpec, N>(p, g, lane, CQ_FLAG_TRIVIAL);
         tl.trivial++;
         return;
     }
@@ -806,22 +886,25 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     // ---- 2. order the weights by |w|; stage w and d by rank ----------------
     // After the sort lane L owns ranks r = 32m + L (m = 0..3).
     {
-        uint32_t wk[4];
+        uint32_t wk[KW];
 #pragma unroll
-        for (int m = 0; m < 4; m++)
-            wk[m] = ((wb[m] & 0x7FFFu) << 7) | static_cast<uint32_t>(4 * lane + m);
-        bitonic_sort_128(wk, lane);
+        for (int m = 0; m < KW; m++)
+            wk[m] = ((wb[m] & 0x7FFFu) << 7) | static_cast<uint32_t>(KW * lane + m);
+        if constexpr (N == 128)
+            bitonic_sort_128(wk, lane);
+        else
+            bitonic_sort_lanes<KW>(wk, lane);
 #pragma unroll
-        for (int m = 0; m < 4; m++)
-            sm.bufB[4 * lane + m] = wk[m];
+        for (int m = 0; m < KW; m++)
+            sm.bufB[KW * lane + m] = wk[m];
     }
     __syncwarp();
     int n7 = 0;
 #pragma unroll 1
-    for (int m = 0; m < 4; m++) {
+    for (int m = 0; m < KW; m++) {
         const uint32_t k = sm.bufB[32 * m + lane];
         const int i = k & 127;
-        const uint32_t bits = p.W[g * kGroup + i];
+        const uint32_t bits = p.W[g * N + i];
         const int r = 32 * m + lane;
         sm.w[r] = half_value(bits);
 #pragma unroll
@@ -836,13 +919,13 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         n7 += __popc(bn);
     }
     if (lane == 0)
-        sm.negpre[kGroup] = static_cast<uint8_t>(n7);
+        sm.negpre[N] = static_cast<uint8_t>(n7);
     __syncwarp();
 
     // ---- 3. a rigorous upper bound U of the minimum -----------------------
     // The fp32 objective at three grid scales near the AbsMax scale |w|max/7,
     // widened by 2^-18 (>= 12 fp32 roundings of nonnegative terms).
-    const float amax = fabsf(sm.w[kGroup - 1]);
+    const float amax = fabsf(sm.w[N - 1]);
     const float invq = kSpec ? 1.0f / static_cast<float>(QP) : (1.0f / 7.0f);
     const uint32_t ja0 = min(max(static_cast<uint32_t>(__half_as_ushort(__float2half_rn(amax * invq))), 1u), kLast);
     float U;
@@ -859,19 +942,14 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
 #pragma unroll
             for (int e = 0; e < E; e++)
                 acc[c][e] = 0.0f;
-        const float4 w4 = *reinterpret_cast<const float4 *>(&sm.w[4 * lane]);
-        const float wq[4] = {w4.x, w4.y, w4.z, w4.w};
-        float dq[E][4];
+        float wq[KW];
+        load_f<KW>(&sm.w[KW * lane], wq);
+        float dq[E][KW];
 #pragma unroll
-        for (int e = 0; e < E; e++) {
-            const float4 t = *reinterpret_cast<const float4 *>(&sm.d[e][4 * lane]);
-            dq[e][0] = t.x;
-            dq[e][1] = t.y;
-            dq[e][2] = t.z;
-            dq[e][3] = t.w;
-        }
+        for (int e = 0; e < E; e++)
+            load_f<KW>(&sm.d[e][KW * lane], dq[e]);
 #pragma unroll
-        for (int m = 0; m < 4; m++) {
+        for (int m = 0; m < KW; m++) {
             const float wv = wq[m];
             const float aw = fabsf(wv);
             const int K = wv < 0.0f ? QN : QP;
@@ -909,19 +987,24 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     uint32_t J0 = 1u, J1 = kLast;
     {
         // prefix sums over ranks of d w^2 (fp32), ph[e][c] = sum over ranks < c
-        float *ph = reinterpret_cast<float *>(sm.bufB);  // [E][kGroup + 1]
-        // lane L sums ranks 4L .. 4L+3 locally, then one warp scan per environment
-        // (w^2 is exact; each entry passes through at most 10 fp32 roundings)
-        const float4 w4 = *reinterpret_cast<const float4 *>(&sm.w[4 * lane]);
-        const float q0 = w4.x * w4.x, q1 = w4.y * w4.y, q2 = w4.z * w4.z, q3 = w4.w * w4.w;
+        float *ph = reinterpret_cast<float *>(sm.bufB);  // [E][N + 1]
+        // lane L sums ranks KW*L .. KW*L+KW-1 locally, then one warp scan per
+        // environment (w^2 is exact; each entry passes through at most 10 fp32
+        // roundings)
+        float wq[KW], q2[KW];
+        load_f<KW>(&sm.w[KW * lane], wq);
+#pragma unroll
+        for (int m = 0; m < KW; m++)
+            q2[m] = wq[m] * wq[m];
 #pragma unroll
         for (int e = 0; e < E; e++) {
-            const float4 d4 = *reinterpret_cast<const float4 *>(&sm.d[e][4 * lane]);
-            const float a0 = d4.x * q0;
-            const float a1 = fmaf(d4.y, q1, a0);
-            const float a2 = fmaf(d4.z, q2, a1);
-            const float a3 = fmaf(d4.w, q3, a2);
-            float v = a3;
+            float dq[KW], a[KW];
+            load_f<KW>(&sm.d[e][KW * lane], dq);
+            a[0] = dq[0] * q2[0];
+#pragma unroll
+            for (int m = 1; m < KW; m++)
+                a[m] = fmaf(dq[m], q2[m], a[m - 1]);
+            float v = a[KW - 1];
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const float u = __shfl_up_sync(kFull, v, o);
@@ -930,13 +1013,12 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
             }
             const float before = __shfl_up_sync(kFull, v, 1);  // sum over lanes < L
             const float base = lane == 0 ? 0.0f : before;
-            float *row = ph + e * (kGroup + 1) + 4 * lane;
+            float *row = ph + e * (N + 1) + KW * lane;
             if (lane == 0)
                 row[0] = 0.0f;
-            row[1] = base + a0;
-            row[2] = base + a1;
-            row[3] = base + a2;
-            row[4] = base + a3;
+#pragma unroll
+            for (int m = 0; m < KW; m++)
+                row[m + 1] = base + a[m];
         }
         // lower end: clip bound of the top 8 weights at scale ja0 - 128 * lane
         const uint32_t jl = ja0 > 128u * lane ? ja0 - 128u * lane : 1u;
@@ -948,7 +1030,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
             for (int e = 0; e < E; e++)
                 le[e] = 0.0f;
 #pragma unroll 1
-            for (int r = kGroup - 8; r < kGroup; r++) {
+            for (int r = N - 8; r < N; r++) {
                 const float wv = sm.w[r];
                 const float ex = fmaxf(fmaf(-static_cast<float>(wv < 0.0f ? QN : QP), sl, fabsf(wv)), 0.0f);
                 const float e2 = ex * ex;
@@ -969,7 +1051,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         // upper end: round-to-zero bound at scale ja0 + 128 * lane
         const uint32_t jh = min(ja0 + 128u * lane, kLast);
         const float half_s = 0.5f * grid_value(jh);
-        int lo = 0, hi = kGroup;
+        int lo = 0, hi = N;
         while (lo < hi) {
             const int mid = (lo + hi) >> 1;
             if (fabsf(sm.w[mid]) <= half_s)
@@ -980,7 +1062,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         float H = 0.0f;
 #pragma unroll
         for (int e = 0; e < E; e++)
-            H = fmaxf(H, ph[e * (kGroup + 1) + lo]);
+            H = fmaxf(H, ph[e * (N + 1) + lo]);
         const unsigned cut_hi = __ballot_sync(kFull, H * (1.0f - 0x1p-18f) > U);
         if (cut_hi) {
             const int j1 = __ffs(cut_hi) - 1;  // smallest excluded scale
@@ -1005,7 +1087,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     if (lane < 16) {
         const int k = lane & 7;
         const float sx = (lane < 8) ? sJ0 : sJ1;
-        int lo = 0, hi = kGroup;
+        int lo = 0, hi = N;
         while (lo < hi) {
             const int mid = (lo + hi) >> 1;
             if (!code_at_least(fabsf(sm.w[mid]), sx, k + 1))
@@ -1015,7 +1097,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         }
         const bool empty = k >= QN;  // no code layer k in this range
         sm.lay[lane] = empty ? 0 : ((negx && k == QP) ? sm.negpre[lo] : lo);  // lanes 0..7: F0_k, 8..15: F1_k
-        sm.lay[16 + lane] = empty ? kGroup : lo;                               // the same as rank thresholds
+        sm.lay[16 + lane] = empty ? N : lo;                               // the same as rank thresholds
     }
     __syncwarp();
     const int *off = sm.lay;  // layer k holds ranks [off[k], off[k + 8]) (layer 7: negative ranks)
@@ -1036,7 +1118,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     for (int k = 0; k < 16; k++)
         th[k] = sm.lay[16 + k];
 #pragma unroll 1
-    for (int m = 0; m < 4; m++) {
+    for (int m = 0; m < KW; m++) {
         const int r = 32 * m + lane;
         const float wv = sm.w[r];
         const float aw = fabsf(wv);
@@ -1214,7 +1296,10 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         if (x >= 0 || lane == 0)
             lbs[x >= 0 ? x * 32 + lane : 1024] = run ? lbv : INFINITY;
         ub_lane = run ? fminf(ub_lane, ubv) : ub_lane;
-        const int r = (kk >> 3) & 127;
+        // A padding key adds d * 0 at the rank its bits decode to, 127: staged
+        // and finite in a 128-weight group, but past a 64-weight one, so there
+        // rank 0 stands in.
+        const int r = (N == 128 || valid) ? static_cast<int>((kk >> 3) & 127) : 0;
         const float aw = valid ? fabsf(sm.w[r]) : 0.0f;
         const float cc = valid ? static_cast<float>(2 * (kk & 7) + 1) : 0.0f;
 #pragma unroll
@@ -1304,7 +1389,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         for (int si = 0; si < nb; si++) {
             const SurvEntry en = ent[base + si];
             if (cur == -2 || cur - en.pos > kWalkMax) {
-                direct_coefficients<E>(sm, grid_value(en.ja), lane, Bc, Cc, QP, QN);
+                direct_coefficients<E, KW>(sm, grid_value(en.ja), lane, Bc, Cc, QP, QN);
             } else {
                 // add the deltas of positions cur, cur-1, ..., en.pos+1
                 int lp = cur / c, x = cur - lp * c;
@@ -1526,15 +1611,15 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         // reported objective are the oracle's bit for bit.  Lane L forms the
         // terms of weights 4L..4L+3; lanes 0..3 sum four environments' 128
         // terms in order through shared memory.
-        double *terms = reinterpret_cast<double *>(sm.bufA);  // [4][kGroup]
+        double *terms = reinterpret_cast<double *>(sm.bufA);  // [4][N]
 #pragma unroll 1
         for (int f = 0; f < (only ? 0 : total); f++) {
             const uint32_t j = static_cast<uint32_t>(fin[f]);
             const float s = grid_value(j);
             const double sd = s;
-            double rr[4];
+            double rr[KW];
 #pragma unroll
-            for (int m = 0; m < 4; m++) {
+            for (int m = 0; m < KW; m++) {
                 const bool neg = (wb[m] & 0x8000u) != 0u;
                 const int aq = abs_code(half_value(wb[m] & 0x7FFFu), s, neg ? QN : QP);
                 const double r_ = static_cast<double>(half_value(wb[m])) - sd * static_cast<double>(neg ? -aq : aq);
@@ -1545,18 +1630,18 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
             for (int e0 = 0; e0 < E; e0 += 4) {
 #pragma unroll
                 for (int e = e0; e < E && e < e0 + 4; e++) {
-                    const float4 dv = *reinterpret_cast<const float4 *>(dv_g.base + e * dv_g.stride + 4 * lane);
-                    const float dq[4] = {dv.x, dv.y, dv.z, dv.w};
+                    float dq[KW];
+                    load_f<KW>(dv_g.base + e * dv_g.stride + KW * lane, dq);
 #pragma unroll
-                    for (int m = 0; m < 4; m++)
-                        terms[(e - e0) * kGroup + 4 * lane + m] = __dmul_rn(static_cast<double>(dq[m]), rr[m]);
+                    for (int m = 0; m < KW; m++)
+                        terms[(e - e0) * N + KW * lane + m] = __dmul_rn(static_cast<double>(dq[m]), rr[m]);
                 }
                 __syncwarp();
                 double a = 0.0;
                 if (lane < 4 && e0 + lane < E) {
 #pragma unroll 8
-                    for (int i = 0; i < kGroup; i++)
-                        a = __dadd_rn(a, terms[lane * kGroup + i]);
+                    for (int i = 0; i < N; i++)
+                        a = __dadd_rn(a, terms[lane * N + i]);
                 }
 #pragma unroll
                 for (int e = e0; e < E && e < e0 + 4; e++)
@@ -1586,7 +1671,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
             for (int e = 0; e < E; e++)
                 acc[e] = 0.0;
 #pragma unroll 1
-            for (int m = 0; m < 4; m++) {
+            for (int m = 0; m < KW; m++) {
                 const int r = 32 * m + lane;
                 const float wv = sm.w[r];
                 const int aq = abs_code(fabsf(wv), s, wv < 0.0f ? 8 : 7);
@@ -1613,9 +1698,9 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
 
     // ---- 10. pack and store ---------------------------------------------------
     const float s = grid_value(bj);
-    int q[4];
+    int q[KW];
 #pragma unroll
-    for (int m = 0; m < 4; m++) {
+    for (int m = 0; m < KW; m++) {
         const int aq = abs_code(half_value(wb[m] & 0x7FFFu), s, (wb[m] & 0x8000u) ? QN : QP);
         q[m] = (wb[m] & 0x8000u) ? -aq : aq;
     }
@@ -1623,9 +1708,12 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     if constexpr (kSpec) {
         uint32_t word = 0;
 #pragma unroll
-        for (int m = 0; m < 4; m++)
+        for (int m = 0; m < KW; m++)
             word |= static_cast<uint32_t>(q[m] & 0xFF) << (8 * m);
-        reinterpret_cast<uint32_t *>(p.out_q + g * kGroup)[lane] = word;  // the codes q as int8
+        if constexpr (KW == 4)
+            reinterpret_cast<uint32_t *>(p.out_q + g * N)[lane] = word;  // the codes q as int8
+        else
+            reinterpret_cast<uint16_t *>(p.out_q + g * N)[lane] = static_cast<uint16_t>(word);
     } else {
         const uint32_t word = pack_lane_codes(q, lane);
         if ((lane & 1) == 0)
@@ -1642,7 +1730,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     tl.finalists += static_cast<uint32_t>(total);
 }
 
-template <int E, bool kIntersect, bool kSpec>
+template <int E, bool kIntersect, bool kSpec, int N>
 __global__ void __launch_bounds__(kWarpsPerCta<E> * 32, 1) select_kernel(Params p)
 {
     constexpr int kWarps = kWarpsPerCta<E>;
@@ -1656,9 +1744,9 @@ __global__ void __launch_bounds__(kWarpsPerCta<E> * 32, 1) select_kernel(Params 
     for (int64_t b0 = static_cast<int64_t>(blockIdx.x) * kWarps; b0 < p.G; b0 += stride) {
         const int64_t g = b0 + wib;
         if (g < p.G) {
-            if (lane < 2 && g + stride < p.G)
-                asm volatile("prefetch.global.L2 [%0];" ::"l"(p.W + (g + stride) * kGroup + 64 * lane));
-            process_group<E, kIntersect, kSpec>(p, sm, g, lane, tl);
+            if (lane < N / 64 && g + stride < p.G)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(p.W + (g + stride) * N + 64 * lane));
+            process_group<E, kIntersect, kSpec, N>(p, sm, g, lane, tl);
         }
         __syncthreads();  // the warps start the next group together
     }
@@ -1693,7 +1781,7 @@ __device__ __forceinline__ Best3 combine(Best3 a, Best3 b)
     return b;
 }
 
-template <int E, bool kSpec>
+template <int E, bool kSpec, int N>
 __global__ void __launch_bounds__(kExThreads) exhaustive_kernel(Params p)
 {
     const int QP = kSpec ? p.qmax : 7, QN = kSpec ? p.nmax : 8;
@@ -1708,12 +1796,12 @@ __global__ void __launch_bounds__(kExThreads) exhaustive_kernel(Params p)
         const uint2 qe = p.queue[qi];
         const int64_t g = qe.x;
         const uint32_t j0 = qe.y & 0xFFFFu, j1 = qe.y >> 16;
-        if (tid < kGroup) {
-            ws[tid] = half_value(p.W[g * kGroup + tid]);
+        if (tid < N) {
+            ws[tid] = half_value(p.W[g * N + tid]);
             wsd[tid] = ws[tid];
 #pragma unroll
             for (int e = 0; e < E; e++)
-                ds[e][tid] = diag_ptr(p, g, e)[tid];
+                ds[e][tid] = diag_ptr<N>(p, g, e)[tid];
         }
         __syncthreads();
         Best3 b{INFINITY, INFINITY, 0u};
@@ -1725,7 +1813,7 @@ __global__ void __launch_bounds__(kExThreads) exhaustive_kernel(Params p)
             for (int e = 0; e < E; e++)
                 acc[e] = 0.0;
             // the definition's own order: i ascending, one sum per environment
-            for (int i = 0; i < kGroup; i++) {
+            for (int i = 0; i < N; i++) {
                 const float w = ws[i];
                 const int aq = abs_code(fabsf(w), s, w < 0.0f ? QN : QP);
                 const double q = (w < 0.0f) ? -static_cast<double>(aq) : static_cast<double>(aq);
@@ -1766,13 +1854,13 @@ __global__ void __launch_bounds__(kExThreads) exhaustive_kernel(Params p)
         }
         __syncthreads();
         const Best3 r = red[0];
-        if (tid < kGroup) {
+        if (tid < N) {
             const float w = ws[tid];
             const float s = grid_value(r.j);
             const int aq = abs_code(fabsf(w), s, w < 0.0f ? QN : QP);
             const int q = (w < 0.0f) ? -aq : aq;
             if constexpr (kSpec)
-                p.out_q[g * kGroup + tid] = static_cast<int8_t>(q);
+                p.out_q[g * N + tid] = static_cast<int8_t>(q);
             else
                 nib[tid] = static_cast<uint32_t>((q + 8) & 0xF);
         }
@@ -1863,17 +1951,17 @@ cudaError_t pool_alloc(void **ptr, size_t bytes, cudaStream_t st)
     return cudaMallocFromPoolAsync(ptr, bytes, g_pool[dev], st);
 }
 
-template <int E, bool kIntersect, bool kSpec>
+template <int E, bool kIntersect, bool kSpec, int N>
 cudaError_t launch_main(const Params &p, cudaStream_t st, int sms)
 {
     constexpr int kWarps = kWarpsPerCta<E>;
     const size_t smem = sizeof(WarpSmem<E>) * kWarps;
-    cudaError_t err = cudaFuncSetAttribute(select_kernel<E, kIntersect, kSpec>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t err = cudaFuncSetAttribute(select_kernel<E, kIntersect, kSpec, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
     if (err != cudaSuccess)
         return err;
     int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel<E, kIntersect, kSpec>, kWarps * 32, smem);
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel<E, kIntersect, kSpec, N>, kWarps * 32, smem);
     if (err != cudaSuccess)
         return err;
     if (per_sm < 1)
@@ -1882,7 +1970,7 @@ cudaError_t launch_main(const Params &p, cudaStream_t st, int sms)
     const int64_t grid = need < static_cast<int64_t>(sms) * per_sm ? need : static_cast<int64_t>(sms) * per_sm;
     if (p.ev_begin && (err = cudaEventRecord(p.ev_begin, st)) != cudaSuccess)
         return err;
-    select_kernel<E, kIntersect, kSpec><<<static_cast<unsigned>(grid), kWarps * 32, smem, st>>>(p);
+    select_kernel<E, kIntersect, kSpec, N><<<static_cast<unsigned>(grid), kWarps * 32, smem, st>>>(p);
     err = cudaGetLastError();
     if (err != cudaSuccess)
         return err;
@@ -1900,15 +1988,22 @@ cudaError_t launch(const Params &p, cudaStream_t st)
         return err;
     const int sms = sm_count(dev);
     if (p.out_q) {  // a general spec (the W4 search's code range from p.qmax, p.nmax)
-        if ((err = launch_main<E, false, true>(p, st, sms)) != cudaSuccess)
-            return err;
-        exhaustive_kernel<E, true><<<static_cast<unsigned>(2 * sms), kExThreads, 0, st>>>(p);
+        if (p.group == 64) {
+            if ((err = launch_main<E, false, true, 64>(p, st, sms)) != cudaSuccess)
+                return err;
+            exhaustive_kernel<E, true, 64><<<static_cast<unsigned>(2 * sms), kExThreads, 0, st>>>(p);
+        } else {
+            if ((err = launch_main<E, false, true, 128>(p, st, sms)) != cudaSuccess)
+                return err;
+            exhaustive_kernel<E, true, 128><<<static_cast<unsigned>(2 * sms), kExThreads, 0, st>>>(p);
+        }
         return cudaGetLastError();
     }
-    err = p.intersections ? launch_main<E, true, false>(p, st, sms) : launch_main<E, false, false>(p, st, sms);
+    err = p.intersections ? launch_main<E, true, false, 128>(p, st, sms)
+                          : launch_main<E, false, false, 128>(p, st, sms);
     if (err != cudaSuccess)
         return err;
-    exhaustive_kernel<E, false><<<static_cast<unsigned>(2 * sms), kExThreads, 0, st>>>(p);
+    exhaustive_kernel<E, false, 128><<<static_cast<unsigned>(2 * sms), kExThreads, 0, st>>>(p);
     return cudaGetLastError();
 }
 
@@ -1984,7 +2079,7 @@ cudaError_t noalloc_scratch(void **ptr)
     return cudaSuccess;
 }
 
-// A general spec through the W4 kernel's search, for group size 128 and a
+// A general spec through the W4 kernel's search, for group size 128 or 64 and a
 // code range [-nmax, qmax] with nmax = qmax or qmax + 1 and nmax <= 8 (the
 // 2-, 3- and 4-bit ranges and the symmetric ones): the same transitions,
 // window, screen and certified run search with the range's caps, the
@@ -1993,11 +2088,11 @@ cudaError_t noalloc_scratch(void **ptr)
 // the caller can take the general kernel.  Shapes are validated by the caller.
 // The workspace comes from the library pool, like cq_select_scales.
 cq_status select_spec_fast(const uint16_t *W, int64_t G, const float *D, int E, int64_t K, int qmin, int qmax,
-                           uint16_t *out_scales, int8_t *out_q, double *out_obj, uint8_t *out_flags,
+                           int n, uint16_t *out_scales, int8_t *out_q, double *out_obj, uint8_t *out_flags,
                            cudaStream_t st)
 {
     const int nmax = -qmin;
-    if (!(qmax >= 1 && nmax <= 8 && (nmax == qmax || nmax == qmax + 1)))
+    if (!(qmax >= 1 && nmax <= 8 && (nmax == qmax || nmax == qmax + 1)) || (n != kGroup && n != 64))
         return CQ_ERR_UNSUPPORTED;
     if (!aligned(W, 16) || !aligned(D, 16) || !aligned(out_q, 4) || !aligned(out_scales, 2) ||
         (out_obj && !aligned(out_obj, 8)))
@@ -2007,9 +2102,10 @@ cq_status select_spec_fast(const uint16_t *W, int64_t G, const float *D, int E, 
     p.D = D;
     p.G = G;
     p.K = K;
-    p.gpr = K > 0 ? K / kGroup : 1;
+    p.gpr = K > 0 ? K / n : 1;
     p.out_scales = out_scales;
     p.out_codes = nullptr;
+    p.group = n;
     p.out_obj = out_obj;
     p.out_flags = out_flags;
     p.finalist_cap = kDefaultFinalists;
@@ -2076,6 +2172,7 @@ cq_status cq_select_scales_ex(const uint16_t *W, int64_t G, const float *D, int 
     p.qmax = 7;
     p.nmax = 8;
     p.out_q = nullptr;
+    p.group = kGroup;
     p.flag_rel_gap = 1e-12;
     p.ev_begin = nullptr;
     p.ev_end = nullptr;

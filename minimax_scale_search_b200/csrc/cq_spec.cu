@@ -607,7 +607,7 @@ cudaError_t launch_spec(const SpecParams &p, cudaStream_t st)
 
 // The W4 kernel's search for eligible specs (cq_select.cu).
 cq_status select_spec_fast(const uint16_t *W, int64_t G, const float *D, int E, int64_t K, int qmin, int qmax,
-                           uint16_t *out_scales, int8_t *out_q, double *out_obj, uint8_t *out_flags,
+                           int n, uint16_t *out_scales, int8_t *out_q, double *out_obj, uint8_t *out_flags,
                            cudaStream_t st);
 }  // namespace cq
 
@@ -638,8 +638,8 @@ cq_status cq_select_scales_spec(const uint16_t *W, int64_t G, const float *D, in
         return CQ_ERR_INVALID_ARG;
     if (spec->kernel != CQ_SPEC_KERNEL_AUTO && spec->kernel != CQ_SPEC_KERNEL_GENERAL)
         return CQ_ERR_INVALID_ARG;
-    if (n == kGroup && spec->kernel == CQ_SPEC_KERNEL_AUTO) {
-        const cq_status fs = select_spec_fast(W, G, D, E, K, spec->qmin, spec->qmax, out_scales, out_codes,
+    if ((n == kGroup || n == 64) && spec->kernel == CQ_SPEC_KERNEL_AUTO) {
+        const cq_status fs = select_spec_fast(W, G, D, E, K, spec->qmin, spec->qmax, n, out_scales, out_codes,
                                               out_objective, out_flags, static_cast<cudaStream_t>(stream));
         if (fs != CQ_ERR_UNSUPPORTED)
             return fs;

@@ -109,33 +109,55 @@ def _run_kernel(W, D, qmin, qmax, n, K, general):
             r.flags.cpu().numpy())
 
 
+@pytest.mark.parametrize("n", [128, 64])
 @pytest.mark.parametrize("spec", [(-8, 7), (-4, 3), (-2, 1), (-1, 1), (-8, 8), (-5, 4)])
-def test_w4_search_and_general_kernel_same_bytes(spec):
-    """Group size 128 with |qmin| = qmax or qmax + 1 runs the W4 kernel's
-    search; the general kernel is the other implementation of the same
-    definition.  On 262,144 sweep groups every scale, code, objective and flag
-    is the same, and a sample meets the oracle."""
+def test_w4_search_and_general_kernel_same_bytes(spec, n):
+    """Group size 128 or 64 with |qmin| = qmax or qmax + 1 runs the W4
+    kernel's search; the general kernel is the other implementation of the
+    same definition.  On the first 2,048 sweep rows (262,144 groups of 128,
+    524,288 of 64) every scale, code, objective and flag is the same, and a
+    sample meets the oracle."""
     qmin, qmax = spec
     wl = synth.workload(3)
     W = synth.make_weights(3, 0, 2048)
     D = synth.make_diagonals(3)
-    a = _run_kernel(W, D, qmin, qmax, 128, wl.cols, general=False)
-    b = _run_kernel(W, D, qmin, qmax, 128, wl.cols, general=True)
+    a = _run_kernel(W, D, qmin, qmax, n, wl.cols, general=False)
+    b = _run_kernel(W, D, qmin, qmax, n, wl.cols, general=True)
     for x, y, name in zip(a, b, ("scales", "codes", "objective", "flags")):
-        assert np.array_equal(x.view(np.uint8), y.view(np.uint8)), (spec, name)
-    sel = synth.sample_groups(3, 20_000, seed=29)
-    sel = sel[sel < W.size // 128][:600]
-    Wg = W.reshape(-1, 128)[sel]
-    Dg = np.ascontiguousarray(D.reshape(4, -1, 128)[:, sel % wl.groups_per_row, :])
+        assert np.array_equal(x.view(np.uint8), y.view(np.uint8)), (spec, n, name)
+    G = W.size // n
+    sel = np.sort(np.random.default_rng(29 + n).choice(G, 600, replace=False))
+    gpr = wl.cols // n
+    Wg = W.reshape(-1, n)[sel]
+    Dg = np.ascontiguousarray(D.reshape(4, gpr, n)[:, sel % gpr, :])
     o = oracle.solve(Wg, Dg, qmin=qmin, qmax=qmax, threads=oracle_threads())
-    assert np.array_equal(a[0][sel], o["best_bits"]), spec
-    assert np.array_equal(a[1][sel], o["codes"][:, :128]), spec
-    assert np.array_equal(a[2][sel].view(np.uint64), o["best_obj"].view(np.uint64)), spec
+    assert np.array_equal(a[0][sel], o["best_bits"]), (spec, n)
+    assert np.array_equal(a[1][sel], o["codes"][:, :n]), (spec, n)
+    assert np.array_equal(a[2][sel].view(np.uint64), o["best_obj"].view(np.uint64)), (spec, n)
 
 
 @pytest.mark.parametrize("E", [1, 2, 3, 5, 8])
 def test_w4_search_each_environment_count(E):
-    W = _groups(160, 128, seed=200 + E)
-    D = _diag(E, 160, 128, seed=300 + E, sigma=2.0)
-    for qmin, qmax in ((-4, 3), (-2, 1), (-8, 8)):
-        _check(W, D, qmin, qmax, 128, where=f"E={E} spec ({qmin}, {qmax})")
+    for n in (128, 64):
+        W = _groups(160, n, seed=200 + E)
+        D = _diag(E, 160, n, seed=300 + E, sigma=2.0)
+        for qmin, qmax in ((-4, 3), (-2, 1), (-8, 8), (-8, 7)):
+            _check(W, D, qmin, qmax, n, where=f"E={E} n={n} spec ({qmin}, {qmax})")
+
+
+def test_w4_search_group64_stress_and_edges():
+    """Group size 64 on the tie/stress workload's classes (exact multiples,
+    zero and single-nonzero halves of groups) and on edge groups."""
+    cls = synth.stress_classes()
+    pick = np.sort(np.concatenate([np.nonzero(cls == c)[0][:40] for c in range(5)]))
+    Wg, Dg = synth.group_rows(4, pick)
+    W64 = np.ascontiguousarray(Wg.reshape(-1, 64))
+    D64 = np.ascontiguousarray(Dg.reshape(Dg.shape[0], -1, 64))
+    _check(W64, D64, -8, 7, 64, where="stress n=64")
+    Wb = _groups(6, 64, seed=3)
+    Wb[1, 5] = 0x7C00
+    Wb[2, :] = 0
+    Wb[3, 0] = 0xFE00
+    s, c, f, fl = _run(Wb, _diag(2, 6, 64), -8, 7, 64)
+    assert list(fl[:4]) == [0, 8, 1, 8]
+    assert np.all(s[1:4] == 1) and np.all(c[1:4] == 0) and np.all(f[1:4] == 0)
