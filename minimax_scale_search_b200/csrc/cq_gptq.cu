@@ -14,8 +14,8 @@
 // nibbles (q + 8), low nibble first: word j of group (r, c) is exactly
 // qweight[16c + j][r].  So the export is a transpose of the [R][K/8] word
 // matrix, a transpose of the [R][K/128] scale matrix and two constant fills;
-// all are HBM-bound and run as 32 x 32 tiles through shared memory (reads and
-// writes both coalesced).
+// all are HBM-bound; the transposes run as 64 x 64 tiles through shared memory
+// (reads and writes both coalesced, 256-byte runs), the dequantiser as 32 x 32.
 
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -32,28 +32,32 @@ constexpr int kTileRowsPerPass = 8;  // transpose: CTA of 32 x 8 threads, 4 elem
 constexpr int kDequantRows = 4;      // dequantisation: CTA of 32 x 4 threads, 8 words per thread, so 16 CTAs
                                      // (twice the loads in flight) fit per SM
 
-// dst[c][r] = src[r][c] for an [rows][cols] matrix, one 32 x 32 tile per CTA
-// iteration (grid-stride over tiles).
+constexpr int kBigTile = 64;         // transpose tile edge
+constexpr int kBigRows = 4;          // CTA of 64 x 4 threads, 16 elements per thread
+
+// dst[c][r] = src[r][c] for an [rows][cols] matrix, one 64 x 64 tile per CTA
+// iteration (grid-stride over tiles): every row segment read and written is
+// 64 elements long, and a thread has 16 loads in flight.
 template <typename T>
-__global__ void __launch_bounds__(kTile * kTileRowsPerPass) transpose_kernel(const T *__restrict__ src, int64_t rows,
-                                                                            int64_t cols, T *__restrict__ dst)
+__global__ void __launch_bounds__(kBigTile * kBigRows) transpose_kernel(const T *__restrict__ src, int64_t rows,
+                                                                       int64_t cols, T *__restrict__ dst)
 {
-    __shared__ T tile[kTile][kTile + 1];
-    const int64_t tiles_c = (cols + kTile - 1) / kTile;
-    const int64_t tiles = ((rows + kTile - 1) / kTile) * tiles_c;
+    __shared__ T tile[kBigTile][kBigTile + 1];
+    const int64_t tiles_c = (cols + kBigTile - 1) / kBigTile;
+    const int64_t tiles = ((rows + kBigTile - 1) / kBigTile) * tiles_c;
     const int tx = threadIdx.x, ty = threadIdx.y;
     for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
-        const int64_t r0 = (t / tiles_c) * kTile, c0 = (t % tiles_c) * kTile;
+        const int64_t r0 = (t / tiles_c) * kBigTile, c0 = (t % tiles_c) * kBigTile;
         __syncthreads();
 #pragma unroll
-        for (int k = 0; k < kTile; k += kTileRowsPerPass) {
+        for (int k = 0; k < kBigTile; k += kBigRows) {
             const int64_t r = r0 + ty + k, c = c0 + tx;
             if (r < rows && c < cols)
                 tile[ty + k][tx] = src[r * cols + c];
         }
         __syncthreads();
 #pragma unroll
-        for (int k = 0; k < kTile; k += kTileRowsPerPass) {
+        for (int k = 0; k < kBigTile; k += kBigRows) {
             const int64_t c = c0 + ty + k, r = r0 + tx;
             if (r < rows && c < cols)
                 dst[c * rows + r] = tile[tx][ty + k];
@@ -221,13 +225,13 @@ cq_status cq_gptq_export(const uint16_t *scales, const uint32_t *codes, int64_t 
         !aligned(g_idx, 4))
         return CQ_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const dim3 block(kTile, kTileRowsPerPass);
+    const dim3 block(kBigTile, kBigRows);
     const int64_t K8 = K / 8, ng = K / 128;
-    transpose_kernel<uint32_t><<<tile_grid(((R + 31) / 32) * ((K8 + 31) / 32)), block, 0, s>>>(
+    transpose_kernel<uint32_t><<<tile_grid(((R + 63) / 64) * ((K8 + 63) / 64)), block, 0, s>>>(
         codes, R, K8, reinterpret_cast<uint32_t *>(qweight));
     if (cudaGetLastError() != cudaSuccess)
         return CQ_ERR_CUDA;
-    transpose_kernel<uint16_t><<<tile_grid(((R + 31) / 32) * ((ng + 31) / 32)), block, 0, s>>>(scales, R, ng,
+    transpose_kernel<uint16_t><<<tile_grid(((R + 63) / 64) * ((ng + 63) / 64)), block, 0, s>>>(scales, R, ng,
                                                                                                gptq_scales);
     if (cudaGetLastError() != cudaSuccess)
         return CQ_ERR_CUDA;
