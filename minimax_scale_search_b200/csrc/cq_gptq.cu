@@ -28,7 +28,6 @@ namespace cq {
 namespace {
 
 constexpr int kTile = 32;
-constexpr int kTileRowsPerPass = 8;  // transpose: CTA of 32 x 8 threads, 4 elements per thread
 constexpr int kDequantRows = 4;      // dequantisation: CTA of 32 x 4 threads, 8 words per thread, so 16 CTAs
                                      // (twice the loads in flight) fit per SM
 
