@@ -509,8 +509,8 @@ SPEC_CASES = ((-8, 7, 128), (-4, 3, 128), (-2, 1, 128), (-8, 7, 64), (-16, 15, 1
 
 def spec_uses_w4_search(qmin: int, qmax: int, n: int) -> bool:
     """Whether cq_select_scales_spec runs the W4 kernel's search for this spec
-    (group size 128 or 64, |qmin| = qmax or qmax + 1, at most 8)."""
-    return n in (128, 64) and qmax >= 1 and -qmin <= 8 and -qmin in (qmax, qmax + 1)
+    (|qmin| = qmax or qmax + 1; at most 16 at group size 128, 8 at 64)."""
+    return (n == 128 and -qmin <= 16 or n == 64 and -qmin <= 8) and qmax >= 1 and -qmin in (qmax, qmax + 1)
 
 
 def bench_spec(args, wl, dev):

@@ -247,8 +247,9 @@ cq_status cq_estimate_diagonals(const void *X, int dtype, int64_t K, const int64
  * such groups get scale 0x0001, zero codes and objective 0).  Scales, codes
  * and objectives are the definition's own fp64 values, bit for bit.
  *
- * Two kernels serve it.  Group size 128 or 64 with a code range [-m, m] or
- * [-m, m - 1], m <= 8 (the 2-, 3- and 4-bit ranges and the symmetric ones),
+ * Two kernels serve it.  A code range [-m, m] or [-m, m - 1] with m <= 16 at
+ * group size 128, or m <= 8 at group size 64 (the 2- to 5-bit ranges and the
+ * symmetric ones),
  * and W, D 16-byte aligned, out_codes 4-byte aligned: the W4 kernel's search
  * with that range's caps, its finalists rescored in the definition's order;
  * this takes a workspace from the library pool, like cq_select_scales.  Any

@@ -431,9 +431,9 @@ def select_scales_spec(W, D, K: int | None = None, *, qmin: int = -8, qmax: int 
     group_size weights).  W: CUDA 16-bit binary16 patterns whose last dimension
     is a multiple of group_size; D: float32 per column [E, K] or per group
     [E, G, group_size].  Returns scales int16 [G] and codes int8 [G, group_size]
-    (the q values).  Group size 128 or 64 with qmin = -qmax or -qmax - 1
-    (|qmin| <= 8) runs the W4 kernel's search; general_kernel=True forces the
-    general one."""
+    (the q values).  qmin = -qmax or -qmax - 1 with |qmin| <= 16 at group size
+    128, or <= 8 at 64, runs the W4 kernel's search; general_kernel=True forces
+    the general one."""
     import torch
     n = int(group_size)
     if not (W.is_cuda and D.is_cuda and W.is_contiguous() and D.is_contiguous()):

@@ -166,9 +166,10 @@ __device__ __forceinline__ void load_f(const float *src, float (&v)[KW])
 // screens are sound for.
 constexpr uint32_t kDLowBits = 0x1F800000u, kDHighBits = 0x68000000u;
 
-// 1 / (k + 1/2), k = 0..7 (only an estimate's accuracy is needed).
-__constant__ float c_inv_half[8] = {2.0f, 2.0f / 3.0f, 2.0f / 5.0f, 2.0f / 7.0f,
-                                    2.0f / 9.0f, 2.0f / 11.0f, 2.0f / 13.0f, 2.0f / 15.0f};
+// 1 / (k + 1/2), k = 0..15 (only an estimate's accuracy is needed).
+__constant__ float c_inv_half[16] = {2.0f,         2.0f / 3.0f,  2.0f / 5.0f,  2.0f / 7.0f,  2.0f / 9.0f,  2.0f / 11.0f,
+                                     2.0f / 13.0f, 2.0f / 15.0f, 2.0f / 17.0f, 2.0f / 19.0f, 2.0f / 21.0f, 2.0f / 23.0f,
+                                     2.0f / 25.0f, 2.0f / 27.0f, 2.0f / 29.0f, 2.0f / 31.0f};
 
 // Smallest grid index j in [1, kBeyond] with |q(s_j)| <= k, kBeyond meaning
 // "still above k at 65504".  The fp32 estimate |w|/(k+1/2) rounded up to
@@ -730,14 +731,15 @@ __device__ __forceinline__ void enqueue(const Params &p, int64_t g, int lane, Ta
     tl.fallback++;
 }
 
-// Key layout: t (grid index of the transition) << 10 | r (rank of the weight
-// in ascending |w|) << 3 | k (the transition |q|: k+1 -> k).
-template <int E>
+// Key layout: t (grid index of the transition) << (KB + 7) | r (rank of the
+// weight in ascending |w|) << KB | k (the transition |q|: k+1 -> k), with KB = 3
+// key bits for the layer up to 8 code layers and 4 up to 16.
+template <int E, int KB>
 __device__ __forceinline__ void add_delta32(const WarpSmem<E> &sm, uint32_t kk, float (&RB)[E], float (&RC)[E])
 {
-    const int r = (kk >> 3) & 127;
+    const int r = (kk >> KB) & 127;
     const float aw = fabsf(sm.w[r]);
-    const float c = static_cast<float>(2 * (kk & 7) + 1);
+    const float c = static_cast<float>(2 * (kk & ((1u << KB) - 1u)) + 1);
 #pragma unroll
     for (int e = 0; e < E; e++) {
         const float dd = sm.d[e][r];
@@ -748,12 +750,12 @@ __device__ __forceinline__ void add_delta32(const WarpSmem<E> &sm, uint32_t kk, 
 
 // Exact fp64 coefficient deltas of one transition (products of a 24-bit d with
 // an 11-bit |w| or an odd number <= 15 are exact in fp64).
-template <int E>
+template <int E, int KB>
 __device__ __forceinline__ void add_delta64(const WarpSmem<E> &sm, uint32_t kk, double (&RB)[E], double (&RC)[E])
 {
-    const int r = (kk >> 3) & 127;
+    const int r = (kk >> KB) & 127;
     const double aw = fabsf(sm.w[r]);
-    const double c = static_cast<double>(2 * (kk & 7) + 1);
+    const double c = static_cast<double>(2 * (kk & ((1u << KB) - 1u)) + 1);
 #pragma unroll
     for (int e = 0; e < E; e++) {
         const double dd = sm.d[e][r];
@@ -801,10 +803,13 @@ __device__ __forceinline__ void direct_coefficients(const WarpSmem<E> &sm, float
     }
 }
 
-template <int E, bool kIntersect, bool kSpec, int N>
+template <int E, bool kIntersect, bool kSpec, int N, int kL>
 __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int lane, Tally &tl)
 {
     constexpr int KW = N / 32;  // weights per lane: 4 for groups of 128, 2 for 64
+    // code layers: 8 (|qmin| <= 8) or 16; the layer takes KB bits of a key
+    constexpr int kKB = kL == 16 ? 4 : 3, kTS = kKB + 7;
+    constexpr uint32_t kKM = (1u << kKB) - 1u;
     // Code range: W4 clips at 7 and -8; a general spec (kSpec) at qmax and
     // -nmax, with nmax = qmax or qmax + 1 and at most 8 code layers.  When
     // nmax > qmax the last layer, k = qmax, holds negative weights only.
@@ -1083,24 +1088,6 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     // weights form one rank range [F0_k, F1_k) (layer 7: negative weights, by
     // their rank among negatives).  Transitions above J1 are active on the
     // whole window and only enter the coefficients, in closed form.
-    uint32_t *layer = sm.bufA;
-    if (lane < 16) {
-        const int k = lane & 7;
-        const float sx = (lane < 8) ? sJ0 : sJ1;
-        int lo = 0, hi = N;
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (!code_at_least(fabsf(sm.w[mid]), sx, k + 1))
-                lo = mid + 1;
-            else
-                hi = mid;
-        }
-        const bool empty = k >= QN;  // no code layer k in this range
-        sm.lay[lane] = empty ? 0 : ((negx && k == QP) ? sm.negpre[lo] : lo);  // lanes 0..7: F0_k, 8..15: F1_k
-        sm.lay[16 + lane] = empty ? N : lo;                               // the same as rank thresholds
-    }
-    __syncwarp();
-    const int *off = sm.lay;  // layer k holds ranks [off[k], off[k + 8]) (layer 7: negative ranks)
     float rbf[E], rcf[E];
 #pragma unroll
     for (int e = 0; e < E; e++) {
@@ -1113,45 +1100,225 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         bb[e] = 0.0f;
         bc[e] = 0.0f;
     }
-    int th[16];
+    int T, c;  // in-window transitions, and sorted keys per lane
+    if constexpr (kL == 8) {
+        uint32_t *layer = sm.bufA;
+        if (lane < 16) {
+            const int k = lane & 7;
+            const float sx = (lane < 8) ? sJ0 : sJ1;
+            int lo = 0, hi = N;
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (!code_at_least(fabsf(sm.w[mid]), sx, k + 1))
+                    lo = mid + 1;
+                else
+                    hi = mid;
+            }
+            const bool empty = k >= QN;  // no code layer k in this range
+            sm.lay[lane] = empty ? 0 : ((negx && k == QP) ? sm.negpre[lo] : lo);  // lanes 0..7: F0_k, 8..15: F1_k
+            sm.lay[16 + lane] = empty ? N : lo;                               // the same as rank thresholds
+        }
+        __syncwarp();
+        const int *off = sm.lay;  // layer k holds ranks [off[k], off[k + 8]) (layer 7: negative ranks)
+        int th[16];
 #pragma unroll
-    for (int k = 0; k < 16; k++)
-        th[k] = sm.lay[16 + k];
+        for (int k = 0; k < 16; k++)
+            th[k] = sm.lay[16 + k];
 #pragma unroll 1
-    for (int m = 0; m < KW; m++) {
-        const int r = 32 * m + lane;
-        const float wv = sm.w[r];
-        const float aw = fabsf(wv);
-        // |q| at s_J1: the layers whose rank threshold r has passed
-        int ktop = 0;
+        for (int m = 0; m < KW; m++) {
+            const int r = 32 * m + lane;
+            const float wv = sm.w[r];
+            const float aw = fabsf(wv);
+            // |q| at s_J1: the layers whose rank threshold r has passed
+            int ktop = 0;
 #pragma unroll
-        for (int k = 0; k < 8; k++) {
-            if (k < QP)
-                ktop += r >= th[8 + k];
-            else if (negx && k == QP && wv < 0.0f)
-                ktop += r >= th[8 + k];
-        }
-        const float fk = static_cast<float>(ktop);
+            for (int k = 0; k < 8; k++) {
+                if (k < QP)
+                    ktop += r >= th[8 + k];
+                else if (negx && k == QP && wv < 0.0f)
+                    ktop += r >= th[8 + k];
+            }
+            const float fk = static_cast<float>(ktop);
 #pragma unroll
-        for (int e = 0; e < E; e++) {
-            const float dd = sm.d[e][r];
-            bb[e] = fmaf(dd, aw * fk, bb[e]);
-            bc[e] = fmaf(dd, fk * fk, bc[e]);
+            for (int e = 0; e < E; e++) {
+                const float dd = sm.d[e][r];
+                bb[e] = fmaf(dd, aw * fk, bb[e]);
+                bc[e] = fmaf(dd, fk * fk, bc[e]);
+            }
         }
-    }
-    // The in-window transitions, layer after layer, spread evenly over the
-    // lanes: item t of layer k is its (t - pre_k)-th rank in the layer's range.
-    {
-        int pre[9];
+        // The in-window transitions, layer after layer, spread evenly over the
+        // lanes: item t of layer k is its (t - pre_k)-th rank in the layer's range.
+        {
+            int pre[9];
+            pre[0] = 0;
+#pragma unroll
+            for (int k = 0; k < 8; k++)
+                pre[k + 1] = pre[k] + (off[k + 8] - off[k]);
+#pragma unroll 1
+            for (int t = lane; t < pre[8]; t += 32) {
+                int k = 0, base = 0;
+#pragma unroll
+                for (int kk = 1; kk < 8; kk++) {
+                    if (t >= pre[kk]) {
+                        k = kk;
+                        base = pre[kk];
+                    }
+                }
+                const int at = t - base;
+                const int r = (negx && k == QP) ? static_cast<int>(sm.negidx[off[k] + at]) : off[k] + at;
+                const float aw = fabsf(sm.w[r]);
+                layer[k * kLayerStride + at] =
+                    (transition_index(aw, k) << 10) | (static_cast<uint32_t>(r) << 3) | static_cast<uint32_t>(k);
+            }
+        }
+        if (lane < 8)
+            layer[lane * kLayerStride + off[lane + 8] - off[lane]] = kInvalidKey;
+        __syncwarp();
+
+        // ---- 4'. merge the eight layers: 4 x 8 lanes, 2 x 16 lanes, 32 lanes ---
+        // Level 0 merges layer pairs into bufB, level 1 pairs of those into bufA,
+        // level 2 the last pair into bufB with element x of lane L at x*32 + L,
+        // where lane L produces outputs [L*c, L*c + c) and sums their deltas.
+        int na3 = 0, nb3 = 0;
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            na3 += off[k + 8] - off[k];
+            nb3 += off[k + 12] - off[k + 4];
+        }
+        T = na3 + nb3;
+        c = (T + 31) >> 5;
+#pragma unroll 1
+        for (int level = 0; level < 3; level++) {
+            const uint32_t *La, *Lb;
+            int na, nb, d0, d1, obase, ostride;
+            uint32_t *out;
+            if (level == 0) {
+                const int mg = lane >> 3, sl = lane & 7;
+                La = layer + (2 * mg) * kLayerStride;
+                Lb = layer + (2 * mg + 1) * kLayerStride;
+                na = off[2 * mg + 8] - off[2 * mg];
+                nb = off[2 * mg + 9] - off[2 * mg + 1];
+                out = sm.bufB + mg * 260;
+                const int tot = na + nb, ch = (tot + 7) >> 3;
+                d0 = min(sl * ch, tot);
+                d1 = min(sl * ch + ch, tot);
+                if (sl == 0)
+                    out[tot] = kInvalidKey;
+            } else if (level == 1) {
+                const int mg = lane >> 4, sl = lane & 15;
+                La = sm.bufB + (2 * mg) * 260;
+                Lb = sm.bufB + (2 * mg + 1) * 260;
+                na = off[4 * mg + 8] - off[4 * mg] + off[4 * mg + 9] - off[4 * mg + 1];
+                nb = off[4 * mg + 10] - off[4 * mg + 2] + off[4 * mg + 11] - off[4 * mg + 3];
+                out = sm.bufA + mg * 520;
+                const int tot = na + nb, ch = (tot + 15) >> 4;
+                d0 = min(sl * ch, tot);
+                d1 = min(sl * ch + ch, tot);
+                if (sl == 0)
+                    out[tot] = kInvalidKey;
+            } else {
+                La = sm.bufA;
+                Lb = sm.bufA + 520;
+                na = na3;
+                nb = nb3;
+                out = sm.bufB;
+                d0 = min(lane * c, T);
+                d1 = min(lane * c + c, T);
+            }
+            obase = (level == 2) ? lane - 32 * d0 : 0;
+            ostride = (level == 2) ? 32 : 1;
+            if (d0 < d1) {
+                int i = merge_split(La, na, Lb, nb, d0);
+                int j = d0 - i;
+                uint32_t va = La[i], vb = Lb[j];
+                for (int o = d0; o < d1; o++) {
+                    const bool ta = va < vb;
+                    const uint32_t kk = ta ? va : vb;
+                    if (ta)
+                        va = La[++i];
+                    else
+                        vb = Lb[++j];
+                    out[obase + o * ostride] = kk;
+                    if (level == 2)
+                        add_delta32<E, kKB>(sm, kk, rbf, rcf);
+                }
+            }
+            if (level == 2)
+                for (int x = d1 - d0; x < c; x++)
+                    sm.bufB[x * 32 + lane] = kInvalidKey;
+            __syncwarp();
+        }
+    } else {
+        // Up to sixteen code layers (|qmin| <= 16, group size 128): the layer
+        // bounds take all 32 lanes (F0_k on lanes 0..15, F1_k on 16..31); the
+        // layers' lists sit back to back in bufB (list k at pre[k] + k, its sentinel
+        // after it), since 16 strided lists would not fit; a four-level merge network
+        // (8 merges of 4 lanes, 4 of 8, 2 of 16, 1 of 32) sorts them, ping-ponging
+        // bufB -> bufA -> bufB -> bufA -> bufB.  A window holding more than 1,024
+        // transitions goes to the exhaustive pass.
+        uint32_t *layer = sm.bufB;  // the window's prefix sums there are no longer read
+        {
+            const int k = lane & 15;
+            const float sx = (lane < 16) ? sJ0 : sJ1;
+            int lo = 0, hi = N;
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (!code_at_least(fabsf(sm.w[mid]), sx, k + 1))
+                    lo = mid + 1;
+                else
+                    hi = mid;
+            }
+            const bool empty = k >= QN;
+            const bool neglayer = negx && k == QP;
+            sm.lay[lane] = empty ? 0 : (neglayer ? sm.negpre[lo] : lo);
+            if (neglayer && lane >= 16)
+                sm.negpre[N + 2] = static_cast<uint8_t>(lo);  // the negative layer's rank threshold at s_J1
+        }
+        __syncwarp();
+        const int *off = sm.lay;  // layer k holds ranks [off[k], off[16 + k]) (the negative layer: negative ranks)
+        const int negthr = sm.negpre[N + 2];
+#pragma unroll 1
+        for (int m = 0; m < KW; m++) {
+            const int r = 32 * m + lane;
+            const float wv = sm.w[r];
+            const float aw = fabsf(wv);
+            int ktop = 0;  // |q| at s_J1: the layers whose rank threshold r has passed
+#pragma unroll
+            for (int k = 0; k < 16; k++) {
+                if (k < QP)
+                    ktop += r >= off[16 + k];
+                else if (negx && k == QP && wv < 0.0f)
+                    ktop += r >= negthr;
+            }
+            const float fk = static_cast<float>(ktop);
+#pragma unroll
+            for (int e = 0; e < E; e++) {
+                const float dd = sm.d[e][r];
+                bb[e] = fmaf(dd, aw * fk, bb[e]);
+                bc[e] = fmaf(dd, fk * fk, bc[e]);
+            }
+        }
+        int pre[17];
         pre[0] = 0;
 #pragma unroll
-        for (int k = 0; k < 8; k++)
-            pre[k + 1] = pre[k] + (off[k + 8] - off[k]);
+        for (int k = 0; k < 16; k++)
+            pre[k + 1] = pre[k] + (off[16 + k] - off[k]);
+        T = pre[16];
+        if (T > 1024) {
+            enqueue(p, g, lane, tl, J0, J1);
+            return;
+        }
+        c = (T + 31) >> 5;
+        int pre_lane = 0;  // pre[lane] for lanes 0..16, read by shuffles in the merge levels
+#pragma unroll
+        for (int k = 0; k <= 16; k++)
+            if (lane == k)
+                pre_lane = pre[k];
 #pragma unroll 1
-        for (int t = lane; t < pre[8]; t += 32) {
+        for (int t = lane; t < T; t += 32) {
             int k = 0, base = 0;
 #pragma unroll
-            for (int kk = 1; kk < 8; kk++) {
+            for (int kk = 1; kk < 16; kk++) {
                 if (t >= pre[kk]) {
                     k = kk;
                     base = pre[kk];
@@ -1160,86 +1327,64 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
             const int at = t - base;
             const int r = (negx && k == QP) ? static_cast<int>(sm.negidx[off[k] + at]) : off[k] + at;
             const float aw = fabsf(sm.w[r]);
-            layer[k * kLayerStride + at] =
-                (transition_index(aw, k) << 10) | (static_cast<uint32_t>(r) << 3) | static_cast<uint32_t>(k);
+            layer[base + k + at] =
+                (transition_index(aw, k) << kTS) | (static_cast<uint32_t>(r) << kKB) | static_cast<uint32_t>(k);
         }
-    }
-    if (lane < 8)
-        layer[lane * kLayerStride + off[lane + 8] - off[lane]] = kInvalidKey;
-    __syncwarp();
-
-    // ---- 4'. merge the eight layers: 4 x 8 lanes, 2 x 16 lanes, 32 lanes ---
-    // Level 0 merges layer pairs into bufB, level 1 pairs of those into bufA,
-    // level 2 the last pair into bufB with element x of lane L at x*32 + L,
-    // where lane L produces outputs [L*c, L*c + c) and sums their deltas.
-    int na3 = 0, nb3 = 0;
-#pragma unroll
-    for (int k = 0; k < 4; k++) {
-        na3 += off[k + 8] - off[k];
-        nb3 += off[k + 12] - off[k + 4];
-    }
-    const int T = na3 + nb3;
-    const int c = (T + 31) >> 5;
-#pragma unroll 1
-    for (int level = 0; level < 3; level++) {
-        const uint32_t *La, *Lb;
-        int na, nb, d0, d1, obase, ostride;
-        uint32_t *out;
-        if (level == 0) {
-            const int mg = lane >> 3, sl = lane & 7;
-            La = layer + (2 * mg) * kLayerStride;
-            Lb = layer + (2 * mg + 1) * kLayerStride;
-            na = off[2 * mg + 8] - off[2 * mg];
-            nb = off[2 * mg + 9] - off[2 * mg + 1];
-            out = sm.bufB + mg * 260;
-            const int tot = na + nb, ch = (tot + 7) >> 3;
-            d0 = min(sl * ch, tot);
-            d1 = min(sl * ch + ch, tot);
-            if (sl == 0)
-                out[tot] = kInvalidKey;
-        } else if (level == 1) {
-            const int mg = lane >> 4, sl = lane & 15;
-            La = sm.bufB + (2 * mg) * 260;
-            Lb = sm.bufB + (2 * mg + 1) * 260;
-            na = off[4 * mg + 8] - off[4 * mg] + off[4 * mg + 9] - off[4 * mg + 1];
-            nb = off[4 * mg + 10] - off[4 * mg + 2] + off[4 * mg + 11] - off[4 * mg + 3];
-            out = sm.bufA + mg * 520;
-            const int tot = na + nb, ch = (tot + 15) >> 4;
-            d0 = min(sl * ch, tot);
-            d1 = min(sl * ch + ch, tot);
-            if (sl == 0)
-                out[tot] = kInvalidKey;
-        } else {
-            La = sm.bufA;
-            Lb = sm.bufA + 520;
-            na = na3;
-            nb = nb3;
-            out = sm.bufB;
-            d0 = min(lane * c, T);
-            d1 = min(lane * c + c, T);
-        }
-        obase = (level == 2) ? lane - 32 * d0 : 0;
-        ostride = (level == 2) ? 32 : 1;
-        if (d0 < d1) {
-            int i = merge_split(La, na, Lb, nb, d0);
-            int j = d0 - i;
-            uint32_t va = La[i], vb = Lb[j];
-            for (int o = d0; o < d1; o++) {
-                const bool ta = va < vb;
-                const uint32_t kk = ta ? va : vb;
-                if (ta)
-                    va = La[++i];
-                else
-                    vb = Lb[++j];
-                out[obase + o * ostride] = kk;
-                if (level == 2)
-                    add_delta32<E>(sm, kk, rbf, rcf);
-            }
-        }
-        if (level == 2)
-            for (int x = d1 - d0; x < c; x++)
-                sm.bufB[x * 32 + lane] = kInvalidKey;
+        const int pre_next = __shfl_down_sync(kFull, pre_lane, 1);  // pre[lane + 1]
+        if (lane < 16)
+            layer[pre_next + lane] = kInvalidKey;  // after list lane: pre[lane] + lane + its size
         __syncwarp();
+        uint32_t *src = sm.bufB, *dst = sm.bufA;
+#pragma unroll 1
+        for (int l = 0; l < 4; l++) {
+            const int lps = 2 + l;  // log2 of the lanes per merge
+            const int mg = lane >> lps, sl = lane & ((1 << lps) - 1), span = 1 << l;
+            const int la0 = 2 * mg * span;
+            const int pa = __shfl_sync(kFull, pre_lane, la0);
+            const int pb = __shfl_sync(kFull, pre_lane, la0 + span);
+            const int pe = __shfl_sync(kFull, pre_lane, la0 + 2 * span);
+            const int na = pb - pa, nb = pe - pb;
+            const uint32_t *La = src + pa + 2 * mg, *Lb = src + pb + 2 * mg + 1;
+            const bool last = l == 3;
+            int d0, d1, obase = 0;
+            if (last) {
+                d0 = min(lane * c, T);
+                d1 = min(lane * c + c, T);
+            } else {
+                const int tot = na + nb, ch = (tot + (1 << lps) - 1) >> lps;
+                d0 = min(sl * ch, tot);
+                d1 = min(sl * ch + ch, tot);
+                obase = pa + mg;
+                if (sl == 0)
+                    dst[obase + tot] = kInvalidKey;
+            }
+            if (d0 < d1) {
+                int i = merge_split(La, na, Lb, nb, d0);
+                int j = d0 - i;
+                uint32_t va = La[i], vb = Lb[j];
+                for (int o = d0; o < d1; o++) {
+                    const bool ta = va < vb;
+                    const uint32_t kk = ta ? va : vb;
+                    if (ta)
+                        va = La[++i];
+                    else
+                        vb = Lb[++j];
+                    if (last) {
+                        sm.bufB[(o - d0) * 32 + lane] = kk;
+                        add_delta32<E, kKB>(sm, kk, rbf, rcf);
+                    } else {
+                        dst[obase + o] = kk;
+                    }
+                }
+            }
+            if (last)
+                for (int x = d1 - d0; x < c; x++)
+                    sm.bufB[x * 32 + lane] = kInvalidKey;
+            __syncwarp();
+            uint32_t *tmp = src;
+            src = dst;
+            dst = tmp;
+        }
     }
     const uint32_t *keys = sm.bufB;
 
@@ -1266,7 +1411,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     {
         const uint32_t kn = (lane < 31 && c > 0) ? keys[lane + 1] : kInvalidKey;
         if (kn != kInvalidKey)
-            t_after = kn >> 10;
+            t_after = kn >> kTS;
     }
 
     // ---- 6. fp32 screen of every run in the window --------------------------
@@ -1287,7 +1432,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     for (int x = c - 1; x >= -1; --x) {
         const uint32_t kk = (x >= 0) ? keys[x * 32 + lane] : kInvalidKey;
         const bool valid = kk != kInvalidKey;
-        const uint32_t t = valid ? (kk >> 10) : ((x >= 0 || lane != 0) ? jend : J0);
+        const uint32_t t = valid ? (kk >> kTS) : ((x >= 0 || lane != 0) ? jend : J0);
         const bool run = t <= J1 && t != next_t;
         const uint32_t ja = run ? t : J0;
         const uint32_t jb = run ? min(next_t, jend) - 1u : J0;
@@ -1299,9 +1444,9 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
         // A padding key adds d * 0 at the rank its bits decode to, 127: staged
         // and finite in a 128-weight group, but past a 64-weight one, so there
         // rank 0 stands in.
-        const int r = (N == 128 || valid) ? static_cast<int>((kk >> 3) & 127) : 0;
+        const int r = (N == 128 || valid) ? static_cast<int>((kk >> kKB) & 127) : 0;
         const float aw = valid ? fabsf(sm.w[r]) : 0.0f;
-        const float cc = valid ? static_cast<float>(2 * (kk & 7) + 1) : 0.0f;
+        const float cc = valid ? static_cast<float>(2 * (kk & kKM) + 1) : 0.0f;
 #pragma unroll
         for (int e = 0; e < E; e++) {
             const float dd = sm.d[e][r];
@@ -1364,7 +1509,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
             const uint32_t kk = keys[x * 32 + lane];
             if (kk == kInvalidKey)
                 continue;
-            const uint32_t t = kk >> 10;
+            const uint32_t t = kk >> kTS;
             if ((smask >> x) & 1u)
                 ent[rk++] = SurvEntry{t, min(nt, jend) - 1u, lane * c + x, 0};
             nt = t;
@@ -1395,7 +1540,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
                 int lp = cur / c, x = cur - lp * c;
 #pragma unroll 1
                 for (int q = cur; q > en.pos; --q) {
-                    add_delta64<E>(sm, keys[x * 32 + lp], Bc, Cc);
+                    add_delta64<E, kKB>(sm, keys[x * 32 + lp], Bc, Cc);
                     if (--x < 0) {
                         x = c - 1;
                         --lp;
@@ -1730,7 +1875,7 @@ __device__ void process_group(const Params &p, WarpSmem<E> &sm, int64_t g, int l
     tl.finalists += static_cast<uint32_t>(total);
 }
 
-template <int E, bool kIntersect, bool kSpec, int N>
+template <int E, bool kIntersect, bool kSpec, int N, int kL>
 __global__ void __launch_bounds__(kWarpsPerCta<E> * 32, 1) select_kernel(Params p)
 {
     constexpr int kWarps = kWarpsPerCta<E>;
@@ -1746,7 +1891,7 @@ __global__ void __launch_bounds__(kWarpsPerCta<E> * 32, 1) select_kernel(Params 
         if (g < p.G) {
             if (lane < N / 64 && g + stride < p.G)
                 asm volatile("prefetch.global.L2 [%0];" ::"l"(p.W + (g + stride) * N + 64 * lane));
-            process_group<E, kIntersect, kSpec, N>(p, sm, g, lane, tl);
+            process_group<E, kIntersect, kSpec, N, kL>(p, sm, g, lane, tl);
         }
         __syncthreads();  // the warps start the next group together
     }
@@ -1951,17 +2096,17 @@ cudaError_t pool_alloc(void **ptr, size_t bytes, cudaStream_t st)
     return cudaMallocFromPoolAsync(ptr, bytes, g_pool[dev], st);
 }
 
-template <int E, bool kIntersect, bool kSpec, int N>
+template <int E, bool kIntersect, bool kSpec, int N, int kL = 8>
 cudaError_t launch_main(const Params &p, cudaStream_t st, int sms)
 {
     constexpr int kWarps = kWarpsPerCta<E>;
     const size_t smem = sizeof(WarpSmem<E>) * kWarps;
-    cudaError_t err = cudaFuncSetAttribute(select_kernel<E, kIntersect, kSpec, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t err = cudaFuncSetAttribute(select_kernel<E, kIntersect, kSpec, N, kL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
     if (err != cudaSuccess)
         return err;
     int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel<E, kIntersect, kSpec, N>, kWarps * 32, smem);
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel<E, kIntersect, kSpec, N, kL>, kWarps * 32, smem);
     if (err != cudaSuccess)
         return err;
     if (per_sm < 1)
@@ -1970,7 +2115,7 @@ cudaError_t launch_main(const Params &p, cudaStream_t st, int sms)
     const int64_t grid = need < static_cast<int64_t>(sms) * per_sm ? need : static_cast<int64_t>(sms) * per_sm;
     if (p.ev_begin && (err = cudaEventRecord(p.ev_begin, st)) != cudaSuccess)
         return err;
-    select_kernel<E, kIntersect, kSpec, N><<<static_cast<unsigned>(grid), kWarps * 32, smem, st>>>(p);
+    select_kernel<E, kIntersect, kSpec, N, kL><<<static_cast<unsigned>(grid), kWarps * 32, smem, st>>>(p);
     err = cudaGetLastError();
     if (err != cudaSuccess)
         return err;
@@ -1993,7 +2138,9 @@ cudaError_t launch(const Params &p, cudaStream_t st)
                 return err;
             exhaustive_kernel<E, true, 64><<<static_cast<unsigned>(2 * sms), kExThreads, 0, st>>>(p);
         } else {
-            if ((err = launch_main<E, false, true, 128>(p, st, sms)) != cudaSuccess)
+            err = p.nmax > 8 ? launch_main<E, false, true, 128, 16>(p, st, sms)
+                             : launch_main<E, false, true, 128>(p, st, sms);
+            if (err != cudaSuccess)
                 return err;
             exhaustive_kernel<E, true, 128><<<static_cast<unsigned>(2 * sms), kExThreads, 0, st>>>(p);
         }
@@ -2092,7 +2239,8 @@ cq_status select_spec_fast(const uint16_t *W, int64_t G, const float *D, int E, 
                            cudaStream_t st)
 {
     const int nmax = -qmin;
-    if (!(qmax >= 1 && nmax <= 8 && (nmax == qmax || nmax == qmax + 1)) || (n != kGroup && n != 64))
+    if (!(qmax >= 1 && (nmax == qmax || nmax == qmax + 1)) || (n != kGroup && n != 64) ||
+        nmax > (n == kGroup ? 16 : 8))
         return CQ_ERR_UNSUPPORTED;
     if (!aligned(W, 16) || !aligned(D, 16) || !aligned(out_q, 4) || !aligned(out_scales, 2) ||
         (out_obj && !aligned(out_obj, 8)))

@@ -109,8 +109,9 @@ def _run_kernel(W, D, qmin, qmax, n, K, general):
             r.flags.cpu().numpy())
 
 
-@pytest.mark.parametrize("n", [128, 64])
-@pytest.mark.parametrize("spec", [(-8, 7), (-4, 3), (-2, 1), (-1, 1), (-8, 8), (-5, 4)])
+@pytest.mark.parametrize("n,spec", [(n, sp) for n in (128, 64)
+                                     for sp in ((-8, 7), (-4, 3), (-2, 1), (-1, 1), (-8, 8), (-5, 4))] +
+                         [(128, sp) for sp in ((-16, 15), (-16, 16), (-12, 11), (-9, 8))])
 def test_w4_search_and_general_kernel_same_bytes(spec, n):
     """Group size 128 or 64 with |qmin| = qmax or qmax + 1 runs the W4
     kernel's search; the general kernel is the other implementation of the
@@ -141,8 +142,19 @@ def test_w4_search_each_environment_count(E):
     for n in (128, 64):
         W = _groups(160, n, seed=200 + E)
         D = _diag(E, 160, n, seed=300 + E, sigma=2.0)
-        for qmin, qmax in ((-4, 3), (-2, 1), (-8, 8), (-8, 7)):
+        specs = ((-4, 3), (-2, 1), (-8, 8), (-8, 7)) + (((-16, 15), (-16, 16)) if n == 128 else ())
+        for qmin, qmax in specs:
             _check(W, D, qmin, qmax, n, where=f"E={E} n={n} spec ({qmin}, {qmax})")
+
+
+def test_w4_search_sixteen_layers_stress():
+    """Code ranges of 16 layers at group size 128 (their own merge network) on
+    the tie/stress workload's classes, with E = 8."""
+    cls = synth.stress_classes()
+    pick = np.sort(np.concatenate([np.nonzero(cls == c)[0][:40] for c in range(5)]))
+    Wg, Dg = synth.group_rows(4, pick)
+    _check(Wg, Dg, -16, 15, 128, where="stress (-16, 15)")
+    _check(Wg, Dg, -12, 11, 128, where="stress (-12, 11)")
 
 
 def test_w4_search_group64_stress_and_edges():
