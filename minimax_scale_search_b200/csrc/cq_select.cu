@@ -1,4 +1,4 @@
-// Exact minimax FP16 group-scale selection (W4, group 128) for sm_100a.
+// Exact minimax FP16 group-scale selection (W4, group 128; and general specs) for sm_100a.
 //
 // Operation (CliffQuant project page, "What CliffQuant changes"): for every
 // group of 128 weights w_i and E environment diagonals d_{e,i}, pick the
@@ -49,6 +49,20 @@
 //     forced or out of range) in the definition's own fp64 evaluation order by
 //     a second kernel, one CTA per group.
 // 10. Pack: each lane packs 4 codes; pairs of lanes form one uint32.
+//
+// The same search serves three more cases, as template parameters of
+// select_kernel<E, kIntersect, kSpec, N, kL> (the W4 default is
+// <E, false, false, 128, 8>):
+//  - kIntersect: step 7 takes each surviving run's minimiser from the pairwise
+//    environment intersections (candidates "induced by ... environment
+//    intersections") before any binary search; same output, off by default.
+//  - kSpec: a general code range [-nmax, qmax] with nmax = qmax or qmax + 1
+//    (cq_select_scales_spec): the caps come from the spec, the finalists are
+//    rescored in the definition's order so objectives and choices are the
+//    oracle's bit for bit, and the codes are written as int8.
+//  - N (128 or 64 weights per group, N/32 per lane) and kL (8 or 16 code
+//    layers; 16 uses a 4-bit layer field in the keys, back-to-back layer
+//    lists and a four-level merge network).
 
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>

@@ -81,3 +81,13 @@ def test_traffic_records_parse_and_match_their_summaries():
         assert os.path.exists(os.path.join(os.path.dirname(prof), "minimax_scale_search_b200", "csrc", rec["src"]))
         names.add(rec["kernel"])
     assert {"absmax_kernel", "objective_kernel<4,", "spec_kernel<4>"} <= names
+
+
+def test_spec_routing_matches_the_header():
+    """bench.py labels a spec line with the kernel cq_select_scales_spec picks:
+    the W4 search for qmin = -qmax or -qmax - 1, up to 16 layers at group size
+    128 and 8 at 64, else the general kernel."""
+    w4 = [(-8, 7, 128), (-4, 3, 128), (-1, 1, 128), (-16, 15, 128), (-16, 16, 128), (-8, 7, 64), (-8, 8, 64)]
+    general = [(-17, 16, 128), (-16, 15, 64), (-3, 5, 128), (-8, 6, 128), (-8, 7, 256), (-8, 7, 100), (-1, 0, 128)]
+    assert all(bench.spec_uses_w4_search(*c) for c in w4)
+    assert not any(bench.spec_uses_w4_search(*c) for c in general)
