@@ -442,11 +442,11 @@ def bench_gptq(args, wl, dev):
     ms = time_calls(lambda: cq.gptq_export(S, C, R, K), args.steps, args.warmup, stream)
     bpg = 64 + 2 + 64 + 2 + 0.5  # codes and scales in, qweight, scales and qzeros out
     lines.append(dict(base, metric="GPTQ v1 export groups/sec", op="gptq_export", value=G / ms * 1e3,
-                      ms_per_step=ms, gpu_launches=3 * args.steps,
+                      ms_per_step=ms, gpu_launches=args.steps,
                       roofline={"bound": "hbm", "achieved": G * bpg / ms / 1e6, "peak": hbm, "unit": "GB/s",
                                 "frac": G * bpg / ms / 1e6 / hbm,
-                                "traffic": recorded_kernel_traffic("transpose_kernel<uint32_t>", G),
-                                "kernel": "transpose_kernel<uint32_t> (+ scales transpose, fills)",
+                                "traffic": recorded_kernel_traffic("export_kernel", G),
+                                "kernel": "export_kernel (word and scale transposes, fills)",
                                 "bytes_per_group": bpg, "peak_note": hsrc}))
     for half in (True, False):
         out = torch.empty((R, K), dtype=torch.float16 if half else torch.float32, device=dev)

@@ -204,7 +204,9 @@ cq_status cq_reconstruction_proxy(const double *per_env, int64_t G, int E, int64
  * pointers are device pointers with their element's alignment. */
 
 /* Export: from the selection's scales [R*K/128] and packed codes [R*K/128][16]
- * (group r*(K/128) + c is row r, columns 128c..128c+127) to the four tensors. */
+ * (group r*(K/128) + c is row r, columns 128c..128c+127) to the four tensors.
+ * One launch when codes and qweight are 16-byte aligned; three (the same
+ * bytes) when either is only 4-byte aligned. */
 cq_status cq_gptq_export(const uint16_t *scales, const uint32_t *codes, int64_t R, int64_t K,
                          int32_t *qweight, int32_t *qzeros, uint16_t *gptq_scales, int32_t *g_idx,
                          void *stream);

@@ -13,9 +13,10 @@
 // The selection's codes of group (r, c) are 16 words of 8 input-adjacent
 // nibbles (q + 8), low nibble first: word j of group (r, c) is exactly
 // qweight[16c + j][r].  So the export is a transpose of the [R][K/8] word
-// matrix, a transpose of the [R][K/128] scale matrix and two constant fills;
-// all are HBM-bound; the transposes run as 64 x 64 tiles through shared memory
-// (reads and writes both coalesced, 256-byte runs), the dequantiser as 32 x 32.
+// matrix, a transpose of the [R][K/128] scale matrix and two constant fills,
+// all HBM-bound and done by one launch: the transposes run as 64 x 64 tiles
+// through shared memory (reads and writes both coalesced, 256-byte runs; the
+// words with 16-byte accesses), the dequantiser as 32 x 32.
 
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -36,7 +37,9 @@ constexpr int kBigRows = 4;          // CTA of 64 x 4 threads, 16 elements per t
 
 // dst[c][r] = src[r][c] for an [rows][cols] matrix, one 64 x 64 tile per CTA
 // iteration (grid-stride over tiles): every row segment read and written is
-// 64 elements long, and a thread has 16 loads in flight.
+// 64 elements long, and a thread has 16 loads in flight.  The export takes
+// this path (three launches) only when the code words or qweight are not
+// 16-byte aligned.
 template <typename T>
 __global__ void __launch_bounds__(kBigTile * kBigRows) transpose_kernel(const T *__restrict__ src, int64_t rows,
                                                                        int64_t cols, T *__restrict__ dst)
@@ -61,6 +64,83 @@ __global__ void __launch_bounds__(kBigTile * kBigRows) transpose_kernel(const T 
             if (r < rows && c < cols)
                 dst[c * rows + r] = tile[tx][ty + k];
         }
+    }
+}
+
+// The whole export in one launch.  CTA iterations [0, tw) transpose 64 x 64
+// tiles of code words with 16-byte loads and stores (4 per thread per tile);
+// [tw, tw + ts) transpose 64 x 64 tiles of scales; then every thread joins a
+// grid-stride fill of qzeros and g_idx.  R % 8 == 0 and K8 % 16 == 0 keep every
+// 16-byte access inside its row.
+constexpr int kExportThreads = 256;
+
+__global__ void __launch_bounds__(kExportThreads) export_kernel(const uint32_t *__restrict__ codes,
+                                                                const uint16_t *__restrict__ scales, int64_t R,
+                                                                int64_t K, uint32_t *__restrict__ qweight,
+                                                                uint16_t *__restrict__ gscales,
+                                                                int32_t *__restrict__ qzeros, int32_t *__restrict__ g_idx)
+{
+    __shared__ uint32_t tile[kBigTile][kBigTile + 1];
+    const int64_t K8 = K / 8, ng = K / 128;
+    const int64_t tr = (R + kBigTile - 1) / kBigTile;
+    const int64_t twc = (K8 + kBigTile - 1) / kBigTile, tsc = (ng + kBigTile - 1) / kBigTile;
+    const int64_t tw = tr * twc, ts = tr * tsc;
+    const int tid = threadIdx.x;
+    for (int64_t t = blockIdx.x; t < tw + ts; t += gridDim.x) {
+        __syncthreads();
+        if (t < tw) {
+            const int64_t r0 = (t / twc) * kBigTile, c0 = (t % twc) * kBigTile;
+            uint4 v[4];
+#pragma unroll
+            for (int k = 0; k < 4; k++) {
+                const int i = tid + kExportThreads * k, r = i >> 4, c4 = i & 15;
+                const int64_t gr = r0 + r, gc = c0 + 4 * c4;
+                v[k] = (gr < R && gc < K8) ? __ldcs(reinterpret_cast<const uint4 *>(codes + gr * K8 + gc))
+                                           : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; k++) {
+                const int i = tid + kExportThreads * k, r = i >> 4, c4 = i & 15;
+                tile[r][4 * c4] = v[k].x;
+                tile[r][4 * c4 + 1] = v[k].y;
+                tile[r][4 * c4 + 2] = v[k].z;
+                tile[r][4 * c4 + 3] = v[k].w;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int k = 0; k < 4; k++) {
+                const int i = tid + kExportThreads * k, c = i >> 4, r4 = i & 15;
+                const int64_t gc = c0 + c, gr = r0 + 4 * r4;
+                if (gc < K8 && gr < R)
+                    *reinterpret_cast<uint4 *>(qweight + gc * R + gr) =
+                        make_uint4(tile[4 * r4][c], tile[4 * r4 + 1][c], tile[4 * r4 + 2][c], tile[4 * r4 + 3][c]);
+            }
+        } else {
+            const int64_t u = t - tw;
+            const int64_t r0 = (u / tsc) * kBigTile, c0 = (u % tsc) * kBigTile;
+            const int tx = tid & 63, ty = tid >> 6;
+#pragma unroll
+            for (int k = 0; k < kBigTile; k += 4) {
+                const int64_t r = r0 + ty + k, c = c0 + tx;
+                if (r < R && c < ng)
+                    tile[ty + k][tx] = scales[r * ng + c];
+            }
+            __syncthreads();
+#pragma unroll
+            for (int k = 0; k < kBigTile; k += 4) {
+                const int64_t c = c0 + ty + k, r = r0 + tx;
+                if (r < R && c < ng)
+                    gscales[c * R + r] = static_cast<uint16_t>(tile[tx][ty + k]);
+            }
+        }
+    }
+    const int64_t nz = ng * (R / 8);
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * kExportThreads;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * kExportThreads + tid; i < nz + K; i += stride) {
+        if (i < nz)
+            qzeros[i] = 0x77777777;
+        else
+            g_idx[i - nz] = static_cast<int32_t>((i - nz) / 128);
     }
 }
 
@@ -224,8 +304,15 @@ cq_status cq_gptq_export(const uint16_t *scales, const uint32_t *codes, int64_t 
         !aligned(g_idx, 4))
         return CQ_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const dim3 block(kBigTile, kBigRows);
     const int64_t K8 = K / 8, ng = K / 128;
+    if (aligned(codes, 16) && aligned(qweight, 16)) {
+        const int64_t tiles = ((R + 63) / 64) * ((K8 + 63) / 64 + (ng + 63) / 64);
+        export_kernel<<<tile_grid(tiles), kExportThreads, 0, s>>>(codes, scales, R, K,
+                                                                  reinterpret_cast<uint32_t *>(qweight),
+                                                                  gptq_scales, qzeros, g_idx);
+        return cudaGetLastError() == cudaSuccess ? CQ_OK : CQ_ERR_CUDA;
+    }
+    const dim3 block(kBigTile, kBigRows);
     transpose_kernel<uint32_t><<<tile_grid(((R + 63) / 64) * ((K8 + 63) / 64)), block, 0, s>>>(
         codes, R, K8, reinterpret_cast<uint32_t *>(qweight));
     if (cudaGetLastError() != cudaSuccess)

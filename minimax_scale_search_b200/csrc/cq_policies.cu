@@ -50,6 +50,24 @@ __device__ __forceinline__ void stage_rows(uint8_t *sm, const uint16_t *__restri
     }
 }
 
+// stage_rows with asynchronous copies (global -> shared, bypassing L1): all 16
+// of a lane's 16-byte copies in flight at once and no registers held; rows
+// r >= n are zero-filled (source size 0).
+template <typename RowOf>
+__device__ __forceinline__ void stage_rows_async(uint8_t *sm, const uint16_t *__restrict__ W, int n, int lane,
+                                                 RowOf row_of)
+{
+#pragma unroll
+    for (int k = 0; k < 16; k++) {
+        const int c = k * 32 + lane, r = c >> 4;
+        const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(sm + r * kRowPitch + (c & 15) * 16));
+        const uint16_t *src = (r < n) ? W + row_of(r) * kGroup + (c & 15) * 8 : W;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(r < n ? 16 : 0)
+                     : "memory");
+    }
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 // min(round-half-even(aw / s), cap) for aw >= 0, exact.  The estimate
 // aw * (1/s) is within one of the answer; adding 1.5 * 2^23 rounds it to the
 // nearest integer (ties even) in the low mantissa bits.  Near a half-integer
@@ -181,12 +199,17 @@ __global__ void __launch_bounds__(kStageWarps * 32, kStageCtas) absmax_kernel(co
         const int64_t g0 = t * 32;
         const int n = static_cast<int>(min(static_cast<int64_t>(32), G - g0));
         __syncwarp();
-        stage_rows(sm, W, n, lane, [g0](int r) { return g0 + r; });
-        {
-            // the warp's next chunk into L2 while this one is computed
-            const int64_t gn = g0 + static_cast<int64_t>(gridDim.x) * kStageWarps * 32;
-            if (gn + 32 <= G)
-                asm volatile("prefetch.global.L2 [%0];" ::"l"(W + gn * kGroup + 64 * lane));
+        stage_rows_async(sm, W, n, lane, [g0](int r) { return g0 + r; });
+        if (lane == 0) {
+            // the warp's chunk two strides ahead into L2 (on the first pass the next one too),
+            // one 8 KB bulk prefetch each, while this one is computed
+            const int64_t step = static_cast<int64_t>(gridDim.x) * kStageWarps * 32;
+            if (g0 + 2 * step + 32 <= G)
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], 8192;" ::"l"(W + (g0 + 2 * step) * kGroup)
+                             : "memory");
+            if (g0 < step && g0 + step + 32 <= G)
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], 8192;" ::"l"(W + (g0 + step) * kGroup)
+                             : "memory");
         }
         __syncwarp();
         if (lane < n) {

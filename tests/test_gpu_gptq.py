@@ -37,6 +37,26 @@ def test_export_bit_exact(R, K):
     assert np.array_equal(t.g_idx.cpu().numpy(), gi)
 
 
+@pytest.mark.parametrize("R,K", [(40, 384), (264, 1024)])
+def test_export_unaligned_words_take_the_three_launch_path(R, K):
+    """Code words that start 4 bytes past a 16-byte boundary: the export runs
+    its scalar transposes, with the same bytes as the oracle."""
+    import torch
+    from minimax_scale_search_b200 import cq
+    G = R * K // 128
+    scales, codes = synth.make_codes(G, seed=R + 3 * K)
+    buf = torch.zeros(G * 16 + 1, dtype=torch.int32, device="cuda")
+    buf[1:] = _cuda(codes).reshape(-1)
+    words = buf[1:].view(G, 16)
+    assert words.data_ptr() % 16 == 4
+    t = cq.gptq_export(_cuda(scales), words, R, K)
+    qw, qz, gs, gi = OQ.export_v1(scales, codes, R, K)
+    assert np.array_equal(_bits(t.qweight, np.uint32), qw.view(np.uint32))
+    assert np.array_equal(_bits(t.qzeros, np.uint32), qz.view(np.uint32))
+    assert np.array_equal(_bits(t.scales, np.uint16), gs)
+    assert np.array_equal(t.g_idx.cpu().numpy(), gi)
+
+
 def test_export_sweep_size_sampled_rows():
     """The sweep's layer shape (30,336 x 16,384): rows sampled in blocks of 8,
     each compared with the oracle's export of just those rows."""
