@@ -227,6 +227,28 @@ __global__ void __launch_bounds__(kTile * kDequantRows) dequant_kernel(const uin
             if (r >= R)
                 continue;
             const uint32_t word = tile[tx][ty + k];
+            if (kHalf && uniform) {
+                const uint16_t sb = scales[g0 * R + r];
+                if ((sb & 0x7C00u) != 0x7C00u) {
+                    // binary16 arithmetic, two values per step: 0x6400 | u is 1024 + u, so
+                    // (1024 + u) - (1024 + z + 1) = u - (z + 1) exactly, and one rounding of
+                    // its product with the scale is the fp32 product (exact) rounded to binary16
+                    const int z1 = static_cast<int>((qzeros[g0 * (R / 8) + r / 8] >> (4 * (r % 8))) & 0xFu) + 1;
+                    const __half2 s2 = __half2half2(__ushort_as_half(sb));
+                    const __half2 zz = __half2half2(__ushort_as_half(static_cast<unsigned short>(0x6400 + z1)));
+                    uint32_t pr[4];
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        const uint32_t x = ((word >> (4 * j)) & 0x000F000Fu) | 0x64006400u;  // values j and j + 4
+                        const __half2 p = __hmul2(__hsub2(*reinterpret_cast<const __half2 *>(&x), zz), s2);
+                        pr[j] = *reinterpret_cast<const uint32_t *>(&p);
+                    }
+                    *reinterpret_cast<uint4 *>(static_cast<__half *>(out) + r * K + 8 * kk) =
+                        make_uint4(__byte_perm(pr[0], pr[1], 0x5410), __byte_perm(pr[2], pr[3], 0x5410),
+                                   __byte_perm(pr[0], pr[1], 0x7632), __byte_perm(pr[2], pr[3], 0x7632));
+                    continue;
+                }
+            }
             float v[8];
             if (uniform) {  // one group for the word's 8 inputs (always so with act-order off)
                 const float s = __half2float(__ushort_as_half(scales[g0 * R + r]));
