@@ -535,11 +535,13 @@ def bench_spec(args, wl, dev):
                                                           general_kernel=general),
                             args.steps, args.warmup, stream)
             ach = (f32 + f64 * p32 / p64) / (ms / 1e3) / 1e12
-            kname = "spec_kernel" if general else f"select_kernel<{wl.E}, false, true, {n}> (W4 search)"
+            layers = 16 if -qmin > 8 else 8
+            kname = "spec_kernel" if general else f"select_kernel<{wl.E}, false, true, {n}, {layers}> (W4 search)"
             if general:
                 traffic = recorded_kernel_traffic("spec_kernel<4>", W.size)
-            else:  # recorded at (-4, 3, 128); the bytes per weight do not depend on the code range
-                traffic = recorded_kernel_traffic("select_kernel<4,false,true>", W.size) if n == 128 else None
+            else:  # recorded at (-4, 3, 128) on the 8-layer kernel; its bytes per weight do not depend on the range
+                traffic = (recorded_kernel_traffic("select_kernel<4,false,true>", W.size)
+                           if n == 128 and layers == 8 else None)
             line = {"metric": "general-spec minimax scale selection groups/sec", "op": "spec",
                     "value": G / ms * 1e3, "unit": "groups/s", "ms_per_step": ms, "n_gpus": 1,
                     "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "dtype": "f64",
