@@ -265,6 +265,22 @@ def oracle_rate(Wg, D, K, groups_target_s: float, seed: int = 5):
     return n / dt, n, dt, threads
 
 
+def oracle_rate_one_thread(Wg, D, K, seconds: float = 3.0, seed: int = 6):
+    """The oracle on one host thread, on a sample of about `seconds` of work;
+    returns groups/s."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    probe = np.sort(rng.choice(Wg.shape[0], size=min(Wg.shape[0], 4), replace=False))
+    t0 = time.perf_counter()
+    oracle.solve(Wg, D, K=K, sel=probe, threads=1)
+    per = (time.perf_counter() - t0) / len(probe)
+    n = int(max(len(probe), min(Wg.shape[0], seconds / max(per, 1e-6))))
+    sel = np.sort(rng.choice(Wg.shape[0], size=n, replace=False))
+    t0 = time.perf_counter()
+    oracle.solve(Wg, D, K=K, sel=sel, threads=1)
+    return n / (time.perf_counter() - t0)
+
+
 def run_reference(args, wl):
     """The oracle arm: each step solves a bounded sample on the host cores."""
     rank = int(os.environ.get("RANK", "0"))
@@ -679,6 +695,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, n, dt, threads = oracle_rate(Wg, D, wl.cols, 12.0)
         cpu = {"value": rate, "unit": "groups/s", "cores": threads, "kind": "oracle",
+               "value_one_thread": oracle_rate_one_thread(Wg, D, wl.cols),
                "sample": f"{n} groups sampled from the {wl.name} workload (rank 0's matrix), exhaustive "
                          f"fp64 over 31,743 scales, {dt:.1f} s"}
 
