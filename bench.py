@@ -555,9 +555,11 @@ def bench_spec(args, wl, dev):
             kname = "spec_kernel" if general else f"select_kernel<{wl.E}, false, true, {n}, {layers}> (W4 search)"
             if general:
                 traffic = recorded_kernel_traffic("spec_kernel<4>", W.size)
-            else:  # recorded at (-4, 3, 128) on the 8-layer kernel; its bytes per weight do not depend on the range
-                traffic = (recorded_kernel_traffic("select_kernel<4,false,true>", W.size)
-                           if n == 128 and layers == 8 else None)
+            elif n == 128:  # recorded at (-4, 3) on the 8-layer kernel, (-16, 15) on the 16-layer one
+                traffic = recorded_kernel_traffic(
+                    "select_kernel<4,false,true>" if layers == 8 else "select_kernel<4,false,true,128,16>", W.size)
+            else:
+                traffic = None
             line = {"metric": "general-spec minimax scale selection groups/sec", "op": "spec",
                     "value": G / ms * 1e3, "unit": "groups/s", "ms_per_step": ms, "n_gpus": 1,
                     "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "dtype": "f64",

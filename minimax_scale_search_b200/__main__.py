@@ -1,7 +1,7 @@
 """Command-line runner for synthetic workloads on the GPU.
 
     python -m minimax_scale_search_b200 --workload 2 [--rows R] [--repeat N]
-        [--matrix M] [--force-exhaustive]
+        [--matrix M] [--force-exhaustive] [--intersections]
     python -m minimax_scale_search_b200 --workload 3 --rows 1024 --qmin -4 --qmax 3 [--group-size 128]
     python -m minimax_scale_search_b200 --ops
 
@@ -67,6 +67,8 @@ def main():
     ap.add_argument("--matrix", type=int, default=0)
     ap.add_argument("--repeat", type=int, default=3)
     ap.add_argument("--force-exhaustive", action="store_true")
+    ap.add_argument("--intersections", action="store_true",
+                    help="search surviving runs with the pairwise environment-intersection solver")
     ap.add_argument("--ops", action="store_true", help="run each of the other kernels once")
     ap.add_argument("--qmin", type=int, default=None, help="general spec: smallest code")
     ap.add_argument("--qmax", type=int, default=None, help="general spec: largest code")
@@ -105,7 +107,8 @@ def main():
     times = []
     res = None
     for _ in range(a.repeat):
-        res, t = timed(lambda: cq.select_scales(Wd, Dd, wl.cols, workspace=ws, force_exhaustive=a.force_exhaustive))
+        res, t = timed(lambda: cq.select_scales(Wd, Dd, wl.cols, workspace=ws, force_exhaustive=a.force_exhaustive,
+                                                intersections=a.intersections))
         times.append(t)
     out = {"workload": wl.name, "rows": rows, "groups": G, "E": wl.E, "gen_s": round(gen_s, 2),
            "ms": times, "groups_per_s": G / (min(times) / 1e3), "counters": res.counters()}
