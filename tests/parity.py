@@ -99,3 +99,17 @@ def objective_np(Wg, Dg, scales):
     q = np.clip(np.rint(w / s), -8, 7)
     r2 = (w - s * q) ** 2
     return np.max(np.einsum("egi,gi->eg", Dg.astype(np.float64), r2), axis=0)
+
+
+def seed_range(var: str, default: int):
+    """Seeds of a seeded-case test: range(default), or the range an environment
+    variable names as "N" (0..N-1) or "A:B" (A..B-1), so a larger campaign runs
+    the same committed cases, e.g. CQ_FUZZ_FAST_SEEDS=100:4500."""
+    import os
+    v = os.environ.get(var, "").strip()
+    if not v:
+        return range(default)
+    if ":" in v:
+        a, b = v.split(":", 1)
+        return range(int(a), int(b))
+    return range(int(v))

@@ -6,12 +6,13 @@ only while no fp32 value overflows or falls below the normal range.  These
 cases put the per-environment sums sum d w^2 far above FLT_MAX (d up to
 FLT_MAX, weights up to 65504) and the terms d r^2 below 2^-126 (subnormal and
 tiny d), alone and mixed across environments and weights, so a kernel must
-route such groups to its fp64 path to stay exact."""
+route such groups to its fp64 path to stay exact.  CQ_EXTREME_SEEDS ("N" or
+"A:B") widens the seed range for a longer campaign."""
 import numpy as np
 import pytest
 
 import oracle
-from parity import check_against_oracle, oracle_threads, run_gpu
+from parity import check_against_oracle, oracle_threads, run_gpu, seed_range
 
 pytestmark = pytest.mark.gpu
 
@@ -54,12 +55,28 @@ def extreme_inputs(seed, G=48, E=4):
     return W, D.astype(np.float32)
 
 
-@pytest.mark.parametrize("seed", [0, 1])
+@pytest.mark.parametrize("seed", seed_range("CQ_EXTREME_SEEDS", 2))
 def test_fast_path_extremes(seed):
     W, D = extreme_inputs(4100 + seed)
     assert np.all(np.isfinite(D)) and np.all(D >= 0)
     gpu = run_gpu(W, D)
     check_against_oracle(W, D, gpu, where=f"extremes seed {seed}")
+
+
+@pytest.mark.parametrize("seed", seed_range("CQ_EXTREME_SEEDS", 2))
+def test_general_kernel_extremes_w4_spec(seed):
+    """The general kernel at (-8, 7, 128) on the same extreme inputs, bit-exact."""
+    import torch
+    from minimax_scale_search_b200 import cq
+    W, D = extreme_inputs(4100 + seed)
+    r = cq.select_scales_spec(torch.from_numpy(W.view(np.int16)).cuda(), torch.from_numpy(D).cuda(),
+                              want_objective=True, want_flags=True, general_kernel=True)
+    torch.cuda.synchronize()
+    o = oracle.solve(W, D, threads=oracle_threads())
+    s = r.scales.cpu().numpy().view(np.uint16)
+    bad = np.nonzero(s != o["best_bits"])[0]
+    assert bad.size == 0, (seed, bad[:8])
+    assert np.array_equal(r.codes.cpu().numpy(), o["codes"])
 
 
 @pytest.mark.parametrize("qmin,qmax,n", [(-8, 7, 128), (-4, 3, 128), (-8, 7, 64)])

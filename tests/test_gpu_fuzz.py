@@ -3,12 +3,14 @@ random E (1..8), diagonal layout (per column or per group), group counts that
 are not multiples of the CTA's warps, weight scales from 1e-6 to 1e3, sparse,
 heavy-tailed and exact-multiple weight patterns, lognormal and zero-heavy
 diagonals.  The W4/G128 path follows the selection's parity rule; the
-general-spec path (random code ranges and group sizes) is bit-exact."""
+general-spec path (random code ranges and group sizes) is bit-exact.
+CQ_FUZZ_FAST_SEEDS and CQ_FUZZ_GENERAL_SEEDS ("N" or "A:B") widen the seed
+ranges for a longer campaign."""
 import numpy as np
 import pytest
 
 import oracle
-from parity import check_against_oracle, groups_and_diag, oracle_threads, run_gpu
+from parity import check_against_oracle, groups_and_diag, oracle_threads, run_gpu, seed_range
 
 pytestmark = pytest.mark.gpu
 
@@ -39,7 +41,7 @@ def random_diagonals(rng, E, shape):
     return d.astype(np.float32)
 
 
-@pytest.mark.parametrize("seed", range(12))
+@pytest.mark.parametrize("seed", seed_range("CQ_FUZZ_FAST_SEEDS", 12))
 def test_fast_path_fuzz(seed):
     rng = np.random.default_rng(1000 + seed)
     E = int(rng.integers(1, 9))
@@ -60,7 +62,7 @@ def test_fast_path_fuzz(seed):
     check_against_oracle(Wg, Dg, gpu, where=f"fuzz seed {seed} E={E}")
 
 
-@pytest.mark.parametrize("seed", range(10))
+@pytest.mark.parametrize("seed", seed_range("CQ_FUZZ_GENERAL_SEEDS", 10))
 def test_general_path_fuzz(seed):
     import torch
     from minimax_scale_search_b200 import cq
