@@ -309,7 +309,7 @@ def run_reference(args, wl):
     value = n * len(times) / tot
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "groups/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(times),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
             "config": {"workload": wl.name, "groups_per_step": n, "E": wl.E, "K": wl.cols},
             "cpu_baseline": {"value": value, "unit": "groups/s", "cores": threads, "kind": "oracle",
