@@ -29,8 +29,8 @@ namespace cq {
 namespace {
 
 constexpr int kTile = 32;
-constexpr int kDequantRows = 4;      // dequantisation: CTA of 32 x 4 threads, 8 words per thread, so 16 CTAs
-                                     // (twice the loads in flight) fit per SM
+constexpr int kDequantRows = 4;      // dequantisation: CTA of 32 x 4 threads, 8 words per thread; registers
+                                     // capped so 8 CTAs fit per SM
 
 constexpr int kBigTile = 64;         // transpose tile edge
 constexpr int kBigRows = 4;          // CTA of 64 x 4 threads, 16 elements per thread
@@ -166,7 +166,7 @@ __device__ __forceinline__ int64_t clamp_group(int g, int64_t ngroups)
 // lane writes the 8 values of one word, so a warp stores 256 consecutive
 // values of one output row.  Group indices outside [0, K/128) are clamped.
 template <bool kHalf>
-__global__ void __launch_bounds__(kTile * kDequantRows) dequant_kernel(const uint32_t *__restrict__ qweight,
+__global__ void __launch_bounds__(kTile * kDequantRows, 8) dequant_kernel(const uint32_t *__restrict__ qweight,
                                                                           const uint32_t *__restrict__ qzeros,
                                                                           const uint16_t *__restrict__ scales,
                                                                           const int32_t *__restrict__ g_idx,
@@ -221,6 +221,18 @@ __global__ void __launch_bounds__(kTile * kDequantRows) dequant_kernel(const uin
         for (int j = 1; j < 8; j++)
             uniform = uniform && gi[j] == gi[0];
         const int64_t g0 = clamp_group(gi[0], ngroups);
+        // fp32 output: the word's scale and zero word for each of this thread's rows,
+        // loaded together before the rows (the fp16 output was faster loading them per row)
+        uint16_t sbq[kPer];
+        uint32_t zwq[kPer];
+        if (!kHalf && uniform) {
+#pragma unroll
+            for (int q = 0; q < kPer; q++) {
+                const int64_t r = r0 + ty + q * kDequantRows;
+                sbq[q] = r < R ? scales[g0 * R + r] : static_cast<uint16_t>(0);
+                zwq[q] = r < R ? qzeros[g0 * (R / 8) + r / 8] : 0u;
+            }
+        }
 #pragma unroll
         for (int k = 0; k < kTile; k += kDequantRows) {
             const int64_t r = r0 + ty + k;
@@ -251,8 +263,9 @@ __global__ void __launch_bounds__(kTile * kDequantRows) dequant_kernel(const uin
             }
             float v[8];
             if (uniform) {  // one group for the word's 8 inputs (always so with act-order off)
-                const float s = __half2float(__ushort_as_half(scales[g0 * R + r]));
-                const int z1 = static_cast<int>((qzeros[g0 * (R / 8) + r / 8] >> (4 * (r % 8))) & 0xFu) + 1;
+                const float s = __half2float(__ushort_as_half(kHalf ? scales[g0 * R + r] : sbq[k / kDequantRows]));
+                const int z1 = static_cast<int>(((kHalf ? qzeros[g0 * (R / 8) + r / 8] : zwq[k / kDequantRows]) >>
+                                                 (4 * (r % 8))) & 0xFu) + 1;
 #pragma unroll
                 for (int j = 0; j < 8; j++)
                     v[j] = s * static_cast<float>(static_cast<int>((word >> (4 * j)) & 0xFu) - z1);
